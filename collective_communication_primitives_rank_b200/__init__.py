@@ -1,0 +1,331 @@
+"""Python binding of libcc, the B200 collective-primitives library (C ABI, include/cc.h).
+
+Argument marshalling only: every function here turns torch tensors into the raw device
+pointers, sizes and the current CUDA stream that the C entry point of the same name takes,
+calls it, and raises CCError on a non-OK status. All computation happens in libcc's CUDA
+kernels. There is no CPU path: the first call without a built libcc.so raises, and passing
+a tensor that is not on the current CUDA device raises before any call.
+
+    import collective_communication_primitives_rank_b200 as cc
+    cc.cc_allreduce(send_tensors, recv_tensors, op="sum", algo="ring", scale=1.0)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcc.so")
+
+_LIB = None
+
+CC_OK, CC_ERR_INVALID_ARG, CC_ERR_UNSUPPORTED, CC_ERR_CUDA, CC_ERR_TIMEOUT = range(5)
+CC_F32, CC_BF16, CC_I32 = 0, 1, 2
+CC_SUM, CC_MAX, CC_MIN, CC_PROD = 0, 1, 2, 3
+CC_ALGO_RING, CC_ALGO_TREE = 0, 1
+MAX_RANKS = 64
+
+_vp, _sz, _i, _f = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_float
+_PP = ctypes.POINTER(ctypes.c_void_p)
+_I32P = ctypes.POINTER(ctypes.c_int32)
+_SZP = ctypes.POINTER(ctypes.c_size_t)
+
+_SIGS = {
+    "cc_status_string": (ctypes.c_char_p, [_i]),
+    "cc_version": (_i, []),
+    "cc_chunk": (_i, [_sz, _i, _i, _SZP, _SZP]),
+    "cc_allreduce": (_i, [_PP, _PP, _i, _sz, _i, _i, _i, _i, _f, _vp]),
+    "cc_reduce_scatter": (_i, [_PP, _PP, _i, _sz, _i, _i, _i, _i, _f, _vp]),
+    "cc_allgather": (_i, [_PP, _PP, _i, _sz, _i, _vp]),
+    "cc_broadcast": (_i, [_vp, _PP, _i, _i, _sz, _i, _vp]),
+    "cc_reduce": (_i, [_PP, _vp, _i, _i, _sz, _i, _i, _i, _f, _vp]),
+    "cc_scatter": (_i, [_vp, _PP, _i, _i, _sz, _i, _vp]),
+    "cc_gather": (_i, [_PP, _vp, _i, _i, _sz, _i, _vp]),
+    "cc_route_topk": (_i, [_PP, _PP, _i, _i, _i, _i, _vp]),
+    "cc_alltoallv_workspace_size": (_sz, [_i, _i, _i, _i]),
+    "cc_alltoallv": (_i, [_PP, _PP, _i, _sz, _PP, _i, _i, _i, _sz, _i, _vp, _sz, _vp]),
+    "cc_alltoallv_recv_counts": (_i, [_vp, _i, _vp, _vp]),
+    "cc_bucket_assign": (_i, [_SZP, _i, _sz, _sz, _I32P, _I32P, _I32P]),
+    "cc_bucket_flatten": (_i, [_PP, _SZP, _i, _vp, _i, _vp]),
+    "cc_bucket_unflatten": (_i, [_vp, _PP, _SZP, _i, _i, _vp]),
+    "cc_bucket_allreduce": (_i, [_PP, _PP, _i, _i, _SZP, _sz, _i, _f, _vp]),
+}
+
+
+def get_lib() -> ctypes.CDLL:
+    """Load libcc.so (once) and declare every entry point's signature."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"libcc.so not found at {LIB_PATH}; build it with "
+                "`python -m collective_communication_primitives_rank_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = handle
+    return _LIB
+
+
+class _Lib:
+    def __getattr__(self, name):
+        return getattr(get_lib(), name)
+
+
+lib = _Lib()
+
+
+class CCError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {lib.cc_status_string(status).decode()}")
+
+
+def _check(status: int, where: str) -> None:
+    if status != CC_OK:
+        raise CCError(status, where)
+
+
+_OPS = {"sum": CC_SUM, "max": CC_MAX, "min": CC_MIN, "prod": CC_PROD}
+_ALGOS = {"ring": CC_ALGO_RING, "tree": CC_ALGO_TREE}
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def dtype_code(t) -> int:
+    torch = _torch()
+    m = {torch.float32: CC_F32, torch.bfloat16: CC_BF16, torch.int32: CC_I32}
+    if t.dtype not in m:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    return m[t.dtype]
+
+
+def _dev_ptr(t) -> int:
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError("libcc takes CUDA tensors only")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"tensor on {t.device}, current device is cuda:{torch.cuda.current_device()}")
+    if not t.is_contiguous():
+        raise ValueError("libcc takes contiguous tensors")
+    return t.data_ptr()
+
+
+def _ptrs(tensors: Sequence) -> ctypes.Array:
+    return (ctypes.c_void_p * len(tensors))(*[_dev_ptr(t) for t in tensors])
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return _torch().cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+def _sizes(vals) -> ctypes.Array:
+    return (ctypes.c_size_t * len(vals))(*[int(v) for v in vals])
+
+
+def cc_chunk(count: int, nranks: int, c: int) -> tuple[int, int]:
+    """(start, length) of ring chunk c (the library's chunk rule)."""
+    a, n = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib.cc_chunk(count, nranks, c, ctypes.byref(a), ctypes.byref(n)), "cc_chunk")
+    return a.value, n.value
+
+
+def _same(tensors, numel: int, dtype, what: str) -> None:
+    for t in tensors:
+        if t.numel() != numel or t.dtype != dtype:
+            raise ValueError(f"{what}: every tensor must have {numel} elements of {dtype}")
+
+
+def _ranks(tensors, what: str) -> int:
+    n = len(tensors)
+    if not 1 <= n <= MAX_RANKS:
+        raise ValueError(f"{what}: 1..{MAX_RANKS} ranks, got {n}")
+    return n
+
+
+# ---- collectives -------------------------------------------------------------------------------
+
+def cc_allreduce(send, recv, *, op="sum", algo="ring", scale=1.0, stream=None) -> None:
+    """recv[r] = reduction of send[0..N-1] in `algo`'s fold order, times scale."""
+    n = _ranks(send, "cc_allreduce")
+    _same(send, send[0].numel(), send[0].dtype, "cc_allreduce send")
+    _same(recv, send[0].numel(), recv[0].dtype, "cc_allreduce recv")
+    if len(recv) != n:
+        raise ValueError("cc_allreduce: one output per rank")
+    _check(lib.cc_allreduce(_ptrs(send), _ptrs(recv), n, send[0].numel(), dtype_code(send[0]),
+                            dtype_code(recv[0]), _OPS[op], _ALGOS[algo], float(scale), _stream(stream)),
+           "cc_allreduce")
+
+
+def cc_reduce_scatter(send, recv, *, op="sum", algo="ring", scale=1.0, stream=None) -> None:
+    """recv[c] = chunk c of the ring reduction of send[0..N-1]."""
+    n = _ranks(send, "cc_reduce_scatter")
+    _same(send, send[0].numel(), send[0].dtype, "cc_reduce_scatter send")
+    if len(recv) != n:
+        raise ValueError("cc_reduce_scatter: one output per rank")
+    for c in range(n):
+        _same([recv[c]], cc_chunk(send[0].numel(), n, c)[1], recv[0].dtype, f"cc_reduce_scatter recv[{c}]")
+    _check(lib.cc_reduce_scatter(_ptrs(send), _ptrs(recv), n, send[0].numel(), dtype_code(send[0]),
+                                 dtype_code(recv[0]), _OPS[op], _ALGOS[algo], float(scale), _stream(stream)),
+           "cc_reduce_scatter")
+
+
+def cc_allgather(send, recv, *, stream=None) -> None:
+    """recv[r] = concatenation of send[0..N-1] (send[c] is chunk c of recv's length)."""
+    n = _ranks(send, "cc_allgather")
+    _same(recv, recv[0].numel(), recv[0].dtype, "cc_allgather recv")
+    if len(recv) != n:
+        raise ValueError("cc_allgather: one output per rank")
+    for c in range(n):
+        _same([send[c]], cc_chunk(recv[0].numel(), n, c)[1], recv[0].dtype, f"cc_allgather send[{c}]")
+    _check(lib.cc_allgather(_ptrs(send), _ptrs(recv), len(send), recv[0].numel(), dtype_code(recv[0]),
+                            _stream(stream)), "cc_allgather")
+
+
+def cc_broadcast(src, recv, root: int = 0, *, stream=None) -> None:
+    _ranks(recv, "cc_broadcast")
+    _same(recv, src.numel(), src.dtype, "cc_broadcast recv")
+    _check(lib.cc_broadcast(_dev_ptr(src), _ptrs(recv), len(recv), root, src.numel(), dtype_code(src),
+                            _stream(stream)), "cc_broadcast")
+
+
+def cc_reduce(send, recv_root, root: int = 0, *, op="sum", scale=1.0, stream=None) -> None:
+    _ranks(send, "cc_reduce")
+    _same(send, send[0].numel(), send[0].dtype, "cc_reduce send")
+    _same([recv_root], send[0].numel(), recv_root.dtype, "cc_reduce recv_root")
+    _check(lib.cc_reduce(_ptrs(send), _dev_ptr(recv_root), len(send), root, send[0].numel(), dtype_code(send[0]),
+                         dtype_code(recv_root), _OPS[op], float(scale), _stream(stream)), "cc_reduce")
+
+
+def cc_scatter(src, recv, root: int = 0, *, stream=None) -> None:
+    n = _ranks(recv, "cc_scatter")
+    for c in range(n):
+        _same([recv[c]], cc_chunk(src.numel(), n, c)[1], src.dtype, f"cc_scatter recv[{c}]")
+    _check(lib.cc_scatter(_dev_ptr(src), _ptrs(recv), len(recv), root, src.numel(), dtype_code(src),
+                          _stream(stream)), "cc_scatter")
+
+
+def cc_gather(send, recv_root, root: int = 0, *, stream=None) -> None:
+    n = _ranks(send, "cc_gather")
+    for c in range(n):
+        _same([send[c]], cc_chunk(recv_root.numel(), n, c)[1], recv_root.dtype, f"cc_gather send[{c}]")
+    _check(lib.cc_gather(_ptrs(send), _dev_ptr(recv_root), len(send), root, recv_root.numel(),
+                         dtype_code(recv_root), _stream(stream)), "cc_gather")
+
+
+# ---- MoE -----------------------------------------------------------------------------------------
+
+def cc_route_topk(logits, expert_ids, *, stream=None) -> None:
+    """expert_ids[r][t] = top-k expert ids of logits[r][t] (larger first, ties to lower id)."""
+    torch = _torch()
+    _ranks(logits, "cc_route_topk")
+    tokens, experts = logits[0].shape
+    _same(logits, tokens * experts, torch.float32, "cc_route_topk logits")
+    _same(expert_ids, tokens * expert_ids[0].shape[1], torch.int32, "cc_route_topk expert_ids")
+    if len(expert_ids) != len(logits):
+        raise ValueError("cc_route_topk: one id tensor per rank")
+    _check(lib.cc_route_topk(_ptrs(logits), _ptrs(expert_ids), len(logits), tokens, experts,
+                             expert_ids[0].shape[1], _stream(stream)), "cc_route_topk")
+
+
+def cc_alltoallv_workspace_size(nranks: int, tokens: int, topk: int, experts_per_rank: int) -> int:
+    return int(lib.cc_alltoallv_workspace_size(nranks, tokens, topk, experts_per_rank))
+
+
+def cc_alltoallv(send, recv, expert_ids, experts_per_rank: int, workspace, *, direction: int = 0,
+                 row_bytes: Optional[int] = None, recv_capacity_rows: Optional[int] = None, stream=None) -> None:
+    """direction 0: dispatch token rows to expert ranks; 1: combine them back.
+
+    Dispatch: send[s] is [tokens, hidden]; recv[d] holds up to recv_capacity_rows rows.
+    Combine: send[d] is rank d's dispatch output; recv[s] is [tokens, topk, hidden]."""
+    torch = _torch()
+    n = _ranks(send, "cc_alltoallv")
+    if len(recv) != n or len(expert_ids) != n:
+        raise ValueError("cc_alltoallv: one send, recv and id tensor per rank")
+    tokens, topk = expert_ids[0].shape
+    _same(expert_ids, tokens * topk, torch.int32, "cc_alltoallv expert_ids")
+    tok = send if direction == 0 else recv
+    if row_bytes is None:
+        row_bytes = tok[0].numel() * tok[0].element_size() // max(1, tokens * (1 if direction == 0 else topk))
+    rows_side = recv if direction == 0 else send
+    cap = min(t.numel() * t.element_size() for t in rows_side) // row_bytes
+    recv_capacity_rows = cap if recv_capacity_rows is None else min(cap, recv_capacity_rows)
+    need = tokens * row_bytes * (1 if direction == 0 else topk)
+    for t in tok:
+        if t.numel() * t.element_size() < need:
+            raise ValueError("cc_alltoallv: token buffer smaller than tokens x row_bytes (x topk for combine)")
+    if workspace.numel() * workspace.element_size() < cc_alltoallv_workspace_size(n, tokens, topk, experts_per_rank):
+        raise ValueError("cc_alltoallv: workspace too small")
+    _check(lib.cc_alltoallv(_ptrs(send), _ptrs(recv), len(send), row_bytes, _ptrs(expert_ids), tokens, topk,
+                            experts_per_rank, recv_capacity_rows, direction, _dev_ptr(workspace),
+                            workspace.numel() * workspace.element_size(), _stream(stream)), "cc_alltoallv")
+
+
+def cc_alltoallv_recv_counts(workspace, nranks: int, out, *, stream=None) -> None:
+    """Stream-ordered copy of the per-destination received row counts into `out` (int32;
+    a CUDA tensor or a pinned host tensor)."""
+    torch = _torch()
+    if out.dtype != torch.int32 or out.numel() < nranks:
+        raise ValueError("cc_alltoallv_recv_counts: out must hold nranks int32")
+    if not out.is_cuda and not out.is_pinned():
+        raise ValueError("cc_alltoallv_recv_counts: a host output must be pinned")
+    ptr = out.data_ptr()
+    _check(lib.cc_alltoallv_recv_counts(_dev_ptr(workspace), nranks, ptr, _stream(stream)),
+           "cc_alltoallv_recv_counts")
+
+
+# ---- DDP buckets ----------------------------------------------------------------------------------
+
+def cc_bucket_assign(numels: Sequence[int], elem_bytes: int = 4, cap_bytes: int = 25 * 1024 * 1024):
+    """Host call: returns the tensor ids of each bucket, buckets in launch order."""
+    n = len(numels)
+    order = (ctypes.c_int32 * max(1, n))()
+    start = (ctypes.c_int32 * (n + 1))()
+    nb = ctypes.c_int32()
+    _check(lib.cc_bucket_assign(_sizes(numels) if n else None, n, elem_bytes, cap_bytes, order, start,
+                                ctypes.byref(nb)), "cc_bucket_assign")
+    return [[order[k] for k in range(start[b], start[b + 1])] for b in range(nb.value)]
+
+
+def cc_bucket_flatten(tensors, bucket, *, stream=None) -> None:
+    if sum(t.numel() for t in tensors) > bucket.numel() or any(t.dtype != bucket.dtype for t in tensors):
+        raise ValueError("cc_bucket_flatten: bucket too small or dtype mismatch")
+    _check(lib.cc_bucket_flatten(_ptrs(tensors), _sizes([t.numel() for t in tensors]), len(tensors),
+                                 _dev_ptr(bucket), dtype_code(bucket), _stream(stream)), "cc_bucket_flatten")
+
+
+def cc_bucket_unflatten(bucket, tensors, *, stream=None) -> None:
+    if sum(t.numel() for t in tensors) > bucket.numel() or any(t.dtype != bucket.dtype for t in tensors):
+        raise ValueError("cc_bucket_unflatten: bucket too small or dtype mismatch")
+    _check(lib.cc_bucket_unflatten(_dev_ptr(bucket), _ptrs(tensors), _sizes([t.numel() for t in tensors]),
+                                   len(tensors), dtype_code(bucket), _stream(stream)), "cc_bucket_unflatten")
+
+
+def cc_bucket_allreduce(grads, out, *, cap_bytes: int = 25 * 1024 * 1024, algo="ring", scale=None,
+                        stream=None) -> None:
+    """grads[r][i] / out[r][i]: rank r's tensor i (registration order). One fused pass."""
+    torch = _torch()
+    n, nt = _ranks(grads, "cc_bucket_allreduce"), len(grads[0])
+    if len(out) != n or any(len(row) != nt for row in list(grads) + list(out)):
+        raise ValueError("cc_bucket_allreduce: grads and out must both be [nranks][ntensors]")
+    for i in range(nt):
+        _same([grads[r][i] for r in range(n)] + [out[r][i] for r in range(n)], grads[0][i].numel(),
+              torch.float32, f"cc_bucket_allreduce tensor {i}")
+    scale = 1.0 / n if scale is None else scale
+    flat_in = [t for row in grads for t in row]
+    flat_out = [t for row in out for t in row]
+    _check(lib.cc_bucket_allreduce(_ptrs(flat_in), _ptrs(flat_out), n, nt, _sizes([t.numel() for t in grads[0]]),
+                                   cap_bytes, _ALGOS[algo], float(scale), _stream(stream)), "cc_bucket_allreduce")
+
+
+def raw_call(name: str, *args) -> int:
+    """Call a C entry point with already-marshalled arguments (tests of the ABI itself)."""
+    return getattr(lib, name)(*args)

@@ -1,0 +1,298 @@
+// MoE expert parallelism: top-k routing and the alltoallv dispatch / combine
+// (lecture 09 §6.4; AllToAll semantics §3.8 and experiment 4 §7.4).
+//
+// Dispatch layout: rank d's receive buffer is the concatenation over source ranks
+// s = 0..N-1 of s's rows for d, each block ordered by (local expert, token, slot).
+// The position of row i = t * topk + k of source s routed to global expert e is
+//   base[s][e] + tile_off[s][tile(i)][e] + rank_in_tile(i)
+// where base[s][e] = rows of earlier sources for the same destination + rows of s for
+// earlier local experts of that destination, tile_off is the exclusive prefix over
+// tiles of 256 rows, and rank_in_tile counts earlier rows of the tile with the same
+// expert (warp match + per-warp counts). All of it is integer and deterministic.
+//
+// Kernels: K1 tile counts and per-row ranks, K2 tile prefix per (s, e), K3 bases and
+// receive counts, K4 the row copy (one warp per token: the token row is read once and
+// written topk times; combine reads topk rows and writes topk rows).
+#include <algorithm>
+
+#include "cc_device.cuh"
+#include "cc_launch.h"
+
+namespace cc {
+
+constexpr int kTileRows = 256;  // rows per K1 tile: 8 warps
+constexpr int kMaxTopk = 8;
+constexpr int kMaxExperts = 1024;
+
+struct A2AWorkspace {
+  // byte offsets inside the caller's workspace; the receive counts sit first, at a
+  // fixed place, so that they can be read back without knowing the other sizes
+  size_t recv_count, tile_cnt, row_rank, totals, base, total;
+};
+
+static A2AWorkspace a2a_layout(int nranks, int tokens, int topk, int experts_per_rank) {
+  const size_t E = (size_t)nranks * experts_per_rank;
+  const size_t rows = (size_t)tokens * topk;
+  const size_t ntiles = (rows + kTileRows - 1) / kTileRows;
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  A2AWorkspace w;
+  w.recv_count = 0;
+  w.tile_cnt = up(sizeof(int) * kMaxRanks);
+  w.row_rank = up(w.tile_cnt + sizeof(int) * nranks * ntiles * E);
+  w.totals = up(w.row_rank + sizeof(int) * nranks * rows);
+  w.base = up(w.totals + sizeof(int) * nranks * E);
+  w.total = up(w.base + sizeof(int) * nranks * E);
+  return w;
+}
+
+size_t a2a_workspace_bytes(int nranks, int tokens, int topk, int experts_per_rank) {
+  return a2a_layout(nranks, tokens, topk, experts_per_rank).total;
+}
+
+struct IdPtrs {
+  const int32_t* ids[kMaxRanks];
+};
+
+// ---- top-k routing ---------------------------------------------------------------------------------
+
+struct RouteParams {
+  const float* logits[kMaxRanks];
+  int32_t* ids[kMaxRanks];
+  int tokens, experts, topk;
+};
+
+__device__ __forceinline__ bool better(float a, int ia, float b, int ib) {
+  return a > b || (a == b && ia < ib);
+}
+
+// One warp per token: topk rounds of a warp arg-max (larger value, then lower id).
+__global__ void __launch_bounds__(256) route_topk_kernel(const __grid_constant__ RouteParams P) {
+  const int lane = threadIdx.x & 31;
+  const int s = blockIdx.y;
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= P.tokens) return;
+  const float* row = P.logits[s] + (size_t)t * P.experts;
+  int chosen[kMaxTopk];
+  for (int j = 0; j < P.topk; ++j) {
+    float bv = 0.f;
+    int bi = -1;
+    for (int e = lane; e < P.experts; e += 32) {
+      bool taken = false;
+      for (int q = 0; q < j; ++q) taken |= (chosen[q] == e);
+      if (taken) continue;
+      const float v = __ldg(row + e);
+      if (bi < 0 || better(v, e, bv, bi)) { bv = v; bi = e; }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+      if (oi >= 0 && (bi < 0 || better(ov, oi, bv, bi))) { bv = ov; bi = oi; }
+    }
+    chosen[j] = bi;
+  }
+  if (lane < P.topk) {
+    int v = chosen[0];
+    for (int q = 1; q < kMaxTopk; ++q)
+      if (q == lane) v = chosen[q];
+    P.ids[s][(size_t)t * P.topk + lane] = v;
+  }
+}
+
+cudaError_t launch_route_topk(const float* const* logits, int32_t* const* ids, int nranks, int tokens,
+                              int experts_total, int topk, cudaStream_t stream) {
+  RouteParams P{};
+  for (int r = 0; r < nranks; ++r) {
+    P.logits[r] = logits[r];
+    P.ids[r] = ids[r];
+  }
+  P.tokens = tokens;
+  P.experts = experts_total;
+  P.topk = topk;
+  dim3 grid((tokens + 7) / 8, nranks);
+  route_topk_kernel<<<grid, 256, 0, stream>>>(P);
+  return cudaGetLastError();
+}
+
+// ---- K1: per-tile expert counts and per-row rank within the tile -------------------------------------
+
+__global__ void __launch_bounds__(kTileRows) a2a_count_kernel(const __grid_constant__ IdPtrs I, int rows, int E,
+                                                              int* __restrict__ tile_cnt, int* __restrict__ row_rank) {
+  extern __shared__ int warp_cnt[];  // [8][E]
+  const int s = blockIdx.y, tile = blockIdx.x, ntiles = gridDim.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < 8 * E; i += blockDim.x) warp_cnt[i] = 0;
+  __syncthreads();
+  const int row = tile * kTileRows + threadIdx.x;
+  int e = row < rows ? I.ids[s][row] : -1;
+  const bool valid = e >= 0 && e < E;  // rows with an out-of-range expert id are not sent
+  if (!valid) e = -1 - lane;           // invalid lanes match nobody
+  const unsigned peers = __match_any_sync(0xffffffffu, e);
+  const unsigned lt = (1u << lane) - 1;
+  const int rank_w = __popc(peers & lt);
+  if (valid && rank_w == 0) warp_cnt[warp * E + e] = __popc(peers);
+  __syncthreads();
+  // exclusive prefix over the 8 warps, per expert; tile total to global memory
+  for (int x = threadIdx.x; x < E; x += blockDim.x) {
+    int run = 0;
+    for (int w = 0; w < 8; ++w) {
+      const int c = warp_cnt[w * E + x];
+      warp_cnt[w * E + x] = run;
+      run += c;
+    }
+    tile_cnt[((size_t)s * ntiles + tile) * E + x] = run;
+  }
+  __syncthreads();
+  if (valid) row_rank[(size_t)s * rows + row] = warp_cnt[warp * E + e] + rank_w;
+}
+
+// ---- K2: exclusive prefix over tiles, per (source, expert); one warp each -----------------------------
+
+__global__ void a2a_tile_scan_kernel(int ntiles, int E, int* __restrict__ tile_cnt, int* __restrict__ totals) {
+  const int s = blockIdx.y, e = blockIdx.x, lane = threadIdx.x;
+  int carry = 0;
+  for (int t0 = 0; t0 < ntiles; t0 += 32) {
+    const int t = t0 + lane;
+    int* p = tile_cnt + ((size_t)s * ntiles + t) * E + e;
+    const int v = t < ntiles ? *p : 0;
+    int inc = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, inc, off);
+      if (lane >= off) inc += o;
+    }
+    if (t < ntiles) *p = carry + inc - v;
+    carry += __shfl_sync(0xffffffffu, inc, 31);
+  }
+  if (lane == 0) totals[(size_t)s * E + e] = carry;
+}
+
+// ---- K3: bases per (source, expert) and receive counts per destination (one CTA) -------------------------
+
+__global__ void __launch_bounds__(1024) a2a_base_kernel(int nranks, int epr, const int* __restrict__ tot,
+                                                        int* __restrict__ base, int* __restrict__ recv_count) {
+  __shared__ int cnt[kMaxRanks * kMaxRanks];  // rows s -> d
+  const int E = nranks * epr;
+  for (int i = threadIdx.x; i < nranks * nranks; i += blockDim.x) {
+    const int s = i / nranks, d = i % nranks;
+    int c = 0;
+    for (int l = 0; l < epr; ++l) c += tot[s * E + d * epr + l];
+    cnt[i] = c;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < nranks * E; i += blockDim.x) {
+    const int s = i / E, e = i % E, d = e / epr;
+    int off = 0;
+    for (int sp = 0; sp < s; ++sp) off += cnt[sp * nranks + d];
+    for (int l = d * epr; l < e; ++l) off += tot[s * E + l];
+    base[i] = off;
+  }
+  for (int d = threadIdx.x; d < nranks; d += blockDim.x) {
+    int c = 0;
+    for (int s = 0; s < nranks; ++s) c += cnt[s * nranks + d];
+    recv_count[d] = c;
+  }
+}
+
+// ---- K4: row copies ----------------------------------------------------------------------------------
+
+struct A2ACopyParams {
+  const char* send[kMaxRanks];
+  char* recv[kMaxRanks];
+  const int32_t* ids[kMaxRanks];
+  const int* tile_off;   // [N][ntiles][E]
+  const int* row_rank;   // [N][rows]
+  const int* base;       // [N][E]
+  uint64_t row_bytes;
+  uint64_t capacity;
+  int tokens, topk, epr, E, ntiles, direction;
+};
+
+__global__ void __launch_bounds__(256) a2a_copy_kernel(const __grid_constant__ A2ACopyParams P) {
+  const int lane = threadIdx.x & 31;
+  const int s = blockIdx.y;
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= P.tokens) return;
+  const int rows = P.tokens * P.topk;
+  char* ptr[kMaxTopk];
+  bool ok[kMaxTopk];
+  for (int k = 0; k < P.topk; ++k) {
+    const int i = t * P.topk + k;
+    const int e = P.ids[s][i];
+    if (e < 0 || e >= P.E) { ok[k] = false; ptr[k] = nullptr; continue; }
+    const int d = e / P.epr;
+    const uint64_t pos = (uint64_t)P.base[s * P.E + e] +
+                         P.tile_off[((size_t)s * P.ntiles + i / kTileRows) * P.E + e] +
+                         P.row_rank[(size_t)s * rows + i];
+    ok[k] = pos < P.capacity;
+    ptr[k] = (P.direction == 0 ? P.recv[d] : const_cast<char*>(P.send[d])) + pos * P.row_bytes;
+  }
+  const uint64_t nvec = P.row_bytes / 16;
+  if (P.direction == 0) {
+    const char* src = P.send[s] + (uint64_t)t * P.row_bytes;
+    for (uint64_t v = lane; v < nvec; v += 32) {
+      const uint4 x = __ldcs(reinterpret_cast<const uint4*>(src) + v);
+      for (int k = 0; k < P.topk; ++k)
+        if (ok[k]) __stcs(reinterpret_cast<uint4*>(ptr[k]) + v, x);
+    }
+  } else {
+    char* dst = P.recv[s] + (uint64_t)t * P.topk * P.row_bytes;
+    for (int k = 0; k < P.topk; ++k) {
+      if (!ok[k]) continue;
+      for (uint64_t v = lane; v < nvec; v += 32)
+        __stcs(reinterpret_cast<uint4*>(dst + k * P.row_bytes) + v, __ldcs(reinterpret_cast<const uint4*>(ptr[k]) + v));
+    }
+  }
+}
+
+cudaError_t launch_alltoallv(const void* const* send, void* const* recv, int nranks, size_t row_bytes,
+                             const int32_t* const* ids, int tokens, int topk, int experts_per_rank,
+                             size_t capacity_rows, int direction, void* workspace, cudaStream_t stream) {
+  const int E = nranks * experts_per_rank;
+  const int rows = tokens * topk;
+  const int ntiles = (rows + kTileRows - 1) / kTileRows;
+  const A2AWorkspace w = a2a_layout(nranks, tokens, topk, experts_per_rank);
+  char* ws = static_cast<char*>(workspace);
+  int* tile_cnt = reinterpret_cast<int*>(ws + w.tile_cnt);
+  int* row_rank = reinterpret_cast<int*>(ws + w.row_rank);
+  int* totals = reinterpret_cast<int*>(ws + w.totals);
+  int* base = reinterpret_cast<int*>(ws + w.base);
+  int* recv_count = reinterpret_cast<int*>(ws + w.recv_count);
+  IdPtrs I{};
+  for (int r = 0; r < nranks; ++r) I.ids[r] = ids[r];
+  if (rows > 0) {
+    a2a_count_kernel<<<dim3(ntiles, nranks), kTileRows, sizeof(int) * 8 * E, stream>>>(I, rows, E, tile_cnt, row_rank);
+    a2a_tile_scan_kernel<<<dim3(E, nranks), 32, 0, stream>>>(ntiles, E, tile_cnt, totals);
+  } else {
+    cudaMemsetAsync(totals, 0, sizeof(int) * nranks * E, stream);
+  }
+  a2a_base_kernel<<<1, 1024, 0, stream>>>(nranks, experts_per_rank, totals, base, recv_count);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess || rows == 0) return err;
+  A2ACopyParams P{};
+  for (int r = 0; r < nranks; ++r) {
+    P.send[r] = static_cast<const char*>(send[r]);
+    P.recv[r] = static_cast<char*>(recv[r]);
+    P.ids[r] = ids[r];
+  }
+  P.tile_off = tile_cnt;
+  P.row_rank = row_rank;
+  P.base = base;
+  P.row_bytes = row_bytes;
+  P.capacity = capacity_rows;
+  P.tokens = tokens;
+  P.topk = topk;
+  P.epr = experts_per_rank;
+  P.E = E;
+  P.ntiles = ntiles;
+  P.direction = direction;
+  a2a_copy_kernel<<<dim3((tokens + 7) / 8, nranks), 256, 0, stream>>>(P);
+  return cudaGetLastError();
+}
+
+cudaError_t copy_recv_counts(const void* workspace, int nranks, int32_t* out, cudaStream_t stream) {
+  return cudaMemcpyAsync(out, static_cast<const char*>(workspace), sizeof(int32_t) * nranks, cudaMemcpyDefault,
+                         stream);
+}
+
+}  // namespace cc

@@ -1,0 +1,464 @@
+// Reduction kernels: fused ring / double-binary-tree allreduce, ring reduce-scatter,
+// binomial reduce-to-root, and the fused DDP bucket allreduce.
+//
+// All simulated ranks live in this GPU's memory, so one pass computes what every rank
+// would hold at the end of the schedule: each thread owns a 16-byte column of the N rank
+// buffers, loads it from every rank (streaming 128-bit loads), folds the N values in the
+// schedule's order in registers, multiplies by the scale, and stores the result to every
+// output (allreduce), to the owning shard (reduce-scatter) or to the root (reduce).
+// HBM traffic is the minimum the operation allows (N·T in + N·T out for allreduce).
+//
+// Fold orders (collective pages: lecture 09 §4.3 and experiment 1 §7.1 for the ring, §5.2
+// and the multi-node page §4.3.2 for the double binary tree, §3.4 for reduce):
+//   ring      chunk c folds ((x_c (+) x_{c+1}) (+) ...) (+) x_{c-1}
+//   tree      half A / half B fold over tree A / tree B, ((S_left (+) x) (+) S_right)
+//   binomial  node v folds x_v, then each child's partial in send order
+#include <algorithm>
+#include <mutex>
+#include <vector>
+
+#include "cc_device.cuh"
+#include "cc_launch.h"
+
+namespace cc {
+
+constexpr int kThreads = 256;
+
+// ---- folds over the N ranks ---------------------------------------------------------------------
+
+// Left fold starting at rank c: loads go out in windows of 8 so that 8 independent
+// 128-bit loads per thread are in flight before the in-order folds consume them.
+template <int IN, int OP, typename V, typename Load>
+__device__ __forceinline__ V ring_fold(int n, int c, Load ld) {
+  V acc = ld(c);
+  int r = c;
+  for (int j0 = 1; j0 < n; j0 += 8) {
+    V x[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (j0 + k < n) { r = (r + 1 == n) ? 0 : r + 1; x[k] = ld(r); }
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (j0 + k < n) comb<IN, OP>(acc, x[k]);
+  }
+  return acc;
+}
+
+// Fold machine (tree / binomial): the position's rank is rmap[p], mirrored for tree B.
+template <int IN, int OP, typename V, int W, typename Load>
+__device__ __forceinline__ V machine_fold(int n, const FoldProgram& prog, bool mirror, Load ld) {
+  V cur;
+  FoldStack<V> st;
+  for (int p0 = 0; p0 < n; p0 += W) {
+    V x[W];
+#pragma unroll
+    for (int k = 0; k < W; ++k)
+      if (p0 + k < n) {
+        const int rk = prog.rmap[p0 + k];
+        x[k] = ld(mirror ? n - 1 - rk : rk);
+      }
+#pragma unroll
+    for (int k = 0; k < W; ++k)
+      if (p0 + k < n) fold_step<IN, OP>(prog.code[p0 + k], x[k], cur, st);
+  }
+  return cur;
+}
+
+// Elements [a, b) of one fold group, spread over threads t = 0..T-1: 16-byte units where
+// every address is aligned, element-wise head and tail around them.
+template <int IN, int OP, bool RING, typename Src, typename EmitU, typename EmitE>
+__device__ __forceinline__ void reduce_range(int n, int g, bool mirror, const FoldProgram& prog,
+                                             uint64_t a, uint64_t b, uint64_t t, uint64_t T, bool vec,
+                                             Src src, EmitU emit_unit, EmitE emit_elem) {
+  using In = typename Tr<IN>::In;
+  using A = typename Tr<IN>::Acc;
+  constexpr int UE = Tr<IN>::UE;
+  constexpr int W = UE == 8 ? 4 : 8;
+  auto fold_elem = [&](uint64_t e) -> A {
+    auto ld = [&](int r) { return load_elem<IN>(src(r) + e); };
+    if constexpr (RING) return ring_fold<IN, OP, A>(n, g, ld);
+    else return machine_fold<IN, OP, A, W>(n, prog, mirror, ld);
+  };
+  if (vec) {
+    uint64_t va = (a + UE - 1) / UE * UE;
+    if (va > b) va = b;
+    uint64_t vb = b / UE * UE;
+    if (vb < va) vb = va;
+    for (uint64_t e = va + t * UE; e < vb; e += T * UE) {
+      auto ld = [&](int r) { return load_unit<IN>(src(r) + e); };
+      Unit<IN> u;
+      if constexpr (RING) u = ring_fold<IN, OP, Unit<IN>>(n, g, ld);
+      else u = machine_fold<IN, OP, Unit<IN>, W>(n, prog, mirror, ld);
+      emit_unit(e, u);
+    }
+    const uint64_t nh = va - a, nt = b - vb;
+    if (t < nh) emit_elem(a + t, fold_elem(a + t));
+    else if (t < nh + nt) emit_elem(vb + (t - nh), fold_elem(vb + (t - nh)));
+  } else {
+    for (uint64_t e = a + t; e < b; e += T) emit_elem(e, fold_elem(e));
+  }
+}
+
+// ---- chunk rule ---------------------------------------------------------------------------------
+// q = count / n, r = count % n; chunk c has q + (c < r) elements, starting at c*q + min(c, r).
+
+__host__ __device__ __forceinline__ void chunk_range(uint64_t count, int n, int c, uint64_t& a, uint64_t& b) {
+  const uint64_t q = count / n, r = count % n, cc_ = (uint64_t)c;
+  a = cc_ * q + (cc_ < r ? cc_ : r);
+  b = a + q + (cc_ < r ? 1 : 0);
+}
+
+// Chunk of element o and the end of that chunk.
+__device__ __forceinline__ int chunk_of(uint64_t count, int n, uint64_t o, uint64_t& end) {
+  const uint64_t q = count / n, r = count % n;
+  const uint64_t big = r * (q + 1);
+  if (o < big) {
+    const uint64_t c = o / (q + 1);
+    end = (c + 1) * (q + 1);
+    return (int)c;
+  }
+  const uint64_t c = r + (o - big) / q;
+  end = big + (c - r + 1) * q;
+  return (int)c;
+}
+
+// ---- plain reduction kernel ------------------------------------------------------------------------
+
+struct ReduceParams {
+  const void* src[kMaxRanks];
+  void* dst[kMaxRanks];
+  FoldProgram prog;
+  uint64_t count;
+  uint64_t dst_aligned;  // bit r: dst[r] is 16-byte aligned
+  int nranks;
+  int mode;
+  int fold;
+  int vec;  // every source (and every allreduce / root destination) is 16-byte aligned
+  float scale;
+  int do_scale;
+};
+
+template <int IN, int OP, bool RING>
+__global__ void __launch_bounds__(kThreads) reduce_kernel(const __grid_constant__ ReduceParams P) {
+  using In = typename Tr<IN>::In;
+  using Out = typename Tr<IN>::Out;
+  using A = typename Tr<IN>::Acc;
+  const int n = P.nranks;
+  const int g = blockIdx.y;
+  uint64_t a, b;
+  if (P.fold == kFoldRing) {
+    chunk_range(P.count, n, g, a, b);
+  } else if (P.fold == kFoldTree) {
+    const uint64_t mid = (P.count + 1) / 2;
+    a = g ? mid : 0;
+    b = g ? P.count : mid;
+  } else {
+    a = 0;
+    b = P.count;
+  }
+  const bool mirror = (P.fold == kFoldTree && g == 1);
+  const uint64_t T = (uint64_t)gridDim.x * blockDim.x;
+  const uint64_t t = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int mode = P.mode;
+  const bool shard_vec = ((P.dst_aligned >> g) & 1) && ((a * sizeof(Out)) % 16 == 0);
+  auto src = [&](int r) { return static_cast<const In*>(P.src[r]); };
+  auto emit_unit = [&](uint64_t e, Unit<IN> u) {
+    if (P.do_scale) scale_unit<IN>(u, P.scale);
+    if (mode == kAllReduce) {
+      for (int r = 0; r < n; ++r) store_unit<IN>(static_cast<Out*>(P.dst[r]) + e, u);
+    } else if (mode == kReduceScatter) {
+      Out* d = static_cast<Out*>(P.dst[g]) + (e - a);
+      if (shard_vec) store_unit<IN>(d, u); else store_unit_scalar<IN>(d, u);
+    } else {
+      store_unit<IN>(static_cast<Out*>(P.dst[0]) + e, u);
+    }
+  };
+  auto emit_elem = [&](uint64_t e, A v) {
+    if constexpr (IN != CC_I32) if (P.do_scale) v = __fmul_rn(v, P.scale);
+    if (mode == kAllReduce) {
+      for (int r = 0; r < n; ++r) store_elem<IN>(static_cast<Out*>(P.dst[r]) + e, v);
+    } else if (mode == kReduceScatter) {
+      store_elem<IN>(static_cast<Out*>(P.dst[g]) + (e - a), v);
+    } else {
+      store_elem<IN>(static_cast<Out*>(P.dst[0]) + e, v);
+    }
+  };
+  reduce_range<IN, OP, RING>(n, g, mirror, P.prog, a, b, t, T, P.vec != 0, src, emit_unit, emit_elem);
+}
+
+// ---- fused DDP bucket allreduce --------------------------------------------------------------------
+// One launch covers a group of gradient tensors. Work is cut into tiles of kBucketTile
+// elements that never cross a tensor; a CTA takes tiles round-robin, finds the tile's
+// tensor by binary search in the tile prefix table, and splits the tile at the fold-group
+// boundaries of the tensor's bucket (ring chunks or tree halves, in bucket coordinates).
+// Every element is folded exactly as in flatten -> allreduce -> unflatten, with no flat
+// buffer: N·G bytes in, N·G bytes out.
+
+constexpr int kBucketMaxTensors = 192;
+constexpr int kBucketMaxPtrs = 1536;
+constexpr uint64_t kBucketTile = 8192;
+
+struct BucketParams {
+  int nranks;
+  int ntensors;
+  int fold;
+  int vec;
+  float scale;
+  int do_scale;
+  FoldProgram prog;
+  uint32_t tile_prefix[kBucketMaxTensors + 1];
+  BucketTensorDesc t[kBucketMaxTensors];
+  const float* in[kBucketMaxPtrs];
+  float* out[kBucketMaxPtrs];
+};
+static_assert(sizeof(BucketParams) <= 32000, "kernel parameter block too large");
+
+template <bool RING>
+__global__ void __launch_bounds__(kThreads) bucket_allreduce_kernel(const __grid_constant__ BucketParams P) {
+  constexpr int IN = CC_F32, OP = CC_SUM;
+  const int n = P.nranks, nt = P.ntensors;
+  const uint32_t ntiles = P.tile_prefix[nt];
+  for (uint32_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    int lo = 0, hi = nt - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (P.tile_prefix[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    const int i = lo;
+    const BucketTensorDesc d = P.t[i];
+    const uint64_t ea = (uint64_t)(tile - P.tile_prefix[i]) * kBucketTile;
+    const uint64_t eb = min(ea + kBucketTile, d.numel);
+    auto src = [&](int r) { return P.in[r * nt + i]; };
+    auto emit_unit = [&](uint64_t e, Unit<IN> u) {
+      if (P.do_scale) scale_unit<IN>(u, P.scale);
+      for (int r = 0; r < n; ++r) store_unit<IN>(P.out[r * nt + i] + e, u);
+    };
+    auto emit_elem = [&](uint64_t e, float v) {
+      if (P.do_scale) v = __fmul_rn(v, P.scale);
+      for (int r = 0; r < n; ++r) store_elem<IN>(P.out[r * nt + i] + e, v);
+    };
+    uint64_t s = ea;
+    while (s < eb) {
+      const uint64_t o = d.bucket_off + s;
+      uint64_t gend;
+      int g;
+      if (RING) {
+        g = chunk_of(d.bucket_count, n, o, gend);
+      } else {
+        const uint64_t mid = (d.bucket_count + 1) / 2;
+        g = o >= mid;
+        gend = g ? d.bucket_count : mid;
+      }
+      const uint64_t se = min(eb, gend - d.bucket_off);
+      reduce_range<IN, OP, RING>(n, g, !RING && g == 1, P.prog, s, se, threadIdx.x, blockDim.x,
+                                 P.vec != 0, src, emit_unit, emit_elem);
+      s = se;
+    }
+  }
+}
+
+// ---- host side --------------------------------------------------------------------------------------
+
+static int ctz_int(int q) { return __builtin_ctz((unsigned)q); }
+
+// Double binary tree, tree A, in fold-machine codes (tree B uses the same codes mirrored).
+static void tree_program(int n, FoldProgram& fp) {
+  int left[kMaxRanks + 2] = {0}, right[kMaxRanks + 2] = {0}, parent[kMaxRanks + 2] = {0};
+  bool is_right[kMaxRanks + 2] = {false};
+  for (int q = 1; q <= n; ++q) {
+    const int h = ctz_int(q);
+    if (h == 0) continue;
+    const int lq = q - (1 << (h - 1));
+    left[q] = lq;
+    parent[lq] = q;
+    for (int j = h; j >= 1; --j) {
+      const int rq = q + (1 << (j - 1));
+      if (rq <= n) {
+        right[q] = rq;
+        parent[rq] = q;
+        is_right[rq] = true;
+        break;
+      }
+    }
+  }
+  for (int p = 0; p < n; ++p) {
+    const int q = p + 1;
+    uint8_t code = left[q] ? kFoldCur : 0;
+    if (right[q]) {
+      code |= kPush;
+    } else {
+      int npop = 0, u = q;
+      while (parent[u] && is_right[u]) { ++npop; u = parent[u]; }
+      code |= (uint8_t)(npop << 2);
+    }
+    fp.code[p] = code;
+    fp.rmap[p] = (uint8_t)p;
+  }
+}
+
+// Binomial tree rooted at `root` (relative rank v = (r - root) mod n; parent v - 2^floor(log2 v);
+// children v + 2^k for 2^k > v), visited in pre-order.
+static void binomial_program(int n, int root, FoldProgram& fp) {
+  auto children = [n](int v) {
+    std::vector<int> ch;
+    int k = 0;
+    if (v) while ((1 << k) <= v) ++k;
+    for (; v + (1 << k) < n; ++k) ch.push_back(v + (1 << k));
+    return ch;
+  };
+  auto parent_of = [](int v) { int k = 0; while ((2 << k) <= v) ++k; return v - (1 << k); };
+  std::vector<int> order;
+  std::vector<int> stack = {0};
+  while (!stack.empty()) {
+    const int v = stack.back();
+    stack.pop_back();
+    order.push_back(v);
+    auto ch = children(v);
+    for (auto it = ch.rbegin(); it != ch.rend(); ++it) stack.push_back(*it);
+  }
+  for (int p = 0; p < n; ++p) {
+    const int v = order[p];
+    uint8_t code = 0;
+    if (!children(v).empty()) {
+      code = kPush;
+    } else {
+      int npop = 0, u = v;
+      while (u != 0) {
+        const int par = parent_of(u);
+        const auto sib = children(par);
+        if (sib.back() == u) { ++npop; u = par; continue; }
+        code |= kFoldTop;
+        break;
+      }
+      code |= (uint8_t)(npop << 2);
+    }
+    fp.code[p] = code;
+    fp.rmap[p] = (uint8_t)((v + root) % n);
+  }
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int sm_count() {
+  static int cached[64];
+  static std::once_flag once[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  std::call_once(once[dev], [dev] {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    cached[dev] = v;
+  });
+  return cached[dev];
+}
+
+template <typename K>
+static int blocks_per_sm(K kernel) {
+  int b = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kernel, kThreads, 0) != cudaSuccess || b <= 0) b = 2;
+  return b;
+}
+
+template <int IN, int OP, bool RING>
+static cudaError_t run_reduce(const ReduceParams& P, int ngroups, cudaStream_t s) {
+  auto k = reduce_kernel<IN, OP, RING>;
+  static const int bps = blocks_per_sm(k);
+  constexpr int UE = Tr<IN>::UE;
+  const uint64_t per_group = P.count / ngroups + 1;
+  const uint64_t want = (per_group + (uint64_t)kThreads * UE - 1) / ((uint64_t)kThreads * UE);
+  uint64_t bx = ((uint64_t)sm_count() * bps + ngroups - 1) / ngroups;
+  bx = std::max<uint64_t>(1, std::min(bx, want));
+  dim3 grid((unsigned)bx, (unsigned)ngroups);
+  k<<<grid, kThreads, 0, s>>>(P);
+  return cudaGetLastError();
+}
+
+template <int IN>
+static cudaError_t dispatch_op(const ReduceParams& P, cc_op op, bool ring, int ngroups, cudaStream_t s) {
+  switch (op) {
+    case CC_SUM: return ring ? run_reduce<IN, CC_SUM, true>(P, ngroups, s) : run_reduce<IN, CC_SUM, false>(P, ngroups, s);
+    case CC_MAX: return ring ? run_reduce<IN, CC_MAX, true>(P, ngroups, s) : run_reduce<IN, CC_MAX, false>(P, ngroups, s);
+    case CC_MIN: return ring ? run_reduce<IN, CC_MIN, true>(P, ngroups, s) : run_reduce<IN, CC_MIN, false>(P, ngroups, s);
+    case CC_PROD: return ring ? run_reduce<IN, CC_PROD, true>(P, ngroups, s) : run_reduce<IN, CC_PROD, false>(P, ngroups, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_reduce(const void* const* send, void* const* dst, int ndst, int nranks, size_t count,
+                          cc_dtype in_t, cc_op op, FoldKind fold, ReduceMode mode, int root, float scale,
+                          cudaStream_t stream) {
+  ReduceParams P{};
+  P.count = count;
+  P.nranks = nranks;
+  P.mode = mode;
+  P.fold = fold;
+  P.scale = scale;
+  P.do_scale = (in_t != CC_I32) && scale != 1.0f;
+  bool vec = true;
+  for (int r = 0; r < nranks; ++r) {
+    P.src[r] = send[r];
+    vec = vec && aligned16(send[r]);
+  }
+  for (int r = 0; r < ndst; ++r) {
+    P.dst[r] = dst[r];
+    if (aligned16(dst[r])) P.dst_aligned |= (1ull << r);
+    else if (mode != kReduceScatter) vec = false;
+  }
+  P.vec = vec;
+  if (fold == kFoldTree) tree_program(nranks, P.prog);
+  else if (fold == kFoldBinomial) binomial_program(nranks, root, P.prog);
+  const int ngroups = fold == kFoldRing ? nranks : (fold == kFoldTree ? 2 : 1);
+  const bool ring = fold == kFoldRing;
+  switch (in_t) {
+    case CC_F32: return dispatch_op<CC_F32>(P, op, ring, ngroups, stream);
+    case CC_BF16: return dispatch_op<CC_BF16>(P, op, ring, ngroups, stream);
+    case CC_I32: return dispatch_op<CC_I32>(P, op, ring, ngroups, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+int bucket_group_limit(int nranks) {
+  return std::max(1, std::min(kBucketMaxTensors, kBucketMaxPtrs / nranks));
+}
+
+cudaError_t launch_bucket_allreduce(const void* const* grads, void* const* out, int nranks, int ntensors_total,
+                                    const int32_t* ids, int nids, const BucketTensorDesc* desc, FoldKind fold,
+                                    float scale, cudaStream_t stream) {
+  static BucketParams P;  // large: keep it off the stack; calls are serialised by the caller's lock
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  P.nranks = nranks;
+  P.ntensors = nids;
+  P.fold = fold;
+  P.scale = scale;
+  P.do_scale = scale != 1.0f;
+  bool vec = true;
+  uint32_t tiles = 0;
+  for (int k = 0; k < nids; ++k) {
+    const int i = ids[k];
+    P.t[k] = desc[i];
+    P.tile_prefix[k] = tiles;
+    tiles += (uint32_t)((desc[i].numel + kBucketTile - 1) / kBucketTile);
+    for (int r = 0; r < nranks; ++r) {
+      const void* g = grads[(size_t)r * ntensors_total + i];
+      void* o = out[(size_t)r * ntensors_total + i];
+      P.in[r * nids + k] = static_cast<const float*>(g);
+      P.out[r * nids + k] = static_cast<float*>(o);
+      vec = vec && aligned16(g) && aligned16(o);
+    }
+  }
+  P.tile_prefix[nids] = tiles;
+  P.vec = vec;
+  if (fold == kFoldTree) tree_program(nranks, P.prog);
+  if (tiles == 0) return cudaSuccess;
+  const bool ring = fold == kFoldRing;
+  auto k = ring ? bucket_allreduce_kernel<true> : bucket_allreduce_kernel<false>;
+  static const int bps_ring = blocks_per_sm(bucket_allreduce_kernel<true>);
+  static const int bps_tree = blocks_per_sm(bucket_allreduce_kernel<false>);
+  const uint32_t grid = std::min<uint32_t>(tiles, (uint32_t)(sm_count() * (ring ? bps_ring : bps_tree)));
+  k<<<grid, kThreads, 0, stream>>>(P);
+  return cudaGetLastError();
+}
+
+}  // namespace cc

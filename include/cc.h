@@ -1,0 +1,188 @@
+/* cc.h — collective primitives over N simulated ranks whose buffers all live in one
+ * GPU's memory (B200, sm_100a). C ABI: plain pointers and sizes, no library types.
+ *
+ * Semantics follow the collective pages:
+ *   lecture 09 "网络通信基础与集合通信 Collective 原语直觉" (§3 the eight primitives,
+ *     §4 ring allreduce, §5 tree allreduce, §6 DDP / ZeRO / MoE dataflow, §7 experiments),
+ *   "多节点训练集群网络优化实战" ch. 4 (§4.3.1 ring pseudocode, §4.3.2 double binary tree),
+ *   "从零实现集合通信" (two-pass ring, per-rank byte table, gradient buckets).
+ * Each rank's result is exactly what that rank would hold after the named schedule; a
+ * floating-point reduction folds in the order the schedule implies:
+ *   ring: chunk c (chunk rule below) is folded starting at rank c:
+ *         ((x_c (+) x_{c+1}) (+) ...) (+) x_{c-1}   (indices mod N)
+ *   tree: elements [0, ceil(count/2)) follow tree A, the rest tree B of the double
+ *         binary tree; a node folds ((S_left (+) x_self) (+) S_right). Tree A is the
+ *         in-order tree on positions 0..N-1 (1-based label q = position + 1, height
+ *         h = ctz(q), left child q - 2^(h-1), right child q + 2^(j-1) for the largest
+ *         j <= h with q + 2^(j-1) <= N, root = largest power of two <= N); tree B is its
+ *         mirror (rank r at position N-1-r).
+ *   chunk rule: q = count / N, r = count % N; chunk c has q + (c < r) elements and
+ *         starts at c*q + min(c, r).
+ * (+) is one IEEE binary32 operation rounded to nearest even (SUM add, PROD multiply,
+ * MAX / MIN with -0 ordered below +0), or the wrapping int32 operation. bf16 inputs are
+ * widened exactly to binary32 before the first operation. `scale` multiplies the final
+ * result once (binary32); it must be 1 for int32.
+ *
+ * Conventions for every call:
+ *   - send / recv are HOST arrays of nranks DEVICE pointers (1 <= nranks <= 64), one per
+ *     simulated rank; the caller owns all buffers; the library keeps no pointer after
+ *     the call returns.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *     They return after enqueuing; only argument and launch errors are reported
+ *     synchronously. A failed launch leaves the outputs undefined.
+ *   - count == 0 is a no-op returning CC_OK.
+ *   - 16-byte aligned buffers take the 128-bit path; any other alignment of 4-byte
+ *     (2-byte for bf16) elements takes an element-wise path with the same results.
+ *   - In-place (recv[r] == send[r]) is allowed where stated; any other overlap between
+ *     inputs and outputs is undefined.
+ *   - Allowed (in, out) dtype pairs for reductions: (F32, F32), (BF16, F32), (I32, I32).
+ */
+#ifndef CC_H_
+#define CC_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CC_OK = 0,
+  CC_ERR_INVALID_ARG = 1, /* bad pointer, size, rank, dtype pair, op or workspace */
+  CC_ERR_UNSUPPORTED = 2, /* a valid combination this build does not implement */
+  CC_ERR_CUDA = 3,        /* a CUDA runtime call failed (launch error, no device) */
+  CC_ERR_TIMEOUT = 4      /* a bounded device-side wait gave up (async status) */
+} cc_status;
+
+typedef enum { CC_F32 = 0, CC_BF16 = 1, CC_I32 = 2 } cc_dtype;
+typedef enum { CC_SUM = 0, CC_MAX = 1, CC_MIN = 2, CC_PROD = 3 } cc_op;
+typedef enum { CC_ALGO_RING = 0, CC_ALGO_TREE = 1 } cc_algo;
+
+#define CC_MAX_RANKS 64
+
+#if defined(__GNUC__)
+#define CC_API __attribute__((visibility("default")))
+#else
+#define CC_API
+#endif
+
+/* Human-readable name of a status code (static string). */
+CC_API const char* cc_status_string(cc_status s);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+CC_API int cc_version(void);
+
+/* The chunk rule (host only): chunk c of a count-element buffer over nranks ranks
+ * starts at *start and has *len elements (lecture 09 §7.1 splits the tensor into N equal
+ * chunks; for a count N does not divide, the first count % N chunks get one more). */
+CC_API cc_status cc_chunk(size_t count, int nranks, int c, size_t* start, size_t* len);
+
+/* AllReduce (lecture 09 §3.5; ring §4.3 and experiment 1 §7.1; tree §5.2 and the
+ * multi-node page §4.3.2). Every rank r receives, in recv[r][0..count), the reduction of
+ * send[0..N-1][0..count) folded in `algo`'s order, times `scale`.
+ *   send[r]: count elements of in_t;  recv[r]: count elements of out_t.
+ *   In place allowed (recv[r] == send[r] for every r, same dtype width).
+ * Errors: CC_ERR_INVALID_ARG for null arrays/pointers, nranks outside [1, 64], a dtype
+ * pair not listed above, op outside cc_op, scale != 1 for I32. */
+CC_API cc_status cc_allreduce(const void* const* send, void* const* recv, int nranks, size_t count,
+                       cc_dtype in_t, cc_dtype out_t, cc_op op, cc_algo algo, float scale,
+                       void* stream);
+
+/* ReduceScatter (lecture 09 §3.6; the from-scratch page's reduce_scatter as the first
+ * half of the ring). Rank c receives, in recv[c], chunk c (chunk rule) of the ring
+ * reduction: q + (c < r) elements of out_t. `count` is the per-rank INPUT length.
+ * algo must be CC_ALGO_RING (else CC_ERR_UNSUPPORTED). No in-place. */
+CC_API cc_status cc_reduce_scatter(const void* const* send, void* const* recv, int nranks, size_t count,
+                            cc_dtype in_t, cc_dtype out_t, cc_op op, cc_algo algo, float scale,
+                            void* stream);
+
+/* AllGather (lecture 09 §3.7; ring N-1 steps, the from-scratch page's table). Rank c
+ * contributes send[c] = chunk c (chunk rule over `count`, the per-rank OUTPUT length);
+ * every recv[r] receives all count elements. Bit copy; dtype only sets the width. */
+CC_API cc_status cc_allgather(const void* const* send, void* const* recv, int nranks, size_t count,
+                       cc_dtype dtype, void* stream);
+
+/* Broadcast (lecture 09 §3.1; a log2(N) tree on the from-scratch page). Every recv[r]
+ * receives the count elements at `src` (rank root's buffer). recv[root] may equal src
+ * (then it is not written). Bit copy. */
+CC_API cc_status cc_broadcast(const void* src, void* const* recv, int nranks, int root, size_t count,
+                       cc_dtype dtype, void* stream);
+
+/* Reduce to root (lecture 09 §3.4). recv_root receives the reduction of the N send
+ * buffers over the binomial tree rooted at `root` (the broadcast tree run upward: node v
+ * folds its own buffer, then each child's partial in the order it would send to them),
+ * times `scale`. */
+CC_API cc_status cc_reduce(const void* const* send, void* recv_root, int nranks, int root, size_t count,
+                    cc_dtype in_t, cc_dtype out_t, cc_op op, float scale, void* stream);
+
+/* Scatter (lecture 09 §3.2): recv[r] receives chunk r (chunk rule over `count`) of the
+ * root buffer `src`. Gather (§3.3): recv_root receives the concatenation of send[r]
+ * (chunk r of `count`) in rank order. Bit copies. */
+CC_API cc_status cc_scatter(const void* src, void* const* recv, int nranks, int root, size_t count,
+                     cc_dtype dtype, void* stream);
+CC_API cc_status cc_gather(const void* const* send, void* recv_root, int nranks, int root, size_t count,
+                    cc_dtype dtype, void* stream);
+
+/* ---- MoE expert parallelism (lecture 09 §6.4, §3.8, experiment 4 §7.4) ---------------
+ * Routing: expert_ids[r] ([tokens, topk] int32, device) receives, per token, the topk
+ * largest of logits[r] ([tokens, experts_total] fp32, device), ties to the lower id,
+ * larger first. topk in [1, 8], experts_total in [topk, 1024]. */
+CC_API cc_status cc_route_topk(const float* const* logits, int32_t* const* expert_ids, int nranks,
+                        int tokens, int experts_total, int topk, void* stream);
+
+/* Workspace bytes cc_alltoallv needs (device memory, caller-allocated, 256-byte aligned). */
+CC_API size_t cc_alltoallv_workspace_size(int nranks, int tokens, int topk, int experts_per_rank);
+
+/* AllToAllv dispatch (direction 0) / combine (direction 1).
+ * Expert e lives on rank e / experts_per_rank. Row (t, k) of source rank s is token t.
+ * Dispatch: send[s] is [tokens, row_bytes]; recv[d] receives every row routed to rank d,
+ *   as the concatenation over s = 0..N-1 of s's rows ordered by (local expert, t, k);
+ *   at most recv_capacity_rows rows are written per rank (rows beyond it are dropped;
+ *   cc_alltoallv_recv_counts tells the true counts).
+ * Combine: send[d] is rank d's [rows, row_bytes] buffer in dispatch order; recv[s] is
+ *   [tokens, topk, row_bytes] and receives each row back at slot [t][k].
+ * Both directions rebuild the routing table from expert_ids in `workspace`.
+ * row_bytes must be a positive multiple of 16. */
+CC_API cc_status cc_alltoallv(const void* const* send, void* const* recv, int nranks, size_t row_bytes,
+                       const int32_t* const* expert_ids, int tokens, int topk, int experts_per_rank,
+                       size_t recv_capacity_rows, int direction, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/* Copies the per-destination received row counts of the last cc_alltoallv that used
+ * `workspace` into recv_rows[0..nranks) (host or device memory), stream-ordered. */
+CC_API cc_status cc_alltoallv_recv_counts(const void* workspace, int nranks, int32_t* recv_rows,
+                                   void* stream);
+
+/* ---- DDP gradient buckets (lecture 09 §6.1; the from-scratch page's bucketing) --------
+ * Bucket assignment (host only): tensors are taken in reverse order of their index
+ * (the order backward produces them), never split; a new bucket starts when the next
+ * tensor would push a non-empty bucket past cap_bytes. Outputs: order[0..ntensors) =
+ * tensor ids in bucket order, bucket_start[0..nbuckets] = offsets into `order`,
+ * *nbuckets. bucket_start must have room for ntensors + 1 entries. */
+CC_API cc_status cc_bucket_assign(const size_t* numels, int ntensors, size_t elem_bytes, size_t cap_bytes,
+                           int32_t* order, int32_t* bucket_start, int32_t* nbuckets);
+
+/* Flatten: bucket[off_i .. off_i + numels[i]) = tensors[i], off_i = prefix sum, for the
+ * ntensors tensors in the given order. Unflatten is the inverse. Bit copies. */
+CC_API cc_status cc_bucket_flatten(const void* const* tensors, const size_t* numels, int ntensors,
+                            void* bucket, cc_dtype dtype, void* stream);
+CC_API cc_status cc_bucket_unflatten(const void* bucket, void* const* tensors, const size_t* numels,
+                              int ntensors, cc_dtype dtype, void* stream);
+
+/* Fused DDP step: for every bucket of cc_bucket_assign(numels, 4, cap_bytes), the result
+ * of flatten -> allreduce(algo, SUM, scale) -> unflatten, computed in one pass without
+ * the flat buffers: out[r * ntensors + i] receives tensor i of rank r.
+ *   grads / out: host arrays of nranks * ntensors device pointers (rank-major,
+ *   registration order); F32; in place allowed (out[j] == grads[j] for every j).
+ * The pointer and bucket tables travel as kernel parameters (no workspace); a tensor
+ * list longer than one launch can carry is split into several launches. */
+CC_API cc_status cc_bucket_allreduce(const void* const* grads, void* const* out, int nranks, int ntensors,
+                              const size_t* numels, size_t cap_bytes, cc_algo algo, float scale,
+                              void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CC_H_ */

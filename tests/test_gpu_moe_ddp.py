@@ -1,0 +1,137 @@
+"""GPU parity for the MoE alltoallv path and the DDP bucket path, against the oracle."""
+import numpy as np
+import pytest
+
+import synth
+from oracle import collectives as C
+from oracle import ddp, moe
+
+from .helpers import Guarded, bits, to_dev, to_host
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA GPU", allow_module_level=True)
+import collective_communication_primitives_rank_b200 as cc  # noqa: E402
+
+
+def _logits(seed, n, tokens, experts):
+    return [synth.normal_f32(seed, r, tokens * experts, stream=3).reshape(tokens, experts) for r in range(n)]
+
+
+@pytest.mark.parametrize("n,tokens,experts,topk", [(8, 1000, 64, 2), (2, 33, 5, 1), (4, 257, 1024, 8), (1, 7, 3, 3)])
+def test_route_topk_matches_oracle(n, tokens, experts, topk):
+    lg = _logits(1, n, tokens, experts)
+    lg[0][0, :4] = np.float32(1.5)     # ties: lower id first
+    lg[0][1, :] = np.float32(0.0)
+    lg[0][1, 3] = np.float32(-0.0)
+    ids = [torch.full((tokens, topk), -7, dtype=torch.int32, device="cuda") for _ in range(n)]
+    cc.cc_route_topk([to_dev(x) for x in lg], ids)
+    torch.cuda.synchronize()
+    for r in range(n):
+        assert np.array_equal(to_host(ids[r]), moe.route_topk(lg[r], topk))
+
+
+def _moe_case(n, tokens, hidden, epr, seed=2):
+    lg = _logits(seed, n, tokens, n * epr)
+    ids = [moe.route_topk(x, 2) for x in lg]
+    toks = [synth.to_bf16_bits(synth.normal_f32(seed, r, tokens * hidden, stream=4)).reshape(tokens, hidden)
+            for r in range(n)]
+    return ids, toks
+
+
+@pytest.mark.parametrize("n,tokens,hidden,epr", [(8, 300, 64, 8), (4, 1000, 8, 2), (3, 17, 16, 1), (1, 50, 8, 4),
+                                                 (8, 2048, 4096, 8)])
+def test_alltoallv_dispatch_and_combine_match_oracle(n, tokens, hidden, epr):
+    ids, toks = _moe_case(n, tokens, hidden, epr)
+    want, _ = moe.dispatch(toks, ids, epr)
+    cap = max(w.shape[0] for w in want) + 5
+    d_ids = [to_dev(i) for i in ids]
+    d_tok = [to_dev(t) for t in toks]
+    recv = [Guarded(cap * hidden, torch.bfloat16, shape=(cap, hidden)) for _ in range(n)]
+    ws = torch.empty(cc.cc_alltoallv_workspace_size(n, tokens, 2, epr) // 4 + 64, dtype=torch.int32, device="cuda")
+    cc.cc_alltoallv(d_tok, [g.t for g in recv], d_ids, epr, ws, direction=0)
+    counts = torch.zeros(n, dtype=torch.int32, device="cuda")
+    cc.cc_alltoallv_recv_counts(ws, n, counts)
+    back = [Guarded(tokens * 2 * hidden, torch.bfloat16, shape=(tokens, 2, hidden)) for _ in range(n)]
+    cc.cc_alltoallv([g.t for g in recv], [g.t for g in back], d_ids, epr, ws, direction=1)
+    torch.cuda.synchronize()
+    assert to_host(counts).tolist() == [w.shape[0] for w in want]
+    combined, _ = moe.combine(want, ids, epr)
+    for d in range(n):
+        got = to_host(recv[d].t)[:want[d].shape[0]]
+        assert np.array_equal(got, want[d]), f"dispatch rank {d}"
+        recv[d].check()
+    for s in range(n):
+        assert np.array_equal(to_host(back[s].t), combined[s]), f"combine rank {s}"
+        back[s].check()
+
+
+def test_alltoallv_capacity_drops_overflow_rows_only():
+    n, tokens, hidden, epr = 4, 200, 8, 2
+    ids, toks = _moe_case(n, tokens, hidden, epr, seed=9)
+    want, _ = moe.dispatch(toks, ids, epr)
+    cap = min(w.shape[0] for w in want) - 3
+    recv = [Guarded(cap * hidden, torch.bfloat16, shape=(cap, hidden)) for _ in range(n)]
+    ws = torch.empty(cc.cc_alltoallv_workspace_size(n, tokens, 2, epr) // 4 + 64, dtype=torch.int32, device="cuda")
+    cc.cc_alltoallv([to_dev(t) for t in toks], [g.t for g in recv], [to_dev(i) for i in ids], epr, ws)
+    counts = torch.zeros(n, dtype=torch.int32, device="cuda")
+    cc.cc_alltoallv_recv_counts(ws, n, counts)
+    torch.cuda.synchronize()
+    assert to_host(counts).tolist() == [w.shape[0] for w in want]
+    for d in range(n):
+        assert np.array_equal(to_host(recv[d].t), want[d][:cap])
+        recv[d].check()
+
+
+# ---- DDP buckets ----------------------------------------------------------------------------------------
+
+def _small_model(n, seed=1, layers=2, d=64, ffn=256, vocab=500):
+    shapes = synth.transformer_grad_shapes(layers, d, ffn, vocab)
+    grads = [[synth.normal_f32(seed, r, synth.numel(s), 1e-3, stream=i).reshape(s)
+              for i, (_, s) in enumerate(shapes)] for r in range(n)]
+    return shapes, grads
+
+
+@pytest.mark.parametrize("algo", ["ring", "tree"])
+@pytest.mark.parametrize("n,cap", [(8, 40_000), (3, 100_000), (8, 25 * 1024 * 1024), (16, 7_000)])
+def test_fused_bucket_allreduce_matches_oracle(algo, n, cap):
+    shapes, grads = _small_model(n)
+    want, _ = ddp.ddp_allreduce(grads, cap_bytes=cap, algo=algo)
+    d_in = [[to_dev(g) for g in row] for row in grads]
+    out = [[Guarded(g.size, torch.float32, shape=g.shape) for g in row] for row in grads]
+    cc.cc_bucket_allreduce(d_in, [[o.t for o in row] for row in out], cap_bytes=cap, algo=algo)
+    cc.cc_bucket_allreduce(d_in, d_in, cap_bytes=cap, algo=algo)  # in place
+    torch.cuda.synchronize()
+    for r in range(n):
+        for i in range(len(shapes)):
+            assert np.array_equal(bits(to_host(out[r][i].t)), bits(want[r][i])), f"rank {r} tensor {i}"
+            assert np.array_equal(bits(to_host(d_in[r][i])), bits(want[r][i])), f"in place rank {r} tensor {i}"
+            out[r][i].check()
+
+
+def test_flatten_allreduce_unflatten_equals_fused():
+    n, cap = 8, 60_000
+    shapes, grads = _small_model(n, seed=4)
+    want, _ = ddp.ddp_allreduce(grads, cap_bytes=cap)
+    buckets = cc.cc_bucket_assign([g.size for g in grads[0]], 4, cap)
+    assert buckets == ddp.assign_buckets([g.size for g in grads[0]], 4, cap)
+    d_in = [[to_dev(g) for g in row] for row in grads]
+    outs = [[torch.empty_like(t) for t in row] for row in d_in]
+    for members in buckets:
+        size = sum(grads[0][i].size for i in members)
+        flats = [Guarded(size, torch.float32) for _ in range(n)]
+        for r in range(n):
+            cc.cc_bucket_flatten([d_in[r][i] for i in members], flats[r].t)
+        red = [torch.empty(size, device="cuda") for _ in range(n)]
+        cc.cc_allreduce([f.t for f in flats], red, scale=1.0 / n)
+        for r in range(n):
+            cc.cc_bucket_unflatten(red[r], [outs[r][i] for i in members])
+        torch.cuda.synchronize()
+        for r in range(n):
+            flats[r].check()
+            assert np.array_equal(to_host(flats[r].t), ddp.flatten(grads[r], members))
+    for r in range(n):
+        for i in range(len(shapes)):
+            assert np.array_equal(bits(to_host(outs[r][i])), bits(want[r][i]))

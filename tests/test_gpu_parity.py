@@ -1,0 +1,218 @@
+"""GPU parity: libcc (through the C ABI, via the binding) against the oracle, element by
+element, on seeded inputs. Bit-exact throughout: integer sums, every data movement, and
+floating-point folds in the schedule's prescribed order."""
+import numpy as np
+import pytest
+
+import synth
+from oracle import collectives as C
+from oracle import layout as L
+
+from .helpers import Guarded, bits, misaligned, to_dev, to_host, torch_dtype
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA GPU", allow_module_level=True)
+import collective_communication_primitives_rank_b200 as cc  # noqa: E402
+
+
+def _inputs(kind, n, count, seed=3):
+    if kind == "f32":
+        return [synth.uniform_f32(seed, r, count) for r in range(n)]
+    if kind == "spread":  # magnitudes 2^-20..2^20: the bracketing shows in the rounding
+        return [(synth.uniform_f32(seed, r, count) *
+                 np.exp2(synth.int32_uniform(seed, r, count, -20, 20, stream=1)).astype(np.float32)).astype(np.float32)
+                for r in range(n)]
+    if kind == "i32":
+        return [synth.int32_uniform(seed, r, count, -2**31, 2**31 - 1) for r in range(n)]
+    if kind == "bf16":
+        return [synth.to_bf16_bits(synth.normal_f32(seed, r, count, 1e-2)) for r in range(n)]
+    raise ValueError(kind)
+
+
+_IN = {"f32": "f32", "spread": "f32", "i32": "i32", "bf16": "bf16"}
+
+
+def _out_dtype(kind):
+    return torch.int32 if kind == "i32" else torch.float32
+
+
+def _assert_same(got: np.ndarray, want: np.ndarray, what=""):
+    g, w = bits(got), bits(want)
+    if not np.array_equal(g, w):
+        bad = np.flatnonzero(g != w)
+        raise AssertionError(f"{what}: {bad.size} of {w.size} elements differ, first at {bad[:5]}: "
+                             f"got {got[bad[:5]]} want {want[bad[:5]]}")
+
+
+# ---- config 1: N = 4, 4096 elements, fp32 uniform[-1, 1] and int32 uniform[-1000, 1000] ------------------
+
+@pytest.mark.parametrize("kind", ["f32", "i32"])
+def test_config1_allreduce_reduce_scatter_allgather(kind):
+    n, count = 4, 4096
+    xs = [synth.uniform_f32(1, r, count) for r in range(n)] if kind == "f32" else \
+        [synth.int32_uniform(1, r, count, -1000, 1000) for r in range(n)]
+    send = [to_dev(x) for x in xs]
+    want_ar, _ = C.ring_allreduce(xs, in_dtype=_IN[kind])
+    out = [Guarded(count, _out_dtype(kind)) for _ in range(n)]
+    cc.cc_allreduce(send, [o.t for o in out])
+    want_rs, _ = C.ring_reduce_scatter(xs, in_dtype=_IN[kind])
+    rs = [Guarded(count // n, _out_dtype(kind)) for _ in range(n)]
+    cc.cc_reduce_scatter(send, [o.t for o in rs])
+    ag = [Guarded(count, _out_dtype(kind)) for _ in range(n)]
+    cc.cc_allgather([o.t for o in rs], [o.t for o in ag])
+    torch.cuda.synchronize()
+    for r in range(n):
+        _assert_same(to_host(out[r].t), want_ar[r], f"allreduce rank {r}")
+        _assert_same(to_host(rs[r].t), want_rs[r], f"reduce_scatter rank {r}")
+        _assert_same(to_host(ag[r].t), want_ar[r], f"allgather(reduce_scatter) rank {r}")
+        for g in (out[r], rs[r], ag[r]):
+            g.check()
+
+
+# ---- allreduce across shapes, dtypes, ops and both algorithms -------------------------------------------
+
+AR_CASES = [(1, 37), (2, 4096), (3, 1001), (4, 5), (5, 12345), (8, 8 * 1024 * 4 + 13), (13, 777),
+            (16, 65536), (33, 2000), (64, 64 * 100 + 63), (64, 40), (7, 3)]
+
+
+@pytest.mark.parametrize("n,count", AR_CASES)
+@pytest.mark.parametrize("algo", ["ring", "tree"])
+@pytest.mark.parametrize("kind", ["spread", "i32", "bf16"])
+def test_allreduce_matches_oracle(n, count, algo, kind):
+    xs = _inputs(kind, n, count)
+    fn = C.ring_allreduce if algo == "ring" else C.tree_allreduce
+    scale = 1.0 if kind == "i32" else 1.0 / n
+    want, _ = fn(xs, in_dtype=_IN[kind], scale=scale)
+    out = [Guarded(count, _out_dtype(kind)) for _ in range(n)]
+    cc.cc_allreduce([to_dev(x) for x in xs], [o.t for o in out], algo=algo, scale=scale)
+    torch.cuda.synchronize()
+    for r in range(n):
+        _assert_same(to_host(out[r].t), want[r], f"{algo} {kind} N={n} rank {r}")
+        out[r].check()
+
+
+@pytest.mark.parametrize("op", ["max", "min", "prod"])
+@pytest.mark.parametrize("algo", ["ring", "tree"])
+@pytest.mark.parametrize("kind", ["spread", "i32"])
+def test_other_ops_match_oracle(op, algo, kind):
+    n, count = 6, 999
+    xs = _inputs(kind, n, count, seed=8)
+    if op == "prod" and kind == "spread":
+        xs = [(1.0 + 0.01 * x).astype(np.float32) for x in _inputs("f32", n, count, seed=8)]
+    xs[0][:7] = np.array([0.0, -0.0, 0.0, -0.0, 0, 0, 0], dtype=xs[0].dtype)
+    xs[1][:7] = np.array([-0.0, 0.0, -0.0, -0.0, 0, 0, 0], dtype=xs[0].dtype)
+    fn = C.ring_allreduce if algo == "ring" else C.tree_allreduce
+    want, _ = fn(xs, op=op, in_dtype=_IN[kind])
+    out = [torch.empty(count, dtype=_out_dtype(kind), device="cuda") for _ in range(n)]
+    cc.cc_allreduce([to_dev(x) for x in xs], out, op=op, algo=algo)
+    torch.cuda.synchronize()
+    for r in range(n):
+        _assert_same(to_host(out[r]), want[r], f"{op} {algo} rank {r}")
+
+
+def test_allreduce_in_place_and_misaligned():
+    n, count = 8, 10_003
+    xs = _inputs("spread", n, count)
+    want, _ = C.ring_allreduce(xs, scale=0.125)
+    buf = [to_dev(x) for x in xs]
+    cc.cc_allreduce(buf, buf, scale=0.125)
+    mis = [misaligned(x) for x in xs]
+    mout = [misaligned(np.zeros(count, np.float32)) for _ in range(n)]
+    cc.cc_allreduce(mis, mout, scale=0.125)
+    torch.cuda.synchronize()
+    for r in range(n):
+        _assert_same(to_host(buf[r]), want[r], "in place")
+        _assert_same(to_host(mout[r]), want[r], "misaligned")
+
+
+def test_allreduce_empty_is_a_no_op():
+    t = [torch.empty(0, device="cuda") for _ in range(4)]
+    cc.cc_allreduce(t, t)
+    torch.cuda.synchronize()
+
+
+# ---- reduce-scatter / allgather ------------------------------------------------------------------------
+
+@pytest.mark.parametrize("n,count", [(2, 9), (4, 4096), (5, 1003), (8, 8 * 4096), (8, 8 * 4096 + 5), (3, 2),
+                                     (16, 160), (64, 64 * 33 + 17)])
+@pytest.mark.parametrize("kind", ["spread", "i32", "bf16"])
+def test_reduce_scatter_and_allgather_match_oracle(n, count, kind):
+    xs = _inputs(kind, n, count)
+    scale = 1.0 if kind == "i32" else 0.25
+    want, _ = C.ring_reduce_scatter(xs, in_dtype=_IN[kind], scale=scale)
+    lens = [b - a for a, b in L.chunk_bounds(count, n)]
+    rs = [Guarded(ln, _out_dtype(kind)) for ln in lens]
+    cc.cc_reduce_scatter([to_dev(x) for x in xs], [g.t for g in rs], scale=scale)
+    ag = [Guarded(count, _out_dtype(kind)) for _ in range(n)]
+    cc.cc_allgather([g.t for g in rs], [g.t for g in ag])
+    want_ag, _ = C.ring_allgather(want, count=count)
+    want_ar, _ = C.ring_allreduce(xs, in_dtype=_IN[kind], scale=scale)
+    torch.cuda.synchronize()
+    for r in range(n):
+        _assert_same(to_host(rs[r].t), want[r], f"RS shard {r}")
+        _assert_same(to_host(ag[r].t), want_ag[r], f"AG rank {r}")
+        _assert_same(to_host(ag[r].t), want_ar[r], f"AG(RS) == AR rank {r}")
+        rs[r].check()
+        ag[r].check()
+
+
+def test_allgather_misaligned_shards_and_bf16_width():
+    n, count = 4, 4 * 1000 + 3
+    shards = [synth.to_bf16_bits(synth.normal_f32(2, r, b - a)) for r, (a, b) in enumerate(L.chunk_bounds(count, n))]
+    want, _ = C.ring_allgather(shards, count=count)
+    out = [Guarded(count, torch.bfloat16, misalign=1) for _ in range(n)]
+    cc.cc_allgather([misaligned(s) for s in shards], [g.t for g in out])
+    torch.cuda.synchronize()
+    for r in range(n):
+        _assert_same(to_host(out[r].t), want[r])
+        out[r].check()
+
+
+# ---- broadcast, reduce, scatter, gather ------------------------------------------------------------------
+
+@pytest.mark.parametrize("n,root,count", [(1, 0, 10), (4, 0, 4099), (7, 3, 100_000), (64, 63, 333)])
+def test_broadcast(n, root, count):
+    x = synth.uniform_f32(5, 0, count)
+    want, _ = C.broadcast(x, n, root)
+    src = to_dev(x)
+    out = [Guarded(count, torch.float32) for _ in range(n)]
+    cc.cc_broadcast(src, [g.t for g in out], root)
+    inplace = [src if r == root else torch.empty(count, device="cuda") for r in range(n)]
+    cc.cc_broadcast(src, inplace, root)
+    torch.cuda.synchronize()
+    for r in range(n):
+        _assert_same(to_host(out[r].t), want[r])
+        _assert_same(to_host(inplace[r]), want[r])
+        out[r].check()
+
+
+@pytest.mark.parametrize("n,root", [(1, 0), (4, 0), (8, 5), (13, 12), (64, 17)])
+@pytest.mark.parametrize("kind", ["spread", "i32"])
+def test_reduce_to_root(n, root, kind):
+    count = 2049
+    xs = _inputs(kind, n, count, seed=12)
+    want, _ = C.reduce(xs, root, in_dtype=_IN[kind])
+    out = Guarded(count, _out_dtype(kind))
+    cc.cc_reduce([to_dev(x) for x in xs], out.t, root)
+    torch.cuda.synchronize()
+    _assert_same(to_host(out.t), want)
+    out.check()
+
+
+@pytest.mark.parametrize("n,count", [(4, 4), (4, 4099), (9, 100_001), (64, 70)])
+def test_scatter_and_gather(n, count):
+    x = synth.int32_uniform(6, 0, count, -5, 5)
+    parts, _ = C.scatter(x, n, root=n - 1)
+    out = [Guarded(p.size, torch.int32) for p in parts]
+    cc.cc_scatter(to_dev(x), [g.t for g in out], n - 1)
+    back = Guarded(count, torch.int32)
+    cc.cc_gather([g.t for g in out], back.t, n - 1)
+    torch.cuda.synchronize()
+    for r in range(n):
+        _assert_same(to_host(out[r].t), parts[r])
+        out[r].check()
+    _assert_same(to_host(back.t), x)
+    back.check()
