@@ -1,0 +1,311 @@
+"""Benchmark: the fused DDP gradient-bucket allreduce of libcc on B200.
+
+Workload (one step): N = 8 simulated ranks, each holding the fp32 gradients of a 12-layer
+d = 768 transformer (147 tensors, 109,632,000 elements = 438.5 MB per rank, values
+normal(0, 1e-3)), packed into 25 MiB buckets (17) in reverse registration order, ring
+allreduce of every bucket with the 1/N scale, unflattened: one fused kernel launch
+(cc_bucket_allreduce), inputs and outputs resident in HBM.
+
+Metric: allreduce effective HBM GB/s = (N·T in + N·T out) / step time, T = 438.5 MB,
+plus its share of ~8 TB/s and elements/s (N·count / step time).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--gpus N > 1 runs under torchrun, one process per GPU, each with its own replica of the
+workload (independent problems: weak scaling); time is the max over ranks.
+--impl reference times the oracle (the plain CPU message-passing simulator) on a bounded
+sample of the same workload.
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "allreduce effective HBM GB/s (N·T in + N·T out) and % of ~8 TB/s; elems/s"
+NOMINAL_HBM_GBS = 8000.0
+N_SIM = 8
+CAP = 25 * 1024 * 1024
+SEED = 0x5EED
+PROFILE = os.path.join(ROOT, "profiles", "bucket_allreduce_ddp.txt")
+KERNEL_SRC = os.path.join(ROOT, "collective_communication_primitives_rank_b200", "csrc", "k_reduce.cu")
+
+
+def workload_desc(layers):
+    return (f"ddp_bucket_allreduce: N={N_SIM} simulated ranks on one GPU, fp32 gradients of a "
+            f"{layers}-layer d=768 ffn=3072 vocab=32000 transformer, 25 MiB buckets in reverse "
+            f"registration order, ring allreduce with scale 1/{N_SIM}, fused flatten/unflatten")
+
+
+def measured_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def profile_traffic():
+    """DRAM bytes per launch of the fused kernel from the committed ncu summary, or None
+    when the kernel source changed since the counters were taken."""
+    try:
+        lines = dict(l.split(":", 1) for l in open(PROFILE).read().splitlines() if ":" in l)
+        src = hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()
+        if lines.get("kernel_source_sha256", "").strip() != src:
+            return None
+        return int(float(lines["dram_bytes_per_launch_full_workload"].strip()))
+    except Exception:
+        return None
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for line in (getattr(self, "out", "") or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) >= 9:
+                rows.append(f)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": float(rows[0][2]),
+                "samples": len(rows), "reasons": reasons}
+
+
+def build_workload(torch, layers, seed, pinned_inputs):
+    import synth
+    shapes = synth.transformer_grad_shapes(layers=layers)
+    numels = [synth.numel(s) for _, s in shapes]
+    total = sum(numels)
+    offs = [0]
+    for n in numels:
+        offs.append(offs[-1] + n)
+
+    def views(flat):
+        return [flat[offs[i]:offs[i + 1]].view(shapes[i][1]) for i in range(len(numels))]
+
+    host = []
+    for r in range(N_SIM):
+        h = torch.empty(total, dtype=torch.float32, pin_memory=pinned_inputs)
+        h.numpy()[:] = synth.normal_f32(seed, r, total, 1e-3)
+        host.append(h)
+    dev_in = [h.to("cuda", non_blocking=False) for h in host]
+    dev_out = [torch.empty_like(d) for d in dev_in]
+    return dict(shapes=shapes, numels=numels, total=total, host=host, views=views,
+                dev_in=[views(d) for d in dev_in], dev_out=[views(d) for d in dev_out],
+                dev_in_flat=dev_in, dev_out_flat=dev_out)
+
+
+def oracle_sample_seconds(numels, rank_arrays, base, nbuckets):
+    """The oracle (message-passing simulator) on the first `nbuckets` buckets of the same
+    host data; rank_arrays[r] holds rank r's flat gradients from element `base` on.
+    Returns (seconds, bytes of N·T in + N·T out covered, elements per rank covered)."""
+    import numpy as np
+    from oracle import ddp
+    from oracle.collectives import ring_allreduce
+    buckets = ddp.assign_buckets(numels)[:nbuckets]
+    offs = np.cumsum([0] + list(numels)) - base
+    t0 = time.perf_counter()
+    moved = 0
+    for members in buckets:
+        flats = [np.concatenate([a[offs[i]:offs[i + 1]] for i in members]) for a in rank_arrays]
+        ring_allreduce(flats, scale=1.0 / N_SIM)
+        moved += 2 * N_SIM * flats[0].nbytes
+    return time.perf_counter() - t0, moved, sum(sum(numels[i] for i in m) for m in buckets)
+
+
+def sample_range(numels, nbuckets):
+    """[lo, hi) of the flat per-rank buffer that the first nbuckets buckets cover."""
+    import numpy as np
+    from oracle import ddp
+    offs = np.cumsum([0] + list(numels))
+    members = [i for m in ddp.assign_buckets(numels)[:nbuckets] for i in m]
+    return int(min(offs[i] for i in members)), int(max(offs[i + 1] for i in members))
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import synth
+    shapes = synth.transformer_grad_shapes(layers=args.layers)
+    numels = [synth.numel(s) for _, s in shapes]
+    lo, hi = sample_range(numels, 1)
+    arrays = [synth.normal_f32(SEED, r, hi - lo, 1e-3, start=lo) for r in range(N_SIM)]
+    times = []
+    moved = elems = 0
+    for step in range(args.warmup + args.steps):
+        dt, moved, elems = oracle_sample_seconds(numels, arrays, lo, 1)
+        if step >= args.warmup:
+            times.append(dt)
+    t = sum(times) / len(times)
+    v = moved / t / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": workload_desc(args.layers), "sample": "bucket 0 of 17 per step"},
+            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": f"bucket 0 ({elems} fp32 per rank, {N_SIM} ranks) per step"},
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--layers", type=int, default=12, help="model depth (12 = the workload; smaller for profiling)")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--oracle-buckets", type=int, default=8)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    import collective_communication_primitives_rank_b200 as cc
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    w = build_workload(torch, args.layers, SEED + 1000 * rank, pinned_inputs=True)
+    bytes_step = 2 * N_SIM * w["total"] * 4
+    stream = torch.cuda.current_stream()
+
+    def step():
+        cc.cc_bucket_allreduce(w["dev_in"], w["dev_out"], cap_bytes=CAP, scale=1.0 / N_SIM)
+
+    launches_per_step = -(-len(w["numels"]) // 192)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    barrier()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Clocks(local) as clk:
+        barrier()
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        end.record(stream)
+        barrier()
+    ms = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    value = world * bytes_step / (ms_step * 1e-3) / 1e9
+
+    # end to end through the host-buffer entry point: H2D + fused allreduce + D2H per step
+    host_out = [torch.empty(w["total"], dtype=torch.float32, pin_memory=True) for _ in range(N_SIM)]
+    h_in = [w["views"](h) for h in w["host"]]
+    h_out = [w["views"](h) for h in host_out]
+
+    def e2e_step():
+        cc.cc_bucket_allreduce_host(h_in, h_out, w["dev_in"], w["dev_out"], cap_bytes=CAP, scale=1.0 / N_SIM)
+
+    e2e_step()
+    barrier()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e2.record(stream)
+    barrier()
+    ems = s2.elapsed_time(e2)
+    if world > 1:
+        t = torch.tensor([ems], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ems = float(t.item())
+    e2e_value = world * bytes_step / (ems / args.e2e_steps * 1e-3) / 1e9
+
+    peak, peak_kind = measured_peak()
+    achieved = bytes_step / launches_per_step / (ms_step / launches_per_step * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "pct_of_8TBps": 100.0 * value / world / NOMINAL_HBM_GBS,
+        "elems_per_s": world * N_SIM * w["total"] / (ms_step * 1e-3),
+        "config": {"workload": workload_desc(args.layers), "sim_ranks": N_SIM, "tensors": len(w["numels"]),
+                   "elems_per_rank": w["total"], "bytes_per_step": bytes_step, "buckets": 17 if args.layers == 12 else None,
+                   "l2": "inputs (3.5 GB) larger than L2 (126 MB); no flush", "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_kind": peak_kind, "traffic": profile_traffic() if args.layers == 12 else None,
+                     "kernel": "bucket_allreduce_kernel<ring>"},
+        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": N_SIM * w["total"] * 4,
+                "d2h_bytes_per_step": N_SIM * w["total"] * 4},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, moved, elems = oracle_sample_seconds(w["numels"], [h.numpy() for h in w["host"]], 0,
+                                                 args.oracle_buckets)
+        line["cpu_baseline"] = {"value": moved / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                "sample": f"first {args.oracle_buckets} of 17 buckets ({elems} fp32 per rank, "
+                                          f"{N_SIM} ranks), {dt:.1f} s single-threaded"}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -50,6 +50,7 @@ _SIGS = {
     "cc_bucket_flatten": (_i, [_PP, _SZP, _i, _vp, _i, _vp]),
     "cc_bucket_unflatten": (_i, [_vp, _PP, _SZP, _i, _i, _vp]),
     "cc_bucket_allreduce": (_i, [_PP, _PP, _i, _i, _SZP, _sz, _i, _f, _vp]),
+    "cc_bucket_allreduce_host": (_i, [_PP, _PP, _PP, _PP, _i, _i, _SZP, _sz, _i, _f, _vp]),
 }
 
 
@@ -324,6 +325,34 @@ def cc_bucket_allreduce(grads, out, *, cap_bytes: int = 25 * 1024 * 1024, algo="
     flat_out = [t for row in out for t in row]
     _check(lib.cc_bucket_allreduce(_ptrs(flat_in), _ptrs(flat_out), n, nt, _sizes([t.numel() for t in grads[0]]),
                                    cap_bytes, _ALGOS[algo], float(scale), _stream(stream)), "cc_bucket_allreduce")
+
+
+def cc_bucket_allreduce_host(host_grads, host_out, dev_grads, dev_out, *, cap_bytes: int = 25 * 1024 * 1024,
+                             algo="ring", scale=None, stream=None) -> None:
+    """The fused DDP step on host-resident gradients: host -> device copies, the fused
+    allreduce, device -> host copies, all on one stream. host_* are CPU tensors (pin them
+    for asynchronous copies); dev_* are CUDA staging tensors of the same shapes."""
+    torch = _torch()
+    n, nt = _ranks(host_grads, "cc_bucket_allreduce_host"), len(host_grads[0])
+    for grid in (host_out, dev_grads, dev_out):
+        if len(grid) != n or any(len(row) != nt for row in grid):
+            raise ValueError("cc_bucket_allreduce_host: all four tables must be [nranks][ntensors]")
+    for i in range(nt):
+        ts = [g[r][i] for g in (host_grads, host_out, dev_grads, dev_out) for r in range(n)]
+        _same(ts, host_grads[0][i].numel(), torch.float32, f"cc_bucket_allreduce_host tensor {i}")
+    for r in range(n):
+        for i in range(nt):
+            if host_grads[r][i].is_cuda or host_out[r][i].is_cuda:
+                raise ValueError("cc_bucket_allreduce_host: host tables must hold CPU tensors")
+            if not (host_grads[r][i].is_contiguous() and host_out[r][i].is_contiguous()):
+                raise ValueError("cc_bucket_allreduce_host: contiguous tensors only")
+    scale = 1.0 / n if scale is None else scale
+    hp = lambda grid: (ctypes.c_void_p * (n * nt))(*[t.data_ptr() for row in grid for t in row])
+    _check(lib.cc_bucket_allreduce_host(hp(host_grads), hp(host_out),
+                                        _ptrs([t for row in dev_grads for t in row]),
+                                        _ptrs([t for row in dev_out for t in row]), n, nt,
+                                        _sizes([t.numel() for t in host_grads[0]]), cap_bytes, _ALGOS[algo],
+                                        float(scale), _stream(stream)), "cc_bucket_allreduce_host")
 
 
 def raw_call(name: str, *args) -> int:

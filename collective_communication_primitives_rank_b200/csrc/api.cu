@@ -70,13 +70,13 @@ cc_status cc_chunk(size_t count, int nranks, int c, size_t* start, size_t* len) 
 
 cc_status cc_allreduce(const void* const* send, void* const* recv, int nranks, size_t count, cc_dtype in_t,
                        cc_dtype out_t, cc_op op, cc_algo algo, float scale, void* stream) {
-  if (!valid_ranks(nranks) || !all_nonnull(send, nranks) || !all_nonnull((const void* const*)recv, nranks))
-    return CC_ERR_INVALID_ARG;
+  if (!valid_ranks(nranks) || !send || !recv) return CC_ERR_INVALID_ARG;
   if (cc_status st = check_reduce(in_t, out_t, op, scale)) return st;
   if (algo != CC_ALGO_RING && algo != CC_ALGO_TREE) return CC_ERR_INVALID_ARG;
+  if (count == 0) return CC_OK;
+  if (!all_nonnull(send, nranks) || !all_nonnull((const void* const*)recv, nranks)) return CC_ERR_INVALID_ARG;
   for (int r = 0; r < nranks; ++r)
     if (recv[r] == send[r] && dtype_bytes(in_t) != dtype_bytes(out_t)) return CC_ERR_INVALID_ARG;
-  if (count == 0) return CC_OK;
   return cuda_status(launch_reduce(send, recv, nranks, nranks, count, in_t, op,
                                    algo == CC_ALGO_RING ? kFoldRing : kFoldTree, kAllReduce, 0, scale,
                                    as_stream(stream)));
@@ -84,22 +84,27 @@ cc_status cc_allreduce(const void* const* send, void* const* recv, int nranks, s
 
 cc_status cc_reduce_scatter(const void* const* send, void* const* recv, int nranks, size_t count, cc_dtype in_t,
                             cc_dtype out_t, cc_op op, cc_algo algo, float scale, void* stream) {
-  if (!valid_ranks(nranks) || !all_nonnull(send, nranks) || !all_nonnull((const void* const*)recv, nranks))
-    return CC_ERR_INVALID_ARG;
+  if (!valid_ranks(nranks) || !send || !recv) return CC_ERR_INVALID_ARG;
   if (cc_status st = check_reduce(in_t, out_t, op, scale)) return st;
   if (algo == CC_ALGO_TREE) return CC_ERR_UNSUPPORTED;
   if (algo != CC_ALGO_RING) return CC_ERR_INVALID_ARG;
   if (count == 0) return CC_OK;
+  if (!all_nonnull(send, nranks)) return CC_ERR_INVALID_ARG;
+  for (int c = 0; c < nranks; ++c) {
+    size_t a, len;
+    chunk_bounds(count, nranks, c, a, len);
+    if (len && !recv[c]) return CC_ERR_INVALID_ARG;  // an empty shard may be null
+  }
   return cuda_status(launch_reduce(send, recv, nranks, nranks, count, in_t, op, kFoldRing, kReduceScatter, 0,
                                    scale, as_stream(stream)));
 }
 
 cc_status cc_reduce(const void* const* send, void* recv_root, int nranks, int root, size_t count, cc_dtype in_t,
                     cc_dtype out_t, cc_op op, float scale, void* stream) {
-  if (!valid_ranks(nranks) || !all_nonnull(send, nranks) || !recv_root || root < 0 || root >= nranks)
-    return CC_ERR_INVALID_ARG;
+  if (!valid_ranks(nranks) || !send || root < 0 || root >= nranks) return CC_ERR_INVALID_ARG;
   if (cc_status st = check_reduce(in_t, out_t, op, scale)) return st;
   if (count == 0) return CC_OK;
+  if (!all_nonnull(send, nranks) || !recv_root) return CC_ERR_INVALID_ARG;
   void* dst[1] = {recv_root};
   return cuda_status(launch_reduce(send, dst, 1, nranks, count, in_t, op, kFoldBinomial, kReduceRoot, root, scale,
                                    as_stream(stream)));
@@ -107,14 +112,14 @@ cc_status cc_reduce(const void* const* send, void* recv_root, int nranks, int ro
 
 cc_status cc_allgather(const void* const* send, void* const* recv, int nranks, size_t count, cc_dtype dtype,
                        void* stream) {
-  if (!valid_ranks(nranks) || !all_nonnull(send, nranks) || !all_nonnull((const void* const*)recv, nranks) ||
-      !valid_dtype(dtype))
-    return CC_ERR_INVALID_ARG;
+  if (!valid_ranks(nranks) || !send || !recv || !valid_dtype(dtype)) return CC_ERR_INVALID_ARG;
   if (count == 0) return CC_OK;
+  if (!all_nonnull((const void* const*)recv, nranks)) return CC_ERR_INVALID_ARG;
   std::vector<CopyEntry> e(nranks);
   for (int c = 0; c < nranks; ++c) {
     size_t a, len;
     chunk_bounds(count, nranks, c, a, len);
+    if (len && !send[c]) return CC_ERR_INVALID_ARG;  // an empty shard may be null
     e[c] = CopyEntry{send[c], nullptr, len, a};
   }
   return cuda_status(launch_copy(e.data(), nranks, recv, nranks, true, -1, dtype_bytes(dtype), as_stream(stream)));
@@ -122,10 +127,10 @@ cc_status cc_allgather(const void* const* send, void* const* recv, int nranks, s
 
 cc_status cc_broadcast(const void* src, void* const* recv, int nranks, int root, size_t count, cc_dtype dtype,
                        void* stream) {
-  if (!valid_ranks(nranks) || !src || !all_nonnull((const void* const*)recv, nranks) || !valid_dtype(dtype) ||
-      root < 0 || root >= nranks)
+  if (!valid_ranks(nranks) || !recv || !valid_dtype(dtype) || root < 0 || root >= nranks)
     return CC_ERR_INVALID_ARG;
   if (count == 0) return CC_OK;
+  if (!src || !all_nonnull((const void* const*)recv, nranks)) return CC_ERR_INVALID_ARG;
   CopyEntry e{src, nullptr, count, 0};
   const int skip = recv[root] == src ? root : -1;
   return cuda_status(launch_copy(&e, 1, recv, nranks, true, skip, dtype_bytes(dtype), as_stream(stream)));
@@ -133,15 +138,16 @@ cc_status cc_broadcast(const void* src, void* const* recv, int nranks, int root,
 
 cc_status cc_scatter(const void* src, void* const* recv, int nranks, int root, size_t count, cc_dtype dtype,
                      void* stream) {
-  if (!valid_ranks(nranks) || !src || !all_nonnull((const void* const*)recv, nranks) || !valid_dtype(dtype) ||
-      root < 0 || root >= nranks)
+  if (!valid_ranks(nranks) || !recv || !valid_dtype(dtype) || root < 0 || root >= nranks)
     return CC_ERR_INVALID_ARG;
   if (count == 0) return CC_OK;
+  if (!src) return CC_ERR_INVALID_ARG;
   const size_t es = dtype_bytes(dtype);
   std::vector<CopyEntry> e(nranks);
   for (int c = 0; c < nranks; ++c) {
     size_t a, len;
     chunk_bounds(count, nranks, c, a, len);
+    if (len && !recv[c]) return CC_ERR_INVALID_ARG;
     e[c] = CopyEntry{static_cast<const char*>(src) + a * es, recv[c], len, 0};
   }
   return cuda_status(launch_copy(e.data(), nranks, nullptr, 0, false, -1, es, as_stream(stream)));
@@ -149,14 +155,15 @@ cc_status cc_scatter(const void* src, void* const* recv, int nranks, int root, s
 
 cc_status cc_gather(const void* const* send, void* recv_root, int nranks, int root, size_t count, cc_dtype dtype,
                     void* stream) {
-  if (!valid_ranks(nranks) || !all_nonnull(send, nranks) || !recv_root || !valid_dtype(dtype) || root < 0 ||
-      root >= nranks)
+  if (!valid_ranks(nranks) || !send || !valid_dtype(dtype) || root < 0 || root >= nranks)
     return CC_ERR_INVALID_ARG;
   if (count == 0) return CC_OK;
+  if (!recv_root) return CC_ERR_INVALID_ARG;
   std::vector<CopyEntry> e(nranks);
   for (int c = 0; c < nranks; ++c) {
     size_t a, len;
     chunk_bounds(count, nranks, c, a, len);
+    if (len && !send[c]) return CC_ERR_INVALID_ARG;
     e[c] = CopyEntry{send[c], recv_root, len, a};
   }
   return cuda_status(launch_copy(e.data(), nranks, nullptr, 0, false, -1, dtype_bytes(dtype), as_stream(stream)));
@@ -237,11 +244,11 @@ cc_status cc_bucket_assign(const size_t* numels, int ntensors, size_t elem_bytes
 
 cc_status cc_bucket_flatten(const void* const* tensors, const size_t* numels, int ntensors, void* bucket,
                             cc_dtype dtype, void* stream) {
-  if (ntensors < 0 || !bucket || !valid_dtype(dtype) || (ntensors > 0 && (!numels || !all_nonnull(tensors, ntensors))))
-    return CC_ERR_INVALID_ARG;
+  if (ntensors < 0 || !valid_dtype(dtype) || (ntensors > 0 && (!numels || !tensors))) return CC_ERR_INVALID_ARG;
   std::vector<CopyEntry> e(ntensors);
   size_t off = 0;
   for (int i = 0; i < ntensors; ++i) {
+    if (numels[i] && (!tensors[i] || !bucket)) return CC_ERR_INVALID_ARG;
     e[i] = CopyEntry{tensors[i], bucket, numels[i], off};
     off += numels[i];
   }
@@ -250,13 +257,12 @@ cc_status cc_bucket_flatten(const void* const* tensors, const size_t* numels, in
 
 cc_status cc_bucket_unflatten(const void* bucket, void* const* tensors, const size_t* numels, int ntensors,
                               cc_dtype dtype, void* stream) {
-  if (ntensors < 0 || !bucket || !valid_dtype(dtype) ||
-      (ntensors > 0 && (!numels || !all_nonnull((const void* const*)tensors, ntensors))))
-    return CC_ERR_INVALID_ARG;
+  if (ntensors < 0 || !valid_dtype(dtype) || (ntensors > 0 && (!numels || !tensors))) return CC_ERR_INVALID_ARG;
   const size_t es = dtype_bytes(dtype);
   std::vector<CopyEntry> e(ntensors);
   size_t off = 0;
   for (int i = 0; i < ntensors; ++i) {
+    if (numels[i] && (!tensors[i] || !bucket)) return CC_ERR_INVALID_ARG;
     e[i] = CopyEntry{static_cast<const char*>(bucket) + off * es, tensors[i], numels[i], 0};
     off += numels[i];
   }
@@ -268,9 +274,11 @@ cc_status cc_bucket_allreduce(const void* const* grads, void* const* out, int nr
   if (!valid_ranks(nranks) || ntensors < 0 || cap_bytes == 0 || !(scale == scale)) return CC_ERR_INVALID_ARG;
   if (algo != CC_ALGO_RING && algo != CC_ALGO_TREE) return CC_ERR_INVALID_ARG;
   if (ntensors == 0) return CC_OK;
-  if (!numels || !all_nonnull(grads, nranks * ntensors) ||
-      !all_nonnull((const void* const*)out, nranks * ntensors))
-    return CC_ERR_INVALID_ARG;
+  if (!numels || !grads || !out) return CC_ERR_INVALID_ARG;
+  for (int r = 0; r < nranks; ++r)
+    for (int i = 0; i < ntensors; ++i)
+      if (numels[i] && (!grads[(size_t)r * ntensors + i] || !out[(size_t)r * ntensors + i]))
+        return CC_ERR_INVALID_ARG;  // empty tensors may be null
   std::vector<int32_t> order(ntensors), start(ntensors + 1);
   int32_t nb = 0;
   cc_bucket_assign(numels, ntensors, 4, cap_bytes, order.data(), start.data(), &nb);
@@ -297,6 +305,33 @@ cc_status cc_bucket_allreduce(const void* const* grads, void* const* out, int nr
       if (err != cudaSuccess) return CC_ERR_CUDA;
       ids.clear();
     }
+  }
+  return CC_OK;
+}
+
+cc_status cc_bucket_allreduce_host(const void* const* host_grads, void* const* host_out, void* const* dev_grads,
+                                   void* const* dev_out, int nranks, int ntensors, const size_t* numels,
+                                   size_t cap_bytes, cc_algo algo, float scale, void* stream) {
+  if (!valid_ranks(nranks) || ntensors < 0 || cap_bytes == 0) return CC_ERR_INVALID_ARG;
+  if (ntensors == 0) return CC_OK;
+  if (!host_grads || !host_out || !dev_grads || !dev_out || !numels) return CC_ERR_INVALID_ARG;
+  const size_t total = (size_t)nranks * ntensors;
+  for (size_t j = 0; j < total; ++j)
+    if (numels[j % ntensors] && (!host_grads[j] || !host_out[j] || !dev_grads[j] || !dev_out[j]))
+      return CC_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  for (size_t j = 0; j < total; ++j) {
+    const size_t nb = numels[j % ntensors] * 4;
+    if (nb && cudaMemcpyAsync(dev_grads[j], host_grads[j], nb, cudaMemcpyHostToDevice, s) != cudaSuccess)
+      return CC_ERR_CUDA;
+  }
+  cc_status st = cc_bucket_allreduce((const void* const*)dev_grads, dev_out, nranks, ntensors, numels, cap_bytes,
+                                     algo, scale, stream);
+  if (st != CC_OK) return st;
+  for (size_t j = 0; j < total; ++j) {
+    const size_t nb = numels[j % ntensors] * 4;
+    if (nb && cudaMemcpyAsync(host_out[j], dev_out[j], nb, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+      return CC_ERR_CUDA;
   }
   return CC_OK;
 }

@@ -216,26 +216,40 @@ static_assert(sizeof(BucketParams) <= 32000, "kernel parameter block too large")
 template <bool RING>
 __global__ void __launch_bounds__(kThreads) bucket_allreduce_kernel(const __grid_constant__ BucketParams P) {
   constexpr int IN = CC_F32, OP = CC_SUM;
+  // the tile's per-rank pointers, staged once per tile: the fold reads them for every
+  // 16-byte unit, and the parameter table is too large to stay in the constant cache
+  __shared__ const float* s_in[kMaxRanks];
+  __shared__ float* s_out[kMaxRanks];
+  __shared__ int s_tensor;
   const int n = P.nranks, nt = P.ntensors;
   const uint32_t ntiles = P.tile_prefix[nt];
   for (uint32_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    int lo = 0, hi = nt - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (P.tile_prefix[mid] <= tile) lo = mid; else hi = mid - 1;
+    if (threadIdx.x == 0) {
+      int lo = 0, hi = nt - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (P.tile_prefix[mid] <= tile) lo = mid; else hi = mid - 1;
+      }
+      s_tensor = lo;
     }
-    const int i = lo;
+    __syncthreads();
+    const int i = s_tensor;
+    if (threadIdx.x < n) {
+      s_in[threadIdx.x] = P.in[threadIdx.x * nt + i];
+      s_out[threadIdx.x] = P.out[threadIdx.x * nt + i];
+    }
+    __syncthreads();
     const BucketTensorDesc d = P.t[i];
     const uint64_t ea = (uint64_t)(tile - P.tile_prefix[i]) * kBucketTile;
     const uint64_t eb = min(ea + kBucketTile, d.numel);
-    auto src = [&](int r) { return P.in[r * nt + i]; };
+    auto src = [&](int r) { return s_in[r]; };
     auto emit_unit = [&](uint64_t e, Unit<IN> u) {
       if (P.do_scale) scale_unit<IN>(u, P.scale);
-      for (int r = 0; r < n; ++r) store_unit<IN>(P.out[r * nt + i] + e, u);
+      for (int r = 0; r < n; ++r) store_unit<IN>(s_out[r] + e, u);
     };
     auto emit_elem = [&](uint64_t e, float v) {
       if (P.do_scale) v = __fmul_rn(v, P.scale);
-      for (int r = 0; r < n; ++r) store_elem<IN>(P.out[r * nt + i] + e, v);
+      for (int r = 0; r < n; ++r) store_elem<IN>(s_out[r] + e, v);
     };
     uint64_t s = ea;
     while (s < eb) {
@@ -254,6 +268,7 @@ __global__ void __launch_bounds__(kThreads) bucket_allreduce_kernel(const __grid
                                  P.vec != 0, src, emit_unit, emit_elem);
       s = se;
     }
+    __syncthreads();  // every thread is done with s_in / s_out before the next tile restages them
   }
 }
 

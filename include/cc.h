@@ -181,6 +181,16 @@ CC_API cc_status cc_bucket_allreduce(const void* const* grads, void* const* out,
                               const size_t* numels, size_t cap_bytes, cc_algo algo, float scale,
                               void* stream);
 
+/* The same fused DDP step for gradients that live in host memory: every host_grads[j] is
+ * copied to dev_grads[j] (host -> device), cc_bucket_allreduce runs on the device copies,
+ * and every dev_out[j] is copied back to host_out[j] (device -> host), all stream-ordered
+ * on `stream`. The caller owns the device staging buffers (dev_grads may equal dev_out);
+ * pinned host memory makes the copies asynchronous. Layouts as cc_bucket_allreduce. */
+CC_API cc_status cc_bucket_allreduce_host(const void* const* host_grads, void* const* host_out,
+                                          void* const* dev_grads, void* const* dev_out, int nranks,
+                                          int ntensors, const size_t* numels, size_t cap_bytes,
+                                          cc_algo algo, float scale, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

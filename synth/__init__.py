@@ -102,16 +102,17 @@ def _fill(out: np.ndarray, fn) -> np.ndarray:
 
 
 def uniform_f32(seed: int, rank: int, count: int, lo: float = -1.0, hi: float = 1.0,
-                stream: int = 0, native: bool = True) -> np.ndarray:
-    """fp32 values lo + (hi - lo) * u, u = top-24-bit fraction; [-1, 1) is exact."""
+                stream: int = 0, native: bool = True, start: int = 0) -> np.ndarray:
+    """fp32 values lo + (hi - lo) * u, u = top-24-bit fraction; [-1, 1) is exact.
+    Values start..start+count-1 of the sequence."""
     out = np.empty(count, dtype=np.float32)
     lib = _native() if native else None
     if lib:
-        lib.synth_uniform_f32(int(stream_key(seed, rank, stream)), 0, count, lo, hi, out.ctypes.data)
+        lib.synth_uniform_f32(int(stream_key(seed, rank, stream)), start, count, lo, hi, out.ctypes.data)
         return out
 
     def fn(a, b, dst):
-        u = (raw_u64(seed, rank, np.arange(a, b, dtype=np.uint64), stream) >> np.uint64(40))
+        u = (raw_u64(seed, rank, np.arange(start + a, start + b, dtype=np.uint64), stream) >> np.uint64(40))
         f = u.astype(np.float32) * np.float32(2.0 ** -24)
         if lo == -1.0 and hi == 1.0:
             dst[:] = f * np.float32(2.0) - np.float32(1.0)
@@ -121,16 +122,17 @@ def uniform_f32(seed: int, rank: int, count: int, lo: float = -1.0, hi: float = 
 
 
 def normal_f32(seed: int, rank: int, count: int, std: float = 1.0, stream: int = 0,
-               native: bool = True) -> np.ndarray:
-    """fp32 normal(0, std): Box-Muller on the two 32-bit halves of one draw, in fp64."""
+               native: bool = True, start: int = 0) -> np.ndarray:
+    """fp32 normal(0, std): Box-Muller on the two 32-bit halves of one draw, in fp64.
+    Values start..start+count-1 of the sequence."""
     out = np.empty(count, dtype=np.float32)
     lib = _native() if native else None
     if lib:
-        lib.synth_normal_f32(int(stream_key(seed, rank, stream)), 0, count, std, out.ctypes.data)
+        lib.synth_normal_f32(int(stream_key(seed, rank, stream)), start, count, std, out.ctypes.data)
         return out
 
     def fn(a, b, dst):
-        z = raw_u64(seed, rank, np.arange(a, b, dtype=np.uint64), stream)
+        z = raw_u64(seed, rank, np.arange(start + a, start + b, dtype=np.uint64), stream)
         u1 = ((z >> np.uint64(32)).astype(np.float64) + 1.0) * (2.0 ** -32)
         u2 = (z & np.uint64(0xFFFFFFFF)).astype(np.float64) * (2.0 ** -32)
         g = np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * np.pi * u2)
@@ -139,17 +141,18 @@ def normal_f32(seed: int, rank: int, count: int, std: float = 1.0, stream: int =
 
 
 def int32_uniform(seed: int, rank: int, count: int, lo: int, hi: int, stream: int = 0,
-                  native: bool = True) -> np.ndarray:
-    """int32 values uniform on [lo, hi] (modulo reduction of a 64-bit draw)."""
+                  native: bool = True, start: int = 0) -> np.ndarray:
+    """int32 values uniform on [lo, hi] (modulo reduction of a 64-bit draw).
+    Values start..start+count-1 of the sequence."""
     span = np.uint64(hi - lo + 1)
     out = np.empty(count, dtype=np.int32)
     lib = _native() if native else None
     if lib:
-        lib.synth_int32(int(stream_key(seed, rank, stream)), 0, count, lo, hi, out.ctypes.data)
+        lib.synth_int32(int(stream_key(seed, rank, stream)), start, count, lo, hi, out.ctypes.data)
         return out
 
     def fn(a, b, dst):
-        z = raw_u64(seed, rank, np.arange(a, b, dtype=np.uint64), stream)
+        z = raw_u64(seed, rank, np.arange(start + a, start + b, dtype=np.uint64), stream)
         dst[:] = ((z % span).astype(np.int64) + lo).astype(np.int32)
     return _fill(out, fn)
 

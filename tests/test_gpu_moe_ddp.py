@@ -25,7 +25,7 @@ def test_route_topk_matches_oracle(n, tokens, experts, topk):
     lg = _logits(1, n, tokens, experts)
     lg[0][0, :4] = np.float32(1.5)     # ties: lower id first
     lg[0][1, :] = np.float32(0.0)
-    lg[0][1, 3] = np.float32(-0.0)
+    lg[0][1, experts - 1] = np.float32(-0.0)
     ids = [torch.full((tokens, topk), -7, dtype=torch.int32, device="cuda") for _ in range(n)]
     cc.cc_route_topk([to_dev(x) for x in lg], ids)
     torch.cuda.synchronize()

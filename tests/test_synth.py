@@ -21,6 +21,17 @@ def test_counter_based_prefix_property_and_rank_independence():
     assert not np.array_equal(a[:1000], synth.uniform_f32(9, 4, 1000))
 
 
+def test_start_offset_selects_the_same_values():
+    for native in (True, False):
+        full = synth.normal_f32(3, 2, 5000, 1e-3, native=native)
+        part = synth.normal_f32(3, 2, 1000, 1e-3, native=native, start=3000)
+        assert np.array_equal(full[3000:4000], part)
+        assert np.array_equal(synth.uniform_f32(1, 1, 900, native=native)[100:],
+                              synth.uniform_f32(1, 1, 800, native=native, start=100))
+        assert np.array_equal(synth.int32_uniform(1, 1, 900, -5, 5, native=native)[7:],
+                              synth.int32_uniform(1, 1, 893, -5, 5, native=native, start=7))
+
+
 def test_distributions():
     u = synth.uniform_f32(0, 0, 1_000_000)
     assert u.min() >= -1 and u.max() < 1 and abs(u.mean()) < 5e-3
