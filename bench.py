@@ -222,8 +222,11 @@ def main():
     bytes_step = 2 * N_SIM * w["total"] * 4
     stream = torch.cuda.current_stream()
 
+    plan = cc.BucketAllreducePlan(w["dev_in"], w["dev_out"], cap_bytes=CAP, scale=1.0 / N_SIM)
+    cuda_stream = stream.cuda_stream
+
     def step():
-        cc.cc_bucket_allreduce(w["dev_in"], w["dev_out"], cap_bytes=CAP, scale=1.0 / N_SIM)
+        plan.run(cuda_stream)
 
     launches_per_step = -(-len(w["numels"]) // 192)
 

@@ -327,6 +327,36 @@ def cc_bucket_allreduce(grads, out, *, cap_bytes: int = 25 * 1024 * 1024, algo="
                                    cap_bytes, _ALGOS[algo], float(scale), _stream(stream)), "cc_bucket_allreduce")
 
 
+class BucketAllreducePlan:
+    """cc_bucket_allreduce with the marshalling done once: the tensor tables are checked
+    and turned into pointer arrays at construction, and run() is a bare C call. The
+    tensors must stay alive (and keep their storage) while the plan is used."""
+
+    def __init__(self, grads, out, *, cap_bytes: int = 25 * 1024 * 1024, algo="ring", scale=None):
+        torch = _torch()
+        n, nt = _ranks(grads, "BucketAllreducePlan"), len(grads[0])
+        if len(out) != n or any(len(row) != nt for row in list(grads) + list(out)):
+            raise ValueError("BucketAllreducePlan: grads and out must both be [nranks][ntensors]")
+        for i in range(nt):
+            _same([grads[r][i] for r in range(n)] + [out[r][i] for r in range(n)], grads[0][i].numel(),
+                  torch.float32, f"BucketAllreducePlan tensor {i}")
+        self._keep = (grads, out)
+        self.n, self.nt = n, nt
+        self._in = _ptrs([t for row in grads for t in row])
+        self._out = _ptrs([t for row in out for t in row])
+        self._numels = _sizes([t.numel() for t in grads[0]])
+        self.cap_bytes = int(cap_bytes)
+        self.algo = _ALGOS[algo]
+        self.scale = float(1.0 / n if scale is None else scale)
+        self._fn = get_lib().cc_bucket_allreduce
+
+    def run(self, stream=None) -> None:
+        st = self._fn(self._in, self._out, self.n, self.nt, self._numels, self.cap_bytes, self.algo, self.scale,
+                      _stream(stream))
+        if st != CC_OK:
+            raise CCError(st, "cc_bucket_allreduce")
+
+
 def cc_bucket_allreduce_host(host_grads, host_out, dev_grads, dev_out, *, cap_bytes: int = 25 * 1024 * 1024,
                              algo="ring", scale=None, stream=None) -> None:
     """The fused DDP step on host-resident gradients: host -> device copies, the fused

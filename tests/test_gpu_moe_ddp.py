@@ -111,6 +111,21 @@ def test_fused_bucket_allreduce_matches_oracle(algo, n, cap):
             out[r][i].check()
 
 
+def test_bucket_plan_matches_direct_call():
+    n, cap = 8, 30_000
+    shapes, grads = _small_model(n, seed=6)
+    want, _ = ddp.ddp_allreduce(grads, cap_bytes=cap)
+    d_in = [[to_dev(g) for g in row] for row in grads]
+    out = [[torch.empty_like(t) for t in row] for row in d_in]
+    plan = cc.BucketAllreducePlan(d_in, out, cap_bytes=cap)
+    for _ in range(2):
+        plan.run()
+    torch.cuda.synchronize()
+    for r in range(n):
+        for i in range(len(shapes)):
+            assert np.array_equal(bits(to_host(out[r][i])), bits(want[r][i]))
+
+
 def test_flatten_allreduce_unflatten_equals_fused():
     n, cap = 8, 60_000
     shapes, grads = _small_model(n, seed=4)
