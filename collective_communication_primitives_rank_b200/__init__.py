@@ -46,6 +46,7 @@ _SIGS = {
     "cc_alltoallv_workspace_size": (_sz, [_i, _i, _i, _i]),
     "cc_alltoallv": (_i, [_PP, _PP, _i, _sz, _PP, _i, _i, _i, _sz, _i, _vp, _sz, _vp]),
     "cc_alltoallv_recv_counts": (_i, [_vp, _i, _vp, _vp]),
+    "cc_alltoallv_noalloc": (_i, [_PP, _PP, _i, _sz, _PP, _i, _i, _i, _sz, _i, _vp, _vp]),
     "cc_bucket_assign": (_i, [_SZP, _i, _sz, _sz, _I32P, _I32P, _I32P]),
     "cc_bucket_flatten": (_i, [_PP, _SZP, _i, _vp, _i, _vp]),
     "cc_bucket_unflatten": (_i, [_vp, _PP, _SZP, _i, _i, _vp]),

@@ -154,6 +154,27 @@ CC_API cc_status cc_alltoallv(const void* const* send, void* const* recv, int nr
 CC_API cc_status cc_alltoallv_recv_counts(const void* workspace, int nranks, int32_t* recv_rows,
                                    void* stream);
 
+/* cc_alltoallv without a workspace, for callers that cannot allocate device memory
+ * (a plugin or custom-operator host that hands over only inputs and outputs, or a runtime
+ * that keeps all device memory in its own pool). The collective pages have no counterpart;
+ * this is a deployment variant of cc_alltoallv with the same arguments and results.
+ *   Scratch: a fixed 1 MiB array inside the library's device memory, one per GPU, held by
+ *   every GPU that loads the library until the process exits. Shapes whose routing scratch
+ *   (cc_alltoallv_workspace_size) exceeds 1 MiB are rejected with CC_ERR_INVALID_ARG
+ *   (N = 8, 8192 tokens, top-2, 8 experts per rank needs 644 KiB).
+ *   Set-up: the first call on a device looks up the array's device address with that
+ *   device current; make that first call before any stream capture.
+ *   Sharing: every call on a device uses the same array and leaves its tables there; each
+ *   call rewrites every entry it reads, so nothing needs clearing, but calls that overlap
+ *   on the GPU (other streams, other threads) race: serialize them.
+ *   recv_rows: NULL, or nranks int32 (device or pinned host memory) that receive the
+ *   per-destination row counts, stream-ordered.
+ *   Allocates nothing: no cudaMalloc, no cudaFree. */
+CC_API cc_status cc_alltoallv_noalloc(const void* const* send, void* const* recv, int nranks,
+                                      size_t row_bytes, const int32_t* const* expert_ids, int tokens,
+                                      int topk, int experts_per_rank, size_t recv_capacity_rows,
+                                      int direction, int32_t* recv_rows, void* stream);
+
 /* ---- DDP gradient buckets (lecture 09 §6.1; the from-scratch page's bucketing) --------
  * Bucket assignment (host only): tensors are taken in reverse order of their index
  * (the order backward produces them), never split; a new bucket starts when the next
