@@ -192,6 +192,179 @@ def run_reference(args):
     return 0
 
 
+# ---- the other hot-path rows (one JSON line each; not the headline) --------------------------------
+
+def _event_time_ms(torch, fn, iters, flush=None):
+    """Sum of per-iteration CUDA-event times of fn(); `flush` (outside the timed spans)
+    evicts L2 between iterations when the working set would fit in it."""
+    total = 0.0
+    stream = torch.cuda.current_stream()
+    for _ in range(iters):
+        if flush is not None:
+            flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        total += a.elapsed_time(b)
+    return total
+
+
+def _prepared_allreduce(cc, x, y, algo, stream):
+    """cc_allreduce with its arguments marshalled once, so that a timed span holds only the
+    C call (the binding's per-call checks would otherwise sit between the events)."""
+    fn = cc.get_lib().cc_allreduce
+    a = (cc._ptrs(x), cc._ptrs(y), len(x), x[0].numel(), cc.CC_F32, cc.CC_F32, cc.CC_SUM,
+         cc.CC_ALGO_RING if algo == "ring" else cc.CC_ALGO_TREE, 1.0, stream)
+
+    def call():
+        if fn(*a) != cc.CC_OK:
+            raise RuntimeError("cc_allreduce failed")
+    return call
+
+
+def _row_line(args, metric, value, unit, ms, config, roofline, launches, extra=None):
+    peak, kind = measured_peak()
+    line = {"metric": metric, "value": value, "unit": unit, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": config.pop("dtype", "f32"), "data": "synthetic", "config": config,
+            "roofline": dict(roofline, peak=peak, peak_kind=kind, unit="GB/s",
+                             frac=roofline["achieved"] / peak, bound="hbm", traffic=None),
+            "gpu_launches": launches}
+    if extra:
+        line.update(extra)
+    print(json.dumps(line))
+
+
+def run_rows(args):
+    import torch
+    import collective_communication_primitives_rank_b200 as cc
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(SEED)
+    iters = max(1, args.steps)
+    if args.workload == "zero":
+        # config 3: N = 8, 300M fp32 per rank normal(0, 1e-2): reduce-scatter to 1/8 shards, then
+        # allgather of the shards; plus the bf16-input reduce-scatter with fp32 accumulation
+        n, count = N_SIM, 300_000_000
+        x = [torch.randn(count, device="cuda", generator=gen) * 1e-2 for _ in range(n)]
+        shard = count // n
+        rs = [torch.empty(shard, device="cuda") for _ in range(n)]
+        ag = [torch.empty(count, device="cuda") for _ in range(n)]
+        for _ in range(args.warmup):
+            cc.cc_reduce_scatter(x, rs)
+            cc.cc_allgather(rs, ag)
+        t_rs = _event_time_ms(torch, lambda: cc.cc_reduce_scatter(x, rs), iters) / iters
+        t_ag = _event_time_ms(torch, lambda: cc.cc_allgather(rs, ag), iters) / iters
+        del ag
+        xb = [t.to(torch.bfloat16) for t in x]
+        del x
+        for _ in range(args.warmup):
+            cc.cc_reduce_scatter(xb, rs)
+        t_bf = _event_time_ms(torch, lambda: cc.cc_reduce_scatter(xb, rs), iters) / iters
+        T = count * 4
+        ms = t_rs + t_ag
+        value = 2 * n * T / (ms * 1e-3) / 1e9
+        _row_line(args, METRIC, value, "GB/s", ms,
+                  {"workload": "zero: N=8 simulated ranks, 300M fp32 per rank normal(0,1e-2), ring reduce-scatter "
+                               "to 37.5M-element shards, then allgather of the shards (device-seeded inputs)",
+                   "l2": "inputs larger than L2; no flush"},
+                  {"achieved": (n + 1) * T / (t_rs * 1e-3) / 1e9, "kernel": "reduce_kernel<f32,sum,ring> (RS)"},
+                  2 * iters,
+                  {"rows": {"reduce_scatter_f32": {"ms": t_rs, "bytes": (n + 1) * T, "GBps": (n + 1) * T / t_rs / 1e6},
+                            "allgather_f32": {"ms": t_ag, "bytes": (n + 1) * T, "GBps": (n + 1) * T / t_ag / 1e6},
+                            "reduce_scatter_bf16_in_f32_out": {"ms": t_bf, "bytes": n * T // 2 + T,
+                                                               "GBps": (n * T // 2 + T) / t_bf / 1e6}}})
+        return 0
+    if args.workload == "moe":
+        # config 4: N = 8, 8192 tokens x 4096 bf16 per rank, 64 experts (8 per rank), top-2
+        n, tokens, hidden, epr, topk = N_SIM, 8192, 4096, 8, 2
+        E = n * epr
+        logits = [torch.randn(tokens, E, device="cuda", generator=gen) for _ in range(n)]
+        toks = [torch.randn(tokens, hidden, device="cuda", generator=gen).to(torch.bfloat16) for _ in range(n)]
+        ids = [torch.empty(tokens, topk, dtype=torch.int32, device="cuda") for _ in range(n)]
+        cc.cc_route_topk(logits, ids)
+        ws = torch.empty(cc.cc_alltoallv_workspace_size(n, tokens, topk, epr) // 4 + 64, dtype=torch.int32,
+                         device="cuda")
+        cap = tokens * topk * 2
+        recv = [torch.empty(cap, hidden, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+        back = [torch.empty(tokens, topk, hidden, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+        counts = torch.zeros(n, dtype=torch.int32, device="cuda")
+        cc.cc_alltoallv(toks, recv, ids, epr, ws, direction=0)
+        cc.cc_alltoallv_recv_counts(ws, n, counts)
+        torch.cuda.synchronize()
+        rows_recv = int(counts.sum().item())
+        row = hidden * 2
+        for _ in range(args.warmup):
+            cc.cc_route_topk(logits, ids)
+            cc.cc_alltoallv(toks, recv, ids, epr, ws, direction=0)
+            cc.cc_alltoallv(recv, back, ids, epr, ws, direction=1)
+        t_route = _event_time_ms(torch, lambda: cc.cc_route_topk(logits, ids), iters) / iters
+        t_d = _event_time_ms(torch, lambda: cc.cc_alltoallv(toks, recv, ids, epr, ws, direction=0), iters) / iters
+        t_c = _event_time_ms(torch, lambda: cc.cc_alltoallv(recv, back, ids, epr, ws, direction=1), iters) / iters
+        b_d = n * tokens * row + rows_recv * row
+        b_c = 2 * rows_recv * row
+        ms = t_route + t_d + t_c
+        _row_line(args, "alltoallv effective HBM GB/s (dispatch: tokens read once + routed rows written; "
+                        "combine: routed rows read + written)", (b_d + b_c) / (ms * 1e-3) / 1e9, "GB/s", ms,
+                  {"workload": "moe: N=8 simulated ranks, 8192 tokens x 4096 bf16 per rank, 64 experts (8 per rank), "
+                               "top-2 routing from normal logits, dispatch then combine (device-seeded inputs)",
+                   "dtype": "bf16 (bit copy)", "l2": "inputs larger than L2; no flush"},
+                  {"achieved": b_d / (t_d * 1e-3) / 1e9, "kernel": "a2a dispatch (count + scan + base + copy)"},
+                  iters * (1 + 4 + 4),
+                  {"rows": {"route_topk": {"ms": t_route},
+                            "dispatch": {"ms": t_d, "bytes": b_d, "GBps": b_d / t_d / 1e6},
+                            "combine": {"ms": t_c, "bytes": b_c, "GBps": b_c / t_c / 1e6}}})
+        return 0
+    # config 5: ring vs double-binary-tree allreduce, N in {2..64}, 1 KiB .. 256 MiB per rank
+    flush_buf = torch.empty(256 * 1024 * 1024 // 4, device="cuda")
+    table = []
+    best = None
+    for n in (2, 4, 8, 16, 32, 64):
+        for i in range(10):
+            size = 1024 * 4 ** i
+            count = size // 4
+            if n * size > 16 * 1024 ** 3:
+                continue
+            x = [torch.rand(count, device="cuda", generator=gen) * 2 - 1 for _ in range(n)]
+            y = [torch.empty_like(t) for t in x]
+            small = 2 * n * size < 2 * 126 * 1024 * 1024
+            flush = (lambda: flush_buf.fill_(1.0)) if small else None
+            reps = max(3, min(50, int(2e9 // (2 * n * size + 1))))
+            row = {"n": n, "bytes_per_rank": size}
+            for algo in ("ring", "tree"):
+                call = _prepared_allreduce(cc, x, y, algo, torch.cuda.current_stream().cuda_stream)
+                for _ in range(3):
+                    call()
+                ms = _event_time_ms(torch, call, reps, flush) / reps
+                row[algo + "_us"] = ms * 1e3
+                row[algo + "_GBps"] = 2 * n * size / (ms * 1e-3) / 1e9
+            if n == 8:
+                src = x[0]
+                ms = _event_time_ms(torch, lambda: cc.cc_broadcast(src, y, 0), reps, flush) / reps
+                row["broadcast_GBps"] = (n + 1) * size / (ms * 1e-3) / 1e9
+            table.append(row)
+            if n == 8 and size == 256 * 1024 * 1024:
+                best = row
+            del x, y
+    cross = {}
+    for n in (2, 4, 8, 16, 32, 64):
+        pts = [r for r in table if r["n"] == n]
+        over = [r["bytes_per_rank"] for r in pts if r["ring_GBps"] > 1.03 * r["tree_GBps"]]
+        under = [r["bytes_per_rank"] for r in pts if r["tree_GBps"] > 1.03 * r["ring_GBps"]]
+        cross[str(n)] = {"ring_faster_by_3pct_at": over, "tree_faster_by_3pct_at": under}
+    lat = min(r["ring_us"] for r in table)
+    _row_line(args, METRIC, best["ring_GBps"], "GB/s", best["ring_us"] / 1e3,
+              {"workload": "sweep: ring vs double-binary-tree allreduce, N in {2,4,8,16,32,64}, fp32 U[-1,1] "
+                           "1 KiB..256 MiB per rank (powers of 4); headline value = N=8, 256 MiB, ring",
+               "l2": "L2 flushed (256 MiB write) before every timed call whose working set fits in L2"},
+              {"achieved": best["ring_GBps"], "kernel": "reduce_kernel<f32,sum,ring>"},
+              len(table) * 2,
+              {"sweep": table, "crossover": cross, "min_launch_latency_us": lat})
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -202,9 +375,13 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--oracle-buckets", type=int, default=8)
+    ap.add_argument("--workload", default="ddp", choices=["ddp", "zero", "moe", "sweep"],
+                    help="ddp = the headline step; the others measure the remaining hot-path rows")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload != "ddp":
+        return run_rows(args)
 
     import torch
     import torch.distributed as dist
