@@ -49,17 +49,20 @@ template <int IN, int OP, typename A> __device__ __forceinline__ A op(A a, A b) 
 
 template <int IN> struct Unit { typename Tr<IN>::Acc v[Tr<IN>::UE]; };
 
-// 16-byte streaming load of one unit (evict-first: every input byte is read once).
-template <int IN> __device__ __forceinline__ Unit<IN> load_unit(const typename Tr<IN>::In* p) {
+// 16-byte streaming load (evict-first: every input byte is read once), kept as raw bits
+// until it is folded, so that a window of loads in flight costs 4 registers per load for
+// every dtype.
+__device__ __forceinline__ uint4 load_raw(const void* p) { return __ldcs(reinterpret_cast<const uint4*>(p)); }
+
+// The raw 16 bytes as one unit of accumulator values (bf16 widens exactly: bits << 16).
+template <int IN> __device__ __forceinline__ Unit<IN> to_unit(const uint4& w) {
   Unit<IN> u;
   if constexpr (IN == CC_F32) {
-    float4 f = __ldcs(reinterpret_cast<const float4*>(p));
-    u.v[0] = f.x; u.v[1] = f.y; u.v[2] = f.z; u.v[3] = f.w;
+    u.v[0] = __uint_as_float(w.x); u.v[1] = __uint_as_float(w.y);
+    u.v[2] = __uint_as_float(w.z); u.v[3] = __uint_as_float(w.w);
   } else if constexpr (IN == CC_I32) {
-    int4 f = __ldcs(reinterpret_cast<const int4*>(p));
-    u.v[0] = f.x; u.v[1] = f.y; u.v[2] = f.z; u.v[3] = f.w;
+    u.v[0] = (int)w.x; u.v[1] = (int)w.y; u.v[2] = (int)w.z; u.v[3] = (int)w.w;
   } else {
-    uint4 w = __ldcs(reinterpret_cast<const uint4*>(p));
     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -68,6 +71,10 @@ template <int IN> __device__ __forceinline__ Unit<IN> load_unit(const typename T
     }
   }
   return u;
+}
+
+template <int IN> __device__ __forceinline__ Unit<IN> load_unit(const typename Tr<IN>::In* p) {
+  return to_unit<IN>(load_raw(p));
 }
 
 template <int IN> __device__ __forceinline__ typename Tr<IN>::Acc load_elem(const typename Tr<IN>::In* p) {
@@ -127,8 +134,11 @@ struct FoldProgram {
   uint8_t rmap[kMaxRanks];
 };
 
-// Combine for a unit (UE lanes) or for one element.
+// Combine for a unit (UE lanes), a raw 16-byte load, or one element.
 template <int IN, int OP> __device__ __forceinline__ void comb(Unit<IN>& a, const Unit<IN>& b) { op_unit<IN, OP>(a, b); }
+template <int IN, int OP> __device__ __forceinline__ void comb(Unit<IN>& a, const uint4& b) {
+  op_unit<IN, OP>(a, to_unit<IN>(b));
+}
 template <int IN, int OP> __device__ __forceinline__ void comb(typename Tr<IN>::Acc& a, const typename Tr<IN>::Acc& b) {
   a = op<IN, OP>(a, b);
 }

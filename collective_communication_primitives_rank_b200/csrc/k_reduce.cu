@@ -28,12 +28,14 @@ constexpr int kThreads = 256;
 
 // Left fold starting at rank c: loads go out in windows of 8 so that 8 independent
 // 128-bit loads per thread are in flight before the in-order folds consume them.
-template <int IN, int OP, typename V, typename Load>
-__device__ __forceinline__ V ring_fold(int n, int c, Load ld) {
-  V acc = ld(c);
+// V is the accumulator (a unit or an element), X what one load returns (raw 16 bytes for a
+// unit, the element itself otherwise).
+template <int IN, int OP, typename V, typename X, typename Load, typename Widen>
+__device__ __forceinline__ V ring_fold(int n, int c, Load ld, Widen widen) {
+  V acc = widen(ld(c));
   int r = c;
   for (int j0 = 1; j0 < n; j0 += 8) {
-    V x[8];
+    X x[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k)
       if (j0 + k < n) { r = (r + 1 == n) ? 0 : r + 1; x[k] = ld(r); }
@@ -45,12 +47,12 @@ __device__ __forceinline__ V ring_fold(int n, int c, Load ld) {
 }
 
 // Fold machine (tree / binomial): the position's rank is rmap[p], mirrored for tree B.
-template <int IN, int OP, typename V, int W, typename Load>
-__device__ __forceinline__ V machine_fold(int n, const FoldProgram& prog, bool mirror, Load ld) {
+template <int IN, int OP, typename V, typename X, int W, typename Load, typename Widen>
+__device__ __forceinline__ V machine_fold(int n, const FoldProgram& prog, bool mirror, Load ld, Widen widen) {
   V cur;
   FoldStack<V> st;
   for (int p0 = 0; p0 < n; p0 += W) {
-    V x[W];
+    X x[W];
 #pragma unroll
     for (int k = 0; k < W; ++k)
       if (p0 + k < n) {
@@ -59,7 +61,7 @@ __device__ __forceinline__ V machine_fold(int n, const FoldProgram& prog, bool m
       }
 #pragma unroll
     for (int k = 0; k < W; ++k)
-      if (p0 + k < n) fold_step<IN, OP>(prog.code[p0 + k], x[k], cur, st);
+      if (p0 + k < n) fold_step<IN, OP>(prog.code[p0 + k], widen(x[k]), cur, st);
   }
   return cur;
 }
@@ -73,11 +75,13 @@ __device__ __forceinline__ void reduce_range(int n, int g, bool mirror, const Fo
   using In = typename Tr<IN>::In;
   using A = typename Tr<IN>::Acc;
   constexpr int UE = Tr<IN>::UE;
-  constexpr int W = UE == 8 ? 4 : 8;
+  constexpr int W = 8;
+  auto same = [](const A& a) { return a; };
+  auto widen = [](const uint4& w) { return to_unit<IN>(w); };
   auto fold_elem = [&](uint64_t e) -> A {
     auto ld = [&](int r) { return load_elem<IN>(src(r) + e); };
-    if constexpr (RING) return ring_fold<IN, OP, A>(n, g, ld);
-    else return machine_fold<IN, OP, A, W>(n, prog, mirror, ld);
+    if constexpr (RING) return ring_fold<IN, OP, A, A>(n, g, ld, same);
+    else return machine_fold<IN, OP, A, A, W>(n, prog, mirror, ld, same);
   };
   if (vec) {
     uint64_t va = (a + UE - 1) / UE * UE;
@@ -85,10 +89,10 @@ __device__ __forceinline__ void reduce_range(int n, int g, bool mirror, const Fo
     uint64_t vb = b / UE * UE;
     if (vb < va) vb = va;
     for (uint64_t e = va + t * UE; e < vb; e += T * UE) {
-      auto ld = [&](int r) { return load_unit<IN>(src(r) + e); };
+      auto ld = [&](int r) { return load_raw(src(r) + e); };
       Unit<IN> u;
-      if constexpr (RING) u = ring_fold<IN, OP, Unit<IN>>(n, g, ld);
-      else u = machine_fold<IN, OP, Unit<IN>, W>(n, prog, mirror, ld);
+      if constexpr (RING) u = ring_fold<IN, OP, Unit<IN>, uint4>(n, g, ld, widen);
+      else u = machine_fold<IN, OP, Unit<IN>, uint4, W>(n, prog, mirror, ld, widen);
       emit_unit(e, u);
     }
     const uint64_t nh = va - a, nt = b - vb;
@@ -139,7 +143,7 @@ struct ReduceParams {
 };
 
 template <int IN, int OP, bool RING>
-__global__ void __launch_bounds__(kThreads) reduce_kernel(const __grid_constant__ ReduceParams P) {
+__global__ void __launch_bounds__(kThreads, RING ? 4 : 2) reduce_kernel(const __grid_constant__ ReduceParams P) {
   using In = typename Tr<IN>::In;
   using Out = typename Tr<IN>::Out;
   using A = typename Tr<IN>::Acc;
@@ -214,7 +218,7 @@ struct BucketParams {
 static_assert(sizeof(BucketParams) <= 32000, "kernel parameter block too large");
 
 template <bool RING>
-__global__ void __launch_bounds__(kThreads) bucket_allreduce_kernel(const __grid_constant__ BucketParams P) {
+__global__ void __launch_bounds__(kThreads, RING ? 3 : 2) bucket_allreduce_kernel(const __grid_constant__ BucketParams P) {
   constexpr int IN = CC_F32, OP = CC_SUM;
   // the tile's per-rank pointers, staged once per tile: the fold reads them for every
   // 16-byte unit, and the parameter table is too large to stay in the constant cache
