@@ -35,6 +35,7 @@ _SIGS = {
     "cc_status_string": (ctypes.c_char_p, [_i]),
     "cc_version": (_i, []),
     "cc_chunk": (_i, [_sz, _i, _i, _SZP, _SZP]),
+    "cc_async_status": (_i, [_i, _vp]),
     "cc_allreduce": (_i, [_PP, _PP, _i, _sz, _i, _i, _i, _i, _f, _vp]),
     "cc_reduce_scatter": (_i, [_PP, _PP, _i, _sz, _i, _i, _i, _i, _f, _vp]),
     "cc_allgather": (_i, [_PP, _PP, _i, _sz, _i, _vp]),
@@ -131,6 +132,12 @@ def _stream(stream) -> Optional[int]:
 
 def _sizes(vals) -> ctypes.Array:
     return (ctypes.c_size_t * len(vals))(*[int(v) for v in vals])
+
+
+def cc_async_status(reset: bool = False, stream=None) -> int:
+    """Synchronizes the stream and returns CC_OK or CC_ERR_TIMEOUT (a device-side bounded
+    wait gave up since the last reset)."""
+    return int(lib.cc_async_status(1 if reset else 0, _stream(stream)))
 
 
 def cc_chunk(count: int, nranks: int, c: int) -> tuple[int, int]:

@@ -62,6 +62,12 @@ const char* cc_status_string(cc_status s) {
 
 int cc_version(void) { return 100; }
 
+cc_status cc_async_status(int reset, void* stream) {
+  int v = 0;
+  if (read_async_status(&v, reset != 0, as_stream(stream)) != cudaSuccess) return CC_ERR_CUDA;
+  return v == CC_OK ? CC_OK : CC_ERR_TIMEOUT;
+}
+
 cc_status cc_chunk(size_t count, int nranks, int c, size_t* start, size_t* len) {
   if (!valid_ranks(nranks) || c < 0 || c >= nranks || !start || !len) return CC_ERR_INVALID_ARG;
   chunk_bounds(count, nranks, c, *start, *len);

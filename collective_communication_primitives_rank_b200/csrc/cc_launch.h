@@ -41,6 +41,10 @@ struct CopyEntry {
 cudaError_t launch_copy(const CopyEntry* entries, int nentries, void* const* dst_base, int ndst,
                         bool fanout, int skip, size_t elem_bytes, cudaStream_t stream);
 
+// Device status word of the bounded waits (CC_OK or CC_ERR_TIMEOUT), read with a
+// stream synchronisation; `reset` clears it afterwards.
+cudaError_t read_async_status(int* out, bool reset, cudaStream_t stream);
+
 // MoE
 cudaError_t launch_route_topk(const float* const* logits, int32_t* const* ids, int nranks, int tokens,
                               int experts_total, int topk, cudaStream_t stream);

@@ -22,7 +22,6 @@ namespace cc {
 
 constexpr int kTileRows = 256;  // rows per K1 tile: 8 warps
 constexpr int kMaxTopk = 8;
-constexpr int kMaxExperts = 1024;
 
 struct A2AWorkspace {
   // byte offsets inside the caller's workspace; the receive counts sit first, at a

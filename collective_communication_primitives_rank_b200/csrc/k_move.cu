@@ -1,11 +1,19 @@
-// Data-movement kernel: allgather, broadcast, scatter, gather, bucket flatten/unflatten.
+// Data-movement kernels: allgather, broadcast, scatter, gather, bucket flatten/unflatten.
 //
 // All of them are "copy entry k (src, bytes) to one destination, or to the same offset
-// of every rank's buffer" (fan-out). The kernel reads each source byte once and writes it
-// to each destination: allgather reads T and writes N·T, the minimum. Entries are cut
-// into 64 KiB tiles; a CTA takes tiles round-robin (binary search in the tile prefix
-// table) and moves them with 128-bit streaming loads/stores when every address of the
-// entry is 16-byte aligned, element by element otherwise.
+// of every rank's buffer" (fan-out). Each source byte is read once and written to each
+// destination: allgather reads T and writes N·T, the minimum. Entries are cut into tiles;
+// a CTA takes tiles round-robin (binary search in the tile prefix table).
+//
+// copy_bulk_kernel (every entry 16-byte aligned): the tensor memory accelerator moves the
+// data. One thread per CTA runs a STAGES-deep pipeline: cp.async.bulk loads a 32 KiB tile
+// into shared memory (completion on an mbarrier), then cp.async.bulk stores the same
+// shared-memory tile to every destination, so a tile costs the SM a handful of
+// instructions however many replicas it has. Waits are bounded: a wait that gives up
+// records CC_ERR_TIMEOUT in the device status word and the CTA drains its copies and exits.
+//
+// copy_kernel (any alignment): 128-bit streaming loads/stores per thread where an entry is
+// 16-byte aligned, element by element otherwise.
 #include <algorithm>
 
 #include "cc_device.cuh"
@@ -71,13 +79,141 @@ __global__ void __launch_bounds__(kCopyThreads) copy_kernel(const __grid_constan
   }
 }
 
+// ---- bulk (TMA) path ----------------------------------------------------------------------------
+
+__device__ int g_async_status;  // CC_OK, or CC_ERR_TIMEOUT after a bounded wait gave up
+
+constexpr int kBulkStages = 4;
+constexpr uint32_t kBulkTile = 32 * 1024;  // bytes; a multiple of 16
+constexpr long kWaitLimit = 1l << 26;      // try_wait polls before a wait gives up (seconds)
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* m) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(m)));
+}
+__device__ __forceinline__ void mbar_arrive_tx(uint64_t* m, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(m)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint64_t* m, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok) : "r"(smem_addr(m)), "r"(parity) : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* m, uint32_t parity) {
+  for (long i = 0; i < kWaitLimit; ++i)
+    if (mbar_test(m, parity)) return true;
+  atomicExch(&g_async_status, (int)CC_ERR_TIMEOUT);
+  return false;
+}
+__device__ __forceinline__ void bulk_load(void* smem, const void* gmem, uint32_t bytes, uint64_t* m) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(smem_addr(smem)), "l"(gmem), "r"(bytes), "r"(smem_addr(m)) : "memory");
+}
+__device__ __forceinline__ void bulk_store(void* gmem, const void* smem, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+               ::"l"(gmem), "r"(smem_addr(smem)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_reads_but_one() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+__global__ void __launch_bounds__(32) copy_bulk_kernel(const __grid_constant__ CopyParams P) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + (size_t)kBulkStages * kBulkTile);
+  if (threadIdx.x != 0) return;
+  const uint32_t ntiles = P.tile_prefix[P.nentries];
+  for (int s = 0; s < kBulkStages; ++s) mbar_init(&bar[s]);
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  struct TileRef { int k; uint64_t a; uint32_t bytes; };
+  auto locate = [&](uint32_t tile) {
+    int lo = 0, hi = P.nentries - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (P.tile_prefix[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    TileRef t;
+    t.k = lo;
+    t.a = (uint64_t)(tile - P.tile_prefix[lo]) * kBulkTile;
+    t.bytes = (uint32_t)min((uint64_t)kBulkTile, P.nbytes[lo] - t.a);
+    return t;
+  };
+  // the bulk part of a tile is its bytes rounded down to 16; the rest is copied by hand
+  auto issue = [&](uint32_t i, int s) {
+    const uint32_t tile = blockIdx.x + i * gridDim.x;
+    if (tile >= ntiles) return;
+    const TileRef t = locate(tile);
+    const uint32_t bulk = t.bytes & ~15u;
+    if (bulk) {
+      mbar_arrive_tx(&bar[s], bulk);
+      bulk_load(smem + (size_t)s * kBulkTile, P.src[t.k] + t.a, bulk, &bar[s]);
+    } else {
+      asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(&bar[s])) : "memory");
+    }
+  };
+  uint32_t parity = 0;  // bit s: the phase to wait for on stage s
+  for (int i = 0; i < kBulkStages - 1; ++i) issue(i, i);
+  for (uint32_t i = 0;; ++i) {
+    const uint32_t tile = blockIdx.x + i * gridDim.x;
+    if (tile >= ntiles) break;
+    const int s = i % kBulkStages;
+    if (!mbar_wait(&bar[s], (parity >> s) & 1)) {
+      // give the loads still in flight (tiles i+1 .. i+STAGES-2) a bounded chance to land
+      // before the CTA's shared memory goes away
+      for (uint32_t j = 1; j + 1 < (uint32_t)kBulkStages; ++j) {
+        if (blockIdx.x + (i + j) * gridDim.x >= ntiles) break;
+        const int sj = (i + j) % kBulkStages;
+        mbar_wait(&bar[sj], (parity >> sj) & 1);
+      }
+      break;
+    }
+    parity ^= 1u << s;
+    const TileRef t = locate(tile);
+    const uint32_t bulk = t.bytes & ~15u;
+    const unsigned char* st = smem + (size_t)s * kBulkTile;
+    if (P.fanout) {
+      for (int r = 0; r < P.ndst; ++r) {
+        if (r == P.skip) continue;
+        char* d = P.dst_base[r] + P.dst_off[t.k] + t.a;
+        if (bulk) bulk_store(d, st, bulk);
+        for (uint32_t o = bulk; o < t.bytes; o += P.esize) copy_elem(d + o, P.src[t.k] + t.a + o, P.esize);
+      }
+    } else {
+      char* d = P.dst[t.k] + t.a;
+      if (bulk) bulk_store(d, st, bulk);
+      for (uint32_t o = bulk; o < t.bytes; o += P.esize) copy_elem(d + o, P.src[t.k] + t.a + o, P.esize);
+    }
+    bulk_commit();
+    // the stage refilled next was stored from one iteration ago: its reads must be done
+    bulk_wait_reads_but_one();
+    issue(i + kBulkStages - 1, (i + kBulkStages - 1) % kBulkStages);
+  }
+  bulk_wait_all();  // no copy may outlive the CTA's shared memory
+}
+
 static bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+cudaError_t read_async_status(int* out, bool reset, cudaStream_t stream) {
+  cudaError_t e = cudaMemcpyFromSymbolAsync(out, g_async_status, sizeof(int), 0, cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e == cudaSuccess && reset) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbolAsync(g_async_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  }
+  return e;
+}
 
 cudaError_t launch_copy(const CopyEntry* entries, int nentries, void* const* dst_base, int ndst, bool fanout,
                         int skip, size_t elem_bytes, cudaStream_t stream) {
   static int bps = 0;
   if (!bps && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, copy_kernel, kCopyThreads, 0) != cudaSuccess || bps <= 0))
     bps = 4;
+  static const size_t bulk_smem = (size_t)kBulkStages * kBulkTile + kBulkStages * sizeof(uint64_t);
+  static const cudaError_t bulk_attr =
+      cudaFuncSetAttribute(copy_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bulk_smem);
   bool bases_aligned = true;
   for (int r = 0; r < ndst && fanout; ++r)
     if (r != skip) bases_aligned = bases_aligned && al16(dst_base[r]);
@@ -108,8 +244,22 @@ cudaError_t launch_copy(const CopyEntry* entries, int nentries, void* const* dst
     P.nentries = m;
     P.tile_prefix[m] = tiles;
     if (tiles == 0) continue;
-    const uint32_t grid = std::min<uint32_t>(tiles, (uint32_t)(sm_count() * bps));
-    copy_kernel<<<grid, kCopyThreads, 0, stream>>>(P);
+    bool all_vec = true;
+    for (int k = 0; k < m; ++k) all_vec = all_vec && ((P.vec_mask[k >> 6] >> (k & 63)) & 1);
+    if (all_vec && bulk_attr == cudaSuccess) {
+      // retile for the bulk kernel: kBulkTile-byte tiles
+      uint32_t bt = 0;
+      for (int k = 0; k < m; ++k) {
+        P.tile_prefix[k] = bt;
+        bt += (uint32_t)((P.nbytes[k] + kBulkTile - 1) / kBulkTile);
+      }
+      P.tile_prefix[m] = bt;
+      const uint32_t grid = std::min<uint32_t>(bt, (uint32_t)sm_count());
+      copy_bulk_kernel<<<grid, 32, bulk_smem, stream>>>(P);
+    } else {
+      const uint32_t grid = std::min<uint32_t>(tiles, (uint32_t)(sm_count() * bps));
+      copy_kernel<<<grid, kCopyThreads, 0, stream>>>(P);
+    }
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }

@@ -23,6 +23,9 @@
 namespace cc {
 
 constexpr int kThreads = 256;
+#ifndef CC_RING_MIN_BLOCKS
+#define CC_RING_MIN_BLOCKS 4  // resident 256-thread CTAs per SM the ring kernel is compiled for
+#endif
 
 // ---- folds over the N ranks ---------------------------------------------------------------------
 
@@ -112,18 +115,37 @@ __host__ __device__ __forceinline__ void chunk_range(uint64_t count, int n, int 
   b = a + q + (cc_ < r ? 1 : 0);
 }
 
-// Chunk of element o and the end of that chunk.
-__device__ __forceinline__ int chunk_of(uint64_t count, int n, uint64_t o, uint64_t& end) {
+// Chunk of element o and that chunk's [start, end).
+__device__ __forceinline__ int chunk_of(uint64_t count, int n, uint64_t o, uint64_t& start, uint64_t& end) {
   const uint64_t q = count / n, r = count % n;
   const uint64_t big = r * (q + 1);
   if (o < big) {
     const uint64_t c = o / (q + 1);
-    end = (c + 1) * (q + 1);
+    start = c * (q + 1);
+    end = start + q + 1;
     return (int)c;
   }
   const uint64_t c = r + (o - big) / q;
-  end = big + (c - r + 1) * q;
+  start = big + (c - r) * q;
+  end = start + q;
   return (int)c;
+}
+
+// The fold group of element o in a buffer of `count` elements: the ring chunk, the tree
+// half, or the single binomial group; returns the group and its [start, end).
+__device__ __forceinline__ int group_of(int fold, uint64_t count, int n, uint64_t o, uint64_t& start,
+                                        uint64_t& end) {
+  if (fold == kFoldRing) return chunk_of(count, n, o, start, end);
+  if (fold == kFoldTree) {
+    const uint64_t mid = (count + 1) / 2;
+    const int g = o >= mid;
+    start = g ? mid : 0;
+    end = g ? count : mid;
+    return g;
+  }
+  start = 0;
+  end = count;
+  return 0;
 }
 
 // ---- plain reduction kernel ------------------------------------------------------------------------
@@ -133,6 +155,7 @@ struct ReduceParams {
   void* dst[kMaxRanks];
   FoldProgram prog;
   uint64_t count;
+  uint64_t tile;         // elements per tile (a multiple of 8)
   uint64_t dst_aligned;  // bit r: dst[r] is 16-byte aligned
   int nranks;
   int mode;
@@ -142,52 +165,53 @@ struct ReduceParams {
   int do_scale;
 };
 
+// Persistent CTAs take contiguous tiles round-robin (the grid is oversubscribed twice over
+// the resident CTAs, which measured faster than one wave); a tile is split where it crosses
+// a fold group (ring chunk or tree half) and each piece is folded by the whole CTA.
 template <int IN, int OP, bool RING>
-__global__ void __launch_bounds__(kThreads, RING ? 4 : 2) reduce_kernel(const __grid_constant__ ReduceParams P) {
+__global__ void __launch_bounds__(kThreads, RING ? CC_RING_MIN_BLOCKS : 2) reduce_kernel(const __grid_constant__ ReduceParams P) {
   using In = typename Tr<IN>::In;
   using Out = typename Tr<IN>::Out;
   using A = typename Tr<IN>::Acc;
   const int n = P.nranks;
-  const int g = blockIdx.y;
-  uint64_t a, b;
-  if (P.fold == kFoldRing) {
-    chunk_range(P.count, n, g, a, b);
-  } else if (P.fold == kFoldTree) {
-    const uint64_t mid = (P.count + 1) / 2;
-    a = g ? mid : 0;
-    b = g ? P.count : mid;
-  } else {
-    a = 0;
-    b = P.count;
-  }
-  const bool mirror = (P.fold == kFoldTree && g == 1);
-  const uint64_t T = (uint64_t)gridDim.x * blockDim.x;
-  const uint64_t t = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int mode = P.mode;
-  const bool shard_vec = ((P.dst_aligned >> g) & 1) && ((a * sizeof(Out)) % 16 == 0);
+  const uint64_t ntiles = (P.count + P.tile - 1) / P.tile;
   auto src = [&](int r) { return static_cast<const In*>(P.src[r]); };
-  auto emit_unit = [&](uint64_t e, Unit<IN> u) {
-    if (P.do_scale) scale_unit<IN>(u, P.scale);
-    if (mode == kAllReduce) {
-      for (int r = 0; r < n; ++r) store_unit<IN>(static_cast<Out*>(P.dst[r]) + e, u);
-    } else if (mode == kReduceScatter) {
-      Out* d = static_cast<Out*>(P.dst[g]) + (e - a);
-      if (shard_vec) store_unit<IN>(d, u); else store_unit_scalar<IN>(d, u);
-    } else {
-      store_unit<IN>(static_cast<Out*>(P.dst[0]) + e, u);
+  for (uint64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const uint64_t ea = tile * P.tile, eb = min(ea + P.tile, P.count);
+    uint64_t s = ea;
+    while (s < eb) {
+      uint64_t ga, gb;
+      const int g = group_of(P.fold, P.count, n, s, ga, gb);
+      const uint64_t se = min(eb, gb);
+      const bool mirror = (P.fold == kFoldTree && g == 1);
+      const bool shard_vec = ((P.dst_aligned >> g) & 1) && ((ga * sizeof(Out)) % 16 == 0);
+      auto emit_unit = [&](uint64_t e, Unit<IN> u) {
+        if (P.do_scale) scale_unit<IN>(u, P.scale);
+        if (mode == kAllReduce) {
+          for (int r = 0; r < n; ++r) store_unit<IN>(static_cast<Out*>(P.dst[r]) + e, u);
+        } else if (mode == kReduceScatter) {
+          Out* d = static_cast<Out*>(P.dst[g]) + (e - ga);
+          if (shard_vec) store_unit<IN>(d, u); else store_unit_scalar<IN>(d, u);
+        } else {
+          store_unit<IN>(static_cast<Out*>(P.dst[0]) + e, u);
+        }
+      };
+      auto emit_elem = [&](uint64_t e, A v) {
+        if constexpr (IN != CC_I32) if (P.do_scale) v = __fmul_rn(v, P.scale);
+        if (mode == kAllReduce) {
+          for (int r = 0; r < n; ++r) store_elem<IN>(static_cast<Out*>(P.dst[r]) + e, v);
+        } else if (mode == kReduceScatter) {
+          store_elem<IN>(static_cast<Out*>(P.dst[g]) + (e - ga), v);
+        } else {
+          store_elem<IN>(static_cast<Out*>(P.dst[0]) + e, v);
+        }
+      };
+      reduce_range<IN, OP, RING>(n, g, mirror, P.prog, s, se, threadIdx.x, blockDim.x, P.vec != 0, src, emit_unit,
+                                 emit_elem);
+      s = se;
     }
-  };
-  auto emit_elem = [&](uint64_t e, A v) {
-    if constexpr (IN != CC_I32) if (P.do_scale) v = __fmul_rn(v, P.scale);
-    if (mode == kAllReduce) {
-      for (int r = 0; r < n; ++r) store_elem<IN>(static_cast<Out*>(P.dst[r]) + e, v);
-    } else if (mode == kReduceScatter) {
-      store_elem<IN>(static_cast<Out*>(P.dst[g]) + (e - a), v);
-    } else {
-      store_elem<IN>(static_cast<Out*>(P.dst[0]) + e, v);
-    }
-  };
-  reduce_range<IN, OP, RING>(n, g, mirror, P.prog, a, b, t, T, P.vec != 0, src, emit_unit, emit_elem);
+  }
 }
 
 // ---- fused DDP bucket allreduce --------------------------------------------------------------------
@@ -261,7 +285,8 @@ __global__ void __launch_bounds__(kThreads, RING ? 3 : 2) bucket_allreduce_kerne
       uint64_t gend;
       int g;
       if (RING) {
-        g = chunk_of(d.bucket_count, n, o, gend);
+        uint64_t gstart;
+        g = chunk_of(d.bucket_count, n, o, gstart, gend);
       } else {
         const uint64_t mid = (d.bucket_count + 1) / 2;
         g = o >= mid;
@@ -380,26 +405,30 @@ static int blocks_per_sm(K kernel) {
 }
 
 template <int IN, int OP, bool RING>
-static cudaError_t run_reduce(const ReduceParams& P, int ngroups, cudaStream_t s) {
+static cudaError_t run_reduce(ReduceParams& P, cudaStream_t s) {
   auto k = reduce_kernel<IN, OP, RING>;
   static const int bps = blocks_per_sm(k);
-  constexpr int UE = Tr<IN>::UE;
-  const uint64_t per_group = P.count / ngroups + 1;
-  const uint64_t want = (per_group + (uint64_t)kThreads * UE - 1) / ((uint64_t)kThreads * UE);
-  uint64_t bx = ((uint64_t)sm_count() * bps + ngroups - 1) / ngroups;
-  bx = std::max<uint64_t>(1, std::min(bx, want));
-  dim3 grid((unsigned)bx, (unsigned)ngroups);
-  k<<<grid, kThreads, 0, s>>>(P);
+  constexpr uint64_t UE = Tr<IN>::UE;
+  const uint64_t resident = (uint64_t)sm_count() * bps;
+  // tiles of 1..8 units per thread: large buffers get 8 (long contiguous streams per CTA),
+  // small ones shrink the tile so that every resident CTA still gets work
+  const uint64_t units = (P.count + UE - 1) / UE;
+  uint64_t upt = units / (resident * kThreads);
+  upt = std::max<uint64_t>(1, std::min<uint64_t>(8, upt));
+  P.tile = upt * kThreads * UE;
+  const uint64_t ntiles = (P.count + P.tile - 1) / P.tile;
+  const uint64_t grid = std::max<uint64_t>(1, std::min<uint64_t>(ntiles, 2 * resident));
+  k<<<(unsigned)grid, kThreads, 0, s>>>(P);
   return cudaGetLastError();
 }
 
 template <int IN>
-static cudaError_t dispatch_op(const ReduceParams& P, cc_op op, bool ring, int ngroups, cudaStream_t s) {
+static cudaError_t dispatch_op(ReduceParams& P, cc_op op, bool ring, cudaStream_t s) {
   switch (op) {
-    case CC_SUM: return ring ? run_reduce<IN, CC_SUM, true>(P, ngroups, s) : run_reduce<IN, CC_SUM, false>(P, ngroups, s);
-    case CC_MAX: return ring ? run_reduce<IN, CC_MAX, true>(P, ngroups, s) : run_reduce<IN, CC_MAX, false>(P, ngroups, s);
-    case CC_MIN: return ring ? run_reduce<IN, CC_MIN, true>(P, ngroups, s) : run_reduce<IN, CC_MIN, false>(P, ngroups, s);
-    case CC_PROD: return ring ? run_reduce<IN, CC_PROD, true>(P, ngroups, s) : run_reduce<IN, CC_PROD, false>(P, ngroups, s);
+    case CC_SUM: return ring ? run_reduce<IN, CC_SUM, true>(P, s) : run_reduce<IN, CC_SUM, false>(P, s);
+    case CC_MAX: return ring ? run_reduce<IN, CC_MAX, true>(P, s) : run_reduce<IN, CC_MAX, false>(P, s);
+    case CC_MIN: return ring ? run_reduce<IN, CC_MIN, true>(P, s) : run_reduce<IN, CC_MIN, false>(P, s);
+    case CC_PROD: return ring ? run_reduce<IN, CC_PROD, true>(P, s) : run_reduce<IN, CC_PROD, false>(P, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -427,12 +456,11 @@ cudaError_t launch_reduce(const void* const* send, void* const* dst, int ndst, i
   P.vec = vec;
   if (fold == kFoldTree) tree_program(nranks, P.prog);
   else if (fold == kFoldBinomial) binomial_program(nranks, root, P.prog);
-  const int ngroups = fold == kFoldRing ? nranks : (fold == kFoldTree ? 2 : 1);
   const bool ring = fold == kFoldRing;
   switch (in_t) {
-    case CC_F32: return dispatch_op<CC_F32>(P, op, ring, ngroups, stream);
-    case CC_BF16: return dispatch_op<CC_BF16>(P, op, ring, ngroups, stream);
-    case CC_I32: return dispatch_op<CC_I32>(P, op, ring, ngroups, stream);
+    case CC_F32: return dispatch_op<CC_F32>(P, op, ring, stream);
+    case CC_BF16: return dispatch_op<CC_BF16>(P, op, ring, stream);
+    case CC_I32: return dispatch_op<CC_I32>(P, op, ring, stream);
   }
   return cudaErrorInvalidValue;
 }
@@ -475,7 +503,7 @@ cudaError_t launch_bucket_allreduce(const void* const* grads, void* const* out, 
   auto k = ring ? bucket_allreduce_kernel<true> : bucket_allreduce_kernel<false>;
   static const int bps_ring = blocks_per_sm(bucket_allreduce_kernel<true>);
   static const int bps_tree = blocks_per_sm(bucket_allreduce_kernel<false>);
-  const uint32_t grid = std::min<uint32_t>(tiles, (uint32_t)(sm_count() * (ring ? bps_ring : bps_tree)));
+  const uint32_t grid = std::min<uint32_t>(tiles, (uint32_t)(2 * sm_count() * (ring ? bps_ring : bps_tree)));
   k<<<grid, kThreads, 0, stream>>>(P);
   return cudaGetLastError();
 }

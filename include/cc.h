@@ -73,6 +73,13 @@ CC_API const char* cc_status_string(cc_status s);
 /* Library version as major * 10000 + minor * 100 + patch. */
 CC_API int cc_version(void);
 
+/* Status of the device-side bounded waits (the bulk-copy pipeline of the data-movement
+ * calls waits on shared-memory barriers with an iteration limit). Synchronizes `stream`,
+ * then returns CC_OK, or CC_ERR_TIMEOUT if a wait gave up since the last reset (the outputs
+ * of that call are then incomplete); `reset` != 0 clears the status. CC_ERR_CUDA if the
+ * device cannot be read. */
+CC_API cc_status cc_async_status(int reset, void* stream);
+
 /* The chunk rule (host only): chunk c of a count-element buffer over nranks ranks
  * starts at *start and has *len elements (lecture 09 §7.1 splits the tensor into N equal
  * chunks; for a count N does not divide, the first count % N chunks get one more). */
