@@ -436,8 +436,10 @@ def main():
     h_in = [w["views"](h) for h in w["host"]]
     h_out = [w["views"](h) for h in host_out]
 
+    host_plan = cc.BucketAllreduceHostPlan(h_in, h_out, w["dev_in"], w["dev_out"], cap_bytes=CAP, scale=1.0 / N_SIM)
+
     def e2e_step():
-        cc.cc_bucket_allreduce_host(h_in, h_out, w["dev_in"], w["dev_out"], cap_bytes=CAP, scale=1.0 / N_SIM)
+        host_plan.run(cuda_stream)
 
     e2e_step()
     barrier()

@@ -365,6 +365,42 @@ class BucketAllreducePlan:
             raise CCError(st, "cc_bucket_allreduce")
 
 
+class BucketAllreduceHostPlan:
+    """cc_bucket_allreduce_host with the marshalling done once (see BucketAllreducePlan)."""
+
+    def __init__(self, host_grads, host_out, dev_grads, dev_out, *, cap_bytes: int = 25 * 1024 * 1024,
+                 algo="ring", scale=None):
+        torch = _torch()
+        n, nt = _ranks(host_grads, "BucketAllreduceHostPlan"), len(host_grads[0])
+        for grid in (host_out, dev_grads, dev_out):
+            if len(grid) != n or any(len(row) != nt for row in grid):
+                raise ValueError("BucketAllreduceHostPlan: all four tables must be [nranks][ntensors]")
+        for i in range(nt):
+            ts = [g[r][i] for g in (host_grads, host_out, dev_grads, dev_out) for r in range(n)]
+            _same(ts, host_grads[0][i].numel(), torch.float32, f"BucketAllreduceHostPlan tensor {i}")
+        for grid in (host_grads, host_out):
+            for row in grid:
+                for t in row:
+                    if t.is_cuda or not t.is_contiguous():
+                        raise ValueError("BucketAllreduceHostPlan: host tables hold contiguous CPU tensors")
+        self._keep = (host_grads, host_out, dev_grads, dev_out)
+        self.n, self.nt = n, nt
+        hp = lambda grid: (ctypes.c_void_p * (n * nt))(*[t.data_ptr() for row in grid for t in row])
+        self._hin, self._hout = hp(host_grads), hp(host_out)
+        self._din = _ptrs([t for row in dev_grads for t in row])
+        self._dout = _ptrs([t for row in dev_out for t in row])
+        self._numels = _sizes([t.numel() for t in host_grads[0]])
+        self.cap_bytes, self.algo = int(cap_bytes), _ALGOS[algo]
+        self.scale = float(1.0 / n if scale is None else scale)
+        self._fn = get_lib().cc_bucket_allreduce_host
+
+    def run(self, stream=None) -> None:
+        st = self._fn(self._hin, self._hout, self._din, self._dout, self.n, self.nt, self._numels, self.cap_bytes,
+                      self.algo, self.scale, _stream(stream))
+        if st != CC_OK:
+            raise CCError(st, "cc_bucket_allreduce_host")
+
+
 def cc_bucket_allreduce_host(host_grads, host_out, dev_grads, dev_out, *, cap_bytes: int = 25 * 1024 * 1024,
                              algo="ring", scale=None, stream=None) -> None:
     """The fused DDP step on host-resident gradients: host -> device copies, the fused

@@ -2,6 +2,7 @@
 // Nothing here allocates device memory; every call is stream-ordered and returns after
 // enqueuing (only argument and launch errors are reported synchronously).
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "cc_launch.h"
@@ -44,6 +45,127 @@ void chunk_bounds(size_t count, int n, int c, size_t& a, size_t& len) {
 }
 
 cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+// Bucket layout of a tensor list: ids in bucket order, bucket boundaries, per-tensor
+// descriptors (offset and element count of the tensor's bucket).
+struct BucketLayout {
+  std::vector<int32_t> order, start;
+  std::vector<BucketTensorDesc> desc;
+  int32_t nb = 0;
+};
+
+BucketLayout bucket_layout(const size_t* numels, int ntensors, size_t cap_bytes) {
+  BucketLayout L;
+  L.order.resize(ntensors);
+  L.start.resize(ntensors + 1);
+  L.desc.resize(ntensors);
+  cc_bucket_assign(numels, ntensors, 4, cap_bytes, L.order.data(), L.start.data(), &L.nb);
+  for (int b = 0; b < L.nb; ++b) {
+    uint64_t count = 0;
+    for (int k = L.start[b]; k < L.start[b + 1]; ++k) count += numels[L.order[k]];
+    uint64_t off = 0;
+    for (int k = L.start[b]; k < L.start[b + 1]; ++k) {
+      L.desc[L.order[k]] = BucketTensorDesc{numels[L.order[k]], off, count};
+      off += numels[L.order[k]];
+    }
+  }
+  return L;
+}
+
+// Launch groups (at most bucket_group_limit tensors each, empty tensors skipped) for the
+// tensors order[first .. last).
+cudaError_t launch_bucket_range(const void* const* grads, void* const* out, int nranks, int ntensors,
+                                const BucketLayout& L, int first, int last, FoldKind fold, float scale,
+                                cudaStream_t s) {
+  const int limit = bucket_group_limit(nranks);
+  std::vector<int32_t> ids;
+  ids.reserve(limit);
+  for (int k = first; k <= last; ++k) {
+    if (k < last && L.desc[L.order[k]].numel > 0) ids.push_back(L.order[k]);
+    if ((int)ids.size() == limit || (k == last && !ids.empty())) {
+      cudaError_t err =
+          launch_bucket_allreduce(grads, out, nranks, ntensors, ids.data(), (int)ids.size(), L.desc.data(), fold, scale, s);
+      if (err != cudaSuccess) return err;
+      ids.clear();
+    }
+  }
+  return cudaSuccess;
+}
+
+// Streams and events of the host-buffer pipeline, created once per device and kept.
+struct HostPipeline {
+  std::mutex mu;
+  bool ready = false;
+  cudaStream_t in = nullptr, out = nullptr;
+  std::vector<cudaEvent_t> ev;  // grows on demand
+  cudaEvent_t event(size_t i) {
+    while (ev.size() <= i) {
+      cudaEvent_t e = nullptr;
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+      ev.push_back(e);
+    }
+    return ev[i];
+  }
+};
+HostPipeline g_pipe[64];
+
+// H2D of bucket b on one stream, its fused allreduce on the caller's stream, D2H of
+// bucket b on a third stream: the two copy directions and the kernels overlap bucket by
+// bucket, and the caller's stream ends after the last device-to-host copy.
+cudaError_t bucket_allreduce_pipelined(const void* const* hg, void* const* ho, void* const* dg, void* const* dout,
+                                       int nranks, int ntensors, const size_t* numels, size_t cap_bytes, FoldKind fold,
+                                       float scale, cudaStream_t s) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  HostPipeline& P = g_pipe[dev];
+  std::lock_guard<std::mutex> lock(P.mu);
+  if (!P.ready) {
+    if ((e = cudaStreamCreateWithFlags(&P.in, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaStreamCreateWithFlags(&P.out, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    P.ready = true;
+  }
+  const BucketLayout L = bucket_layout(numels, ntensors, cap_bytes);
+  size_t ne = 0;
+  auto next_event = [&]() { return P.event(ne++); };
+  cudaEvent_t start = next_event();
+  if (!start) return cudaErrorMemoryAllocation;
+  if ((e = cudaEventRecord(start, s)) != cudaSuccess) return e;
+  if ((e = cudaStreamWaitEvent(P.in, start, 0)) != cudaSuccess) return e;
+  if ((e = cudaStreamWaitEvent(P.out, start, 0)) != cudaSuccess) return e;
+  for (int b = 0; b < L.nb; ++b) {
+    for (int k = L.start[b]; k < L.start[b + 1]; ++k) {
+      const int i = L.order[k];
+      for (int r = 0; r < nranks; ++r) {
+        const size_t j = (size_t)r * ntensors + i;
+        if (numels[i] && (e = cudaMemcpyAsync(dg[j], hg[j], numels[i] * 4, cudaMemcpyHostToDevice, P.in)) != cudaSuccess)
+          return e;
+      }
+    }
+    cudaEvent_t in_done = next_event(), red_done = next_event();
+    if (!in_done || !red_done) return cudaErrorMemoryAllocation;
+    if ((e = cudaEventRecord(in_done, P.in)) != cudaSuccess) return e;
+    if ((e = cudaStreamWaitEvent(s, in_done, 0)) != cudaSuccess) return e;
+    if ((e = launch_bucket_range((const void* const*)dg, dout, nranks, ntensors, L, L.start[b], L.start[b + 1], fold,
+                                 scale, s)) != cudaSuccess)
+      return e;
+    if ((e = cudaEventRecord(red_done, s)) != cudaSuccess) return e;
+    if ((e = cudaStreamWaitEvent(P.out, red_done, 0)) != cudaSuccess) return e;
+    for (int k = L.start[b]; k < L.start[b + 1]; ++k) {
+      const int i = L.order[k];
+      for (int r = 0; r < nranks; ++r) {
+        const size_t j = (size_t)r * ntensors + i;
+        if (numels[i] && (e = cudaMemcpyAsync(ho[j], dout[j], numels[i] * 4, cudaMemcpyDeviceToHost, P.out)) != cudaSuccess)
+          return e;
+      }
+    }
+  }
+  cudaEvent_t end = next_event();
+  if (!end) return cudaErrorMemoryAllocation;
+  if ((e = cudaEventRecord(end, P.out)) != cudaSuccess) return e;
+  return cudaStreamWaitEvent(s, end, 0);
+}
 
 }  // namespace
 
@@ -285,61 +407,27 @@ cc_status cc_bucket_allreduce(const void* const* grads, void* const* out, int nr
     for (int i = 0; i < ntensors; ++i)
       if (numels[i] && (!grads[(size_t)r * ntensors + i] || !out[(size_t)r * ntensors + i]))
         return CC_ERR_INVALID_ARG;  // empty tensors may be null
-  std::vector<int32_t> order(ntensors), start(ntensors + 1);
-  int32_t nb = 0;
-  cc_bucket_assign(numels, ntensors, 4, cap_bytes, order.data(), start.data(), &nb);
-  std::vector<BucketTensorDesc> desc(ntensors);
-  for (int b = 0; b < nb; ++b) {
-    uint64_t count = 0;
-    for (int k = start[b]; k < start[b + 1]; ++k) count += numels[order[k]];
-    uint64_t off = 0;
-    for (int k = start[b]; k < start[b + 1]; ++k) {
-      desc[order[k]] = BucketTensorDesc{numels[order[k]], off, count};
-      off += numels[order[k]];
-    }
-  }
-  // launch groups in bucket order, skipping empty tensors
-  const int limit = bucket_group_limit(nranks);
-  std::vector<int32_t> ids;
-  ids.reserve(limit);
-  const FoldKind fold = algo == CC_ALGO_RING ? kFoldRing : kFoldTree;
-  for (int k = 0; k <= ntensors; ++k) {
-    if (k < ntensors && numels[order[k]] > 0) ids.push_back(order[k]);
-    if ((int)ids.size() == limit || (k == ntensors && !ids.empty())) {
-      cudaError_t err = launch_bucket_allreduce(grads, out, nranks, ntensors, ids.data(), (int)ids.size(),
-                                                desc.data(), fold, scale, as_stream(stream));
-      if (err != cudaSuccess) return CC_ERR_CUDA;
-      ids.clear();
-    }
-  }
+  const BucketLayout L = bucket_layout(numels, ntensors, cap_bytes);
+  if (launch_bucket_range(grads, out, nranks, ntensors, L, 0, ntensors, algo == CC_ALGO_RING ? kFoldRing : kFoldTree,
+                          scale, as_stream(stream)) != cudaSuccess)
+    return CC_ERR_CUDA;
   return CC_OK;
 }
 
 cc_status cc_bucket_allreduce_host(const void* const* host_grads, void* const* host_out, void* const* dev_grads,
                                    void* const* dev_out, int nranks, int ntensors, const size_t* numels,
                                    size_t cap_bytes, cc_algo algo, float scale, void* stream) {
-  if (!valid_ranks(nranks) || ntensors < 0 || cap_bytes == 0) return CC_ERR_INVALID_ARG;
+  if (!valid_ranks(nranks) || ntensors < 0 || cap_bytes == 0 || !(scale == scale)) return CC_ERR_INVALID_ARG;
+  if (algo != CC_ALGO_RING && algo != CC_ALGO_TREE) return CC_ERR_INVALID_ARG;
   if (ntensors == 0) return CC_OK;
   if (!host_grads || !host_out || !dev_grads || !dev_out || !numels) return CC_ERR_INVALID_ARG;
   const size_t total = (size_t)nranks * ntensors;
   for (size_t j = 0; j < total; ++j)
     if (numels[j % ntensors] && (!host_grads[j] || !host_out[j] || !dev_grads[j] || !dev_out[j]))
       return CC_ERR_INVALID_ARG;
-  cudaStream_t s = as_stream(stream);
-  for (size_t j = 0; j < total; ++j) {
-    const size_t nb = numels[j % ntensors] * 4;
-    if (nb && cudaMemcpyAsync(dev_grads[j], host_grads[j], nb, cudaMemcpyHostToDevice, s) != cudaSuccess)
-      return CC_ERR_CUDA;
-  }
-  cc_status st = cc_bucket_allreduce((const void* const*)dev_grads, dev_out, nranks, ntensors, numels, cap_bytes,
-                                     algo, scale, stream);
-  if (st != CC_OK) return st;
-  for (size_t j = 0; j < total; ++j) {
-    const size_t nb = numels[j % ntensors] * 4;
-    if (nb && cudaMemcpyAsync(host_out[j], dev_out[j], nb, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-      return CC_ERR_CUDA;
-  }
-  return CC_OK;
+  return cuda_status(bucket_allreduce_pipelined(host_grads, host_out, dev_grads, dev_out, nranks, ntensors, numels,
+                                                cap_bytes, algo == CC_ALGO_RING ? kFoldRing : kFoldTree, scale,
+                                                as_stream(stream)));
 }
 
 }  // extern "C"

@@ -143,12 +143,26 @@ template <int IN, int OP> __device__ __forceinline__ void comb(typename Tr<IN>::
   a = op<IN, OP>(a, b);
 }
 
-template <typename V> struct FoldStack {
-  V s[kStackSlots];
+// U units side by side (U columns of one thread), and U raw loads: small rank counts fold
+// several columns at once so that a thread still has about 8 loads in flight.
+template <int IN, int U> struct MU { Unit<IN> u[U]; };
+template <int U> struct MX { uint4 w[U]; };
+template <int IN, int OP, int U> __device__ __forceinline__ void comb(MU<IN, U>& a, const MU<IN, U>& b) {
+#pragma unroll
+  for (int k = 0; k < U; ++k) op_unit<IN, OP>(a.u[k], b.u[k]);
+}
+template <int IN, int OP, int U> __device__ __forceinline__ void comb(MU<IN, U>& a, const MX<U>& b) {
+#pragma unroll
+  for (int k = 0; k < U; ++k) op_unit<IN, OP>(a.u[k], to_unit<IN>(b.w[k]));
+}
+
+template <typename V, int S = kStackSlots> struct FoldStack {
+  static_assert(S >= 1 && S <= 8, "1..8 stack slots");
+  V s[S];
   int depth = 0;
   __device__ __forceinline__ void push(const V& u) {
     switch (depth) {
-#define CC_PUSH_CASE(k) case k: s[k] = u; break;
+#define CC_PUSH_CASE(k) case k: if constexpr (k < S) s[k] = u; break;
       CC_PUSH_CASE(0) CC_PUSH_CASE(1) CC_PUSH_CASE(2) CC_PUSH_CASE(3)
       CC_PUSH_CASE(4) CC_PUSH_CASE(5) CC_PUSH_CASE(6) CC_PUSH_CASE(7)
 #undef CC_PUSH_CASE
@@ -157,16 +171,16 @@ template <typename V> struct FoldStack {
   }
   __device__ __forceinline__ V top() const {
     switch (depth - 1) {
-#define CC_TOP_CASE(k) case k: return s[k];
+#define CC_TOP_CASE(k) case k: if constexpr (k < S) return s[k]; break;
       CC_TOP_CASE(0) CC_TOP_CASE(1) CC_TOP_CASE(2) CC_TOP_CASE(3)
       CC_TOP_CASE(4) CC_TOP_CASE(5) CC_TOP_CASE(6)
 #undef CC_TOP_CASE
-      default: return s[7];
     }
+    return s[S - 1];
   }
   __device__ __forceinline__ void set_top(const V& u) {
     switch (depth - 1) {
-#define CC_SET_CASE(k) case k: s[k] = u; break;
+#define CC_SET_CASE(k) case k: if constexpr (k < S) s[k] = u; break;
       CC_SET_CASE(0) CC_SET_CASE(1) CC_SET_CASE(2) CC_SET_CASE(3)
       CC_SET_CASE(4) CC_SET_CASE(5) CC_SET_CASE(6) CC_SET_CASE(7)
 #undef CC_SET_CASE
@@ -175,8 +189,8 @@ template <typename V> struct FoldStack {
 };
 
 // One position of the machine; `x` is the position's loaded value (a unit or an element).
-template <int IN, int OP, typename V>
-__device__ __forceinline__ void fold_step(uint8_t code, const V& x, V& cur, FoldStack<V>& st) {
+template <int IN, int OP, typename V, int S>
+__device__ __forceinline__ void fold_step(uint8_t code, const V& x, V& cur, FoldStack<V, S>& st) {
   V node = x;
   if (code & kFoldCur) { node = cur; comb<IN, OP>(node, x); }
   if (code & kPush) st.push(node); else cur = node;

@@ -33,27 +33,27 @@ constexpr int kThreads = 256;
 // 128-bit loads per thread are in flight before the in-order folds consume them.
 // V is the accumulator (a unit or an element), X what one load returns (raw 16 bytes for a
 // unit, the element itself otherwise).
-template <int IN, int OP, typename V, typename X, typename Load, typename Widen>
+template <int IN, int OP, typename V, typename X, int W = 8, typename Load, typename Widen>
 __device__ __forceinline__ V ring_fold(int n, int c, Load ld, Widen widen) {
   V acc = widen(ld(c));
   int r = c;
-  for (int j0 = 1; j0 < n; j0 += 8) {
-    X x[8];
+  for (int j0 = 1; j0 < n; j0 += W) {
+    X x[W];
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
+    for (int k = 0; k < W; ++k)
       if (j0 + k < n) { r = (r + 1 == n) ? 0 : r + 1; x[k] = ld(r); }
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
+    for (int k = 0; k < W; ++k)
       if (j0 + k < n) comb<IN, OP>(acc, x[k]);
   }
   return acc;
 }
 
 // Fold machine (tree / binomial): the position's rank is rmap[p], mirrored for tree B.
-template <int IN, int OP, typename V, typename X, int W, typename Load, typename Widen>
+template <int IN, int OP, typename V, typename X, int W, int S = kStackSlots, typename Load, typename Widen>
 __device__ __forceinline__ V machine_fold(int n, const FoldProgram& prog, bool mirror, Load ld, Widen widen) {
   V cur;
-  FoldStack<V> st;
+  FoldStack<V, S> st;
   for (int p0 = 0; p0 < n; p0 += W) {
     X x[W];
 #pragma unroll
@@ -69,34 +69,53 @@ __device__ __forceinline__ V machine_fold(int n, const FoldProgram& prog, bool m
   return cur;
 }
 
+// Pending-partial slots the fold machine needs with U columns per thread: U > 1 is only
+// used for N <= 8 / U ranks, whose trees need at most 2 (U = 4) or 3 (U = 2) slots.
+template <int U> constexpr int stack_slots() { return U == 1 ? kStackSlots : (U == 2 ? 4 : 2); }
+
 // Elements [a, b) of one fold group, spread over threads t = 0..T-1: 16-byte units where
-// every address is aligned, element-wise head and tail around them.
-template <int IN, int OP, bool RING, typename Src, typename EmitU, typename EmitE>
+// every address is aligned, element-wise head and tail around them. Each thread folds U
+// units at once (units T apart, so warps stay coalesced) with windows of 8 / U positions:
+// about 8 loads in flight per thread for any rank count.
+template <int IN, int OP, bool RING, int U, typename Src, typename EmitU, typename EmitE>
 __device__ __forceinline__ void reduce_range(int n, int g, bool mirror, const FoldProgram& prog,
                                              uint64_t a, uint64_t b, uint64_t t, uint64_t T, bool vec,
                                              Src src, EmitU emit_unit, EmitE emit_elem) {
-  using In = typename Tr<IN>::In;
   using A = typename Tr<IN>::Acc;
   constexpr int UE = Tr<IN>::UE;
-  constexpr int W = 8;
-  auto same = [](const A& a) { return a; };
-  auto widen = [](const uint4& w) { return to_unit<IN>(w); };
+  constexpr int W = 8 / U;
+  auto same = [](const A& x) { return x; };
   auto fold_elem = [&](uint64_t e) -> A {
     auto ld = [&](int r) { return load_elem<IN>(src(r) + e); };
     if constexpr (RING) return ring_fold<IN, OP, A, A>(n, g, ld, same);
-    else return machine_fold<IN, OP, A, A, W>(n, prog, mirror, ld, same);
+    else return machine_fold<IN, OP, A, A, 8>(n, prog, mirror, ld, same);
   };
   if (vec) {
     uint64_t va = (a + UE - 1) / UE * UE;
     if (va > b) va = b;
     uint64_t vb = b / UE * UE;
     if (vb < va) vb = va;
-    for (uint64_t e = va + t * UE; e < vb; e += T * UE) {
-      auto ld = [&](int r) { return load_raw(src(r) + e); };
-      Unit<IN> u;
-      if constexpr (RING) u = ring_fold<IN, OP, Unit<IN>, uint4>(n, g, ld, widen);
-      else u = machine_fold<IN, OP, Unit<IN>, uint4, W>(n, prog, mirror, ld, widen);
-      emit_unit(e, u);
+    const uint64_t step = T * UE;
+    auto widen = [](const MX<U>& x) {
+      MU<IN, U> m;
+#pragma unroll
+      for (int k = 0; k < U; ++k) m.u[k] = to_unit<IN>(x.w[k]);
+      return m;
+    };
+    for (uint64_t e0 = va + t * UE; e0 < vb; e0 += step * U) {
+      auto ld = [&](int r) {
+        MX<U> x;
+#pragma unroll
+        for (int k = 0; k < U; ++k)
+          if (k == 0 || e0 + k * step < vb) x.w[k] = load_raw(src(r) + e0 + k * step);
+        return x;
+      };
+      MU<IN, U> m;
+      if constexpr (RING) m = ring_fold<IN, OP, MU<IN, U>, MX<U>, W>(n, g, ld, widen);
+      else m = machine_fold<IN, OP, MU<IN, U>, MX<U>, W, stack_slots<U>()>(n, prog, mirror, ld, widen);
+#pragma unroll
+      for (int k = 0; k < U; ++k)
+        if (k == 0 || e0 + k * step < vb) emit_unit(e0 + k * step, m.u[k]);
     }
     const uint64_t nh = va - a, nt = b - vb;
     if (t < nh) emit_elem(a + t, fold_elem(a + t));
@@ -168,8 +187,8 @@ struct ReduceParams {
 // Persistent CTAs take contiguous tiles round-robin (the grid is oversubscribed twice over
 // the resident CTAs, which measured faster than one wave); a tile is split where it crosses
 // a fold group (ring chunk or tree half) and each piece is folded by the whole CTA.
-template <int IN, int OP, bool RING>
-__global__ void __launch_bounds__(kThreads, RING ? CC_RING_MIN_BLOCKS : 2) reduce_kernel(const __grid_constant__ ReduceParams P) {
+template <int IN, int OP, bool RING, int U>
+__global__ void __launch_bounds__(kThreads, (RING && U == 1) ? CC_RING_MIN_BLOCKS : 2) reduce_kernel(const __grid_constant__ ReduceParams P) {
   using In = typename Tr<IN>::In;
   using Out = typename Tr<IN>::Out;
   using A = typename Tr<IN>::Acc;
@@ -207,8 +226,8 @@ __global__ void __launch_bounds__(kThreads, RING ? CC_RING_MIN_BLOCKS : 2) reduc
           store_elem<IN>(static_cast<Out*>(P.dst[0]) + e, v);
         }
       };
-      reduce_range<IN, OP, RING>(n, g, mirror, P.prog, s, se, threadIdx.x, blockDim.x, P.vec != 0, src, emit_unit,
-                                 emit_elem);
+      reduce_range<IN, OP, RING, U>(n, g, mirror, P.prog, s, se, threadIdx.x, blockDim.x, P.vec != 0, src, emit_unit,
+                                    emit_elem);
       s = se;
     }
   }
@@ -293,8 +312,8 @@ __global__ void __launch_bounds__(kThreads, RING ? 3 : 2) bucket_allreduce_kerne
         gend = g ? d.bucket_count : mid;
       }
       const uint64_t se = min(eb, gend - d.bucket_off);
-      reduce_range<IN, OP, RING>(n, g, !RING && g == 1, P.prog, s, se, threadIdx.x, blockDim.x,
-                                 P.vec != 0, src, emit_unit, emit_elem);
+      reduce_range<IN, OP, RING, 1>(n, g, !RING && g == 1, P.prog, s, se, threadIdx.x, blockDim.x,
+                                    P.vec != 0, src, emit_unit, emit_elem);
       s = se;
     }
     __syncthreads();  // every thread is done with s_in / s_out before the next tile restages them
@@ -404,11 +423,11 @@ static int blocks_per_sm(K kernel) {
   return b;
 }
 
-template <int IN, int OP, bool RING>
+template <int IN, int OP, bool RING, int U>
 static cudaError_t run_reduce(ReduceParams& P, cudaStream_t s) {
-  auto k = reduce_kernel<IN, OP, RING>;
+  auto k = reduce_kernel<IN, OP, RING, U>;
   static const int bps = blocks_per_sm(k);
-  constexpr uint64_t UE = Tr<IN>::UE;
+  constexpr uint64_t UE = Tr<IN>::UE * U;
   const uint64_t resident = (uint64_t)sm_count() * bps;
   // tiles of 1..8 units per thread: large buffers get 8 (long contiguous streams per CTA),
   // small ones shrink the tile so that every resident CTA still gets work
@@ -422,15 +441,30 @@ static cudaError_t run_reduce(ReduceParams& P, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// Columns per thread for SUM (the other operators fold one column): 4 for N <= 2, 2 for
+// N <= 4, else 1 (when the fold program fits the smaller stack).
 template <int IN>
-static cudaError_t dispatch_op(ReduceParams& P, cc_op op, bool ring, cudaStream_t s) {
+static cudaError_t dispatch_op(ReduceParams& P, cc_op op, bool ring, int cols, cudaStream_t s) {
   switch (op) {
-    case CC_SUM: return ring ? run_reduce<IN, CC_SUM, true>(P, s) : run_reduce<IN, CC_SUM, false>(P, s);
-    case CC_MAX: return ring ? run_reduce<IN, CC_MAX, true>(P, s) : run_reduce<IN, CC_MAX, false>(P, s);
-    case CC_MIN: return ring ? run_reduce<IN, CC_MIN, true>(P, s) : run_reduce<IN, CC_MIN, false>(P, s);
-    case CC_PROD: return ring ? run_reduce<IN, CC_PROD, true>(P, s) : run_reduce<IN, CC_PROD, false>(P, s);
+    case CC_SUM:
+      if (cols == 4) return ring ? run_reduce<IN, CC_SUM, true, 4>(P, s) : run_reduce<IN, CC_SUM, false, 4>(P, s);
+      if (cols == 2) return ring ? run_reduce<IN, CC_SUM, true, 2>(P, s) : run_reduce<IN, CC_SUM, false, 2>(P, s);
+      return ring ? run_reduce<IN, CC_SUM, true, 1>(P, s) : run_reduce<IN, CC_SUM, false, 1>(P, s);
+    case CC_MAX: return ring ? run_reduce<IN, CC_MAX, true, 1>(P, s) : run_reduce<IN, CC_MAX, false, 1>(P, s);
+    case CC_MIN: return ring ? run_reduce<IN, CC_MIN, true, 1>(P, s) : run_reduce<IN, CC_MIN, false, 1>(P, s);
+    case CC_PROD: return ring ? run_reduce<IN, CC_PROD, true, 1>(P, s) : run_reduce<IN, CC_PROD, false, 1>(P, s);
   }
   return cudaErrorInvalidValue;
+}
+
+// Deepest stack of pending partials a fold program reaches.
+static int program_depth(int n, const FoldProgram& fp) {
+  int d = 0, m = 0;
+  for (int p = 0; p < n; ++p) {
+    if (fp.code[p] & kPush) m = std::max(m, ++d);
+    d -= npop_of(fp.code[p]);
+  }
+  return m;
 }
 
 cudaError_t launch_reduce(const void* const* send, void* const* dst, int ndst, int nranks, size_t count,
@@ -457,10 +491,16 @@ cudaError_t launch_reduce(const void* const* send, void* const* dst, int ndst, i
   if (fold == kFoldTree) tree_program(nranks, P.prog);
   else if (fold == kFoldBinomial) binomial_program(nranks, root, P.prog);
   const bool ring = fold == kFoldRing;
+  int cols = nranks <= 2 ? 4 : (nranks <= 4 ? 2 : 1);
+  if (in_t == CC_BF16) cols = std::min(cols, 2);  // a bf16 column already holds 8 elements
+  if (!ring) {
+    const int depth = program_depth(nranks, P.prog);
+    if (depth > (cols == 4 ? 2 : cols == 2 ? 4 : kStackSlots)) cols = 1;
+  }
   switch (in_t) {
-    case CC_F32: return dispatch_op<CC_F32>(P, op, ring, stream);
-    case CC_BF16: return dispatch_op<CC_BF16>(P, op, ring, stream);
-    case CC_I32: return dispatch_op<CC_I32>(P, op, ring, stream);
+    case CC_F32: return dispatch_op<CC_F32>(P, op, ring, cols, stream);
+    case CC_BF16: return dispatch_op<CC_BF16>(P, op, ring, cols, stream);
+    case CC_I32: return dispatch_op<CC_I32>(P, op, ring, cols, stream);
   }
   return cudaErrorInvalidValue;
 }

@@ -126,6 +126,24 @@ def test_bucket_plan_matches_direct_call():
             assert np.array_equal(bits(to_host(out[r][i])), bits(want[r][i]))
 
 
+@pytest.mark.parametrize("cap", [30_000, 25 * 1024 * 1024])
+def test_host_buffer_pipeline_matches_oracle(cap):
+    n = 8
+    shapes, grads = _small_model(n, seed=7)
+    want, _ = ddp.ddp_allreduce(grads, cap_bytes=cap)
+    h_in = [[torch.from_numpy(g).pin_memory() for g in row] for row in grads]
+    h_out = [[torch.empty(g.shape, dtype=torch.float32).pin_memory() for g in row] for row in grads]
+    d_in = [[torch.empty(g.shape, device="cuda") for g in row] for row in grads]
+    d_out = [[torch.empty(g.shape, device="cuda") for g in row] for row in grads]
+    plan = cc.BucketAllreduceHostPlan(h_in, h_out, d_in, d_out, cap_bytes=cap)
+    for _ in range(2):
+        plan.run()
+    torch.cuda.synchronize()
+    for r in range(n):
+        for i in range(len(shapes)):
+            assert np.array_equal(bits(h_out[r][i].numpy()), bits(want[r][i])), f"rank {r} tensor {i}"
+
+
 def test_flatten_allreduce_unflatten_equals_fused():
     n, cap = 8, 60_000
     shapes, grads = _small_model(n, seed=4)
