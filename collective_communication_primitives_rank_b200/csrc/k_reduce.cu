@@ -441,8 +441,7 @@ static cudaError_t run_reduce(ReduceParams& P, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-// Columns per thread for SUM (the other operators fold one column): 4 for N <= 2, 2 for
-// N <= 4, else 1 (when the fold program fits the smaller stack).
+// Columns per thread for SUM (the other operators fold one column).
 template <int IN>
 static cudaError_t dispatch_op(ReduceParams& P, cc_op op, bool ring, int cols, cudaStream_t s) {
   switch (op) {
@@ -491,7 +490,9 @@ cudaError_t launch_reduce(const void* const* send, void* const* dst, int ndst, i
   if (fold == kFoldTree) tree_program(nranks, P.prog);
   else if (fold == kFoldBinomial) binomial_program(nranks, root, P.prog);
   const bool ring = fold == kFoldRing;
-  int cols = nranks <= 2 ? 4 : (nranks <= 4 ? 2 : 1);
+  // several columns per thread pay off for the fold machine (tree, binomial) at small N;
+  // the ring's plain left fold is faster with one column and twice the resident CTAs
+  int cols = ring ? 1 : (nranks <= 2 ? 4 : (nranks <= 4 ? 2 : 1));
   if (in_t == CC_BF16) cols = std::min(cols, 2);  // a bf16 column already holds 8 elements
   if (!ring) {
     const int depth = program_depth(nranks, P.prog);
