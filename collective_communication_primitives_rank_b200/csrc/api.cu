@@ -1,6 +1,7 @@
 // C-ABI entry points of libcc: argument validation, then a launch of the matching kernel.
 // Nothing here allocates device memory; every call is stream-ordered and returns after
 // enqueuing (only argument and launch errors are reported synchronously).
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -109,9 +110,16 @@ struct HostPipeline {
 };
 HostPipeline g_pipe[64];
 
-// H2D of bucket b on one stream, its fused allreduce on the caller's stream, D2H of
-// bucket b on a third stream: the two copy directions and the kernels overlap bucket by
-// bucket, and the caller's stream ends after the last device-to-host copy.
+// Host-buffer pipeline. The gradients are cut, in bucket order, into slices of at most
+// kSliceElems elements per rank; consecutive slices form stages of about kStageElems per
+// rank. A stage's host-to-device copies run on one stream, its fused allreduce on the
+// caller's stream, its device-to-host copies on a third stream, so the two PCIe directions
+// and the kernels overlap stage by stage. A slice keeps its offset inside its bucket, so
+// every element is folded exactly as in the unsliced call. The caller's stream ends after
+// the last device-to-host copy.
+constexpr uint64_t kSliceElems = 1ull << 20;
+constexpr uint64_t kStageElems = 2ull << 20;
+
 cudaError_t bucket_allreduce_pipelined(const void* const* hg, void* const* ho, void* const* dg, void* const* dout,
                                        int nranks, int ntensors, const size_t* numels, size_t cap_bytes, FoldKind fold,
                                        float scale, cudaStream_t s) {
@@ -134,33 +142,77 @@ cudaError_t bucket_allreduce_pipelined(const void* const* hg, void* const* ho, v
   if ((e = cudaEventRecord(start, s)) != cudaSuccess) return e;
   if ((e = cudaStreamWaitEvent(P.in, start, 0)) != cudaSuccess) return e;
   if ((e = cudaStreamWaitEvent(P.out, start, 0)) != cudaSuccess) return e;
-  for (int b = 0; b < L.nb; ++b) {
-    for (int k = L.start[b]; k < L.start[b + 1]; ++k) {
-      const int i = L.order[k];
+
+  struct Slice { int i; uint64_t a, len; };
+  std::vector<Slice> stage;
+  uint64_t stage_elems = 0;
+  std::vector<const void*> vg;
+  std::vector<void*> vo;
+  std::vector<BucketTensorDesc> vd;
+  std::vector<int32_t> ids;
+  const int limit = bucket_group_limit(nranks);
+  auto at = [](const void* p, uint64_t elems) { return static_cast<const char*>(p) + elems * 4; };
+  auto atw = [](void* p, uint64_t elems) { return static_cast<char*>(p) + elems * 4; };
+
+  auto run_stage = [&]() -> cudaError_t {
+    cudaError_t err;
+    for (const Slice& c : stage)
       for (int r = 0; r < nranks; ++r) {
-        const size_t j = (size_t)r * ntensors + i;
-        if (numels[i] && (e = cudaMemcpyAsync(dg[j], hg[j], numels[i] * 4, cudaMemcpyHostToDevice, P.in)) != cudaSuccess)
-          return e;
+        const size_t j = (size_t)r * ntensors + c.i;
+        if ((err = cudaMemcpyAsync(atw(dg[j], c.a), at(hg[j], c.a), c.len * 4, cudaMemcpyHostToDevice, P.in)) !=
+            cudaSuccess)
+          return err;
       }
-    }
     cudaEvent_t in_done = next_event(), red_done = next_event();
     if (!in_done || !red_done) return cudaErrorMemoryAllocation;
-    if ((e = cudaEventRecord(in_done, P.in)) != cudaSuccess) return e;
-    if ((e = cudaStreamWaitEvent(s, in_done, 0)) != cudaSuccess) return e;
-    if ((e = launch_bucket_range((const void* const*)dg, dout, nranks, ntensors, L, L.start[b], L.start[b + 1], fold,
-                                 scale, s)) != cudaSuccess)
-      return e;
-    if ((e = cudaEventRecord(red_done, s)) != cudaSuccess) return e;
-    if ((e = cudaStreamWaitEvent(P.out, red_done, 0)) != cudaSuccess) return e;
-    for (int k = L.start[b]; k < L.start[b + 1]; ++k) {
-      const int i = L.order[k];
-      for (int r = 0; r < nranks; ++r) {
-        const size_t j = (size_t)r * ntensors + i;
-        if (numels[i] && (e = cudaMemcpyAsync(ho[j], dout[j], numels[i] * 4, cudaMemcpyDeviceToHost, P.out)) != cudaSuccess)
-          return e;
+    if ((err = cudaEventRecord(in_done, P.in)) != cudaSuccess) return err;
+    if ((err = cudaStreamWaitEvent(s, in_done, 0)) != cudaSuccess) return err;
+    // the stage's slices as tensors of their own, launched in groups that fit one launch
+    for (size_t g0 = 0; g0 < stage.size(); g0 += limit) {
+      const int nv = (int)std::min<size_t>(limit, stage.size() - g0);
+      vg.assign((size_t)nranks * nv, nullptr);
+      vo.assign((size_t)nranks * nv, nullptr);
+      vd.resize(nv);
+      ids.resize(nv);
+      for (int v = 0; v < nv; ++v) {
+        const Slice& c = stage[g0 + v];
+        const BucketTensorDesc& d = L.desc[c.i];
+        vd[v] = BucketTensorDesc{c.len, d.bucket_off + c.a, d.bucket_count};
+        ids[v] = v;
+        for (int r = 0; r < nranks; ++r) {
+          const size_t j = (size_t)r * ntensors + c.i;
+          vg[(size_t)r * nv + v] = at(dg[j], c.a);
+          vo[(size_t)r * nv + v] = atw(dout[j], c.a);
+        }
       }
+      if ((err = launch_bucket_allreduce(vg.data(), vo.data(), nranks, nv, ids.data(), nv, vd.data(), fold, scale, s)) !=
+          cudaSuccess)
+        return err;
+    }
+    if ((err = cudaEventRecord(red_done, s)) != cudaSuccess) return err;
+    if ((err = cudaStreamWaitEvent(P.out, red_done, 0)) != cudaSuccess) return err;
+    for (const Slice& c : stage)
+      for (int r = 0; r < nranks; ++r) {
+        const size_t j = (size_t)r * ntensors + c.i;
+        if ((err = cudaMemcpyAsync(atw(ho[j], c.a), at(dout[j], c.a), c.len * 4, cudaMemcpyDeviceToHost, P.out)) !=
+            cudaSuccess)
+          return err;
+      }
+    stage.clear();
+    stage_elems = 0;
+    return cudaSuccess;
+  };
+
+  for (int k = 0; k < ntensors; ++k) {
+    const int i = L.order[k];
+    for (uint64_t a = 0; a < numels[i]; a += kSliceElems) {
+      const uint64_t len = std::min<uint64_t>(kSliceElems, numels[i] - a);
+      stage.push_back(Slice{i, a, len});
+      stage_elems += len;
+      if (stage_elems >= kStageElems && (e = run_stage()) != cudaSuccess) return e;
     }
   }
+  if (!stage.empty() && (e = run_stage()) != cudaSuccess) return e;
   cudaEvent_t end = next_event();
   if (!end) return cudaErrorMemoryAllocation;
   if ((e = cudaEventRecord(end, P.out)) != cudaSuccess) return e;

@@ -210,10 +210,15 @@ CC_API cc_status cc_bucket_allreduce(const void* const* grads, void* const* out,
                               void* stream);
 
 /* The same fused DDP step for gradients that live in host memory: every host_grads[j] is
- * copied to dev_grads[j] (host -> device), cc_bucket_allreduce runs on the device copies,
- * and every dev_out[j] is copied back to host_out[j] (device -> host), all stream-ordered
- * on `stream`. The caller owns the device staging buffers (dev_grads may equal dev_out);
- * pinned host memory makes the copies asynchronous. Layouts as cc_bucket_allreduce. */
+ * copied to dev_grads[j] (host -> device), the fused allreduce runs on the device copies,
+ * and every dev_out[j] is copied back to host_out[j] (device -> host). The work is cut in
+ * bucket order into slices (at most 2^20 elements per rank), and the copies in, the
+ * kernels and the copies out of consecutive slices overlap on two library-owned streams
+ * (created once per device) and `stream`; a slice keeps its bucket offset, so the results
+ * equal cc_bucket_allreduce's. From the caller's view the call is ordered on `stream`
+ * (it starts after earlier work on `stream`; later work on `stream` sees the host outputs
+ * written). The caller owns the device staging buffers (dev_grads may equal dev_out);
+ * host buffers must be pinned for the copies to overlap. Layouts as cc_bucket_allreduce. */
 CC_API cc_status cc_bucket_allreduce_host(const void* const* host_grads, void* const* host_out,
                                           void* const* dev_grads, void* const* dev_out, int nranks,
                                           int ntensors, const size_t* numels, size_t cap_bytes,
