@@ -143,39 +143,61 @@ cudaError_t bucket_allreduce_pipelined(const void* const* hg, void* const* ho, v
   if ((e = cudaStreamWaitEvent(P.in, start, 0)) != cudaSuccess) return e;
   if ((e = cudaStreamWaitEvent(P.out, start, 0)) != cudaSuccess) return e;
 
+  // cut the work into stages of slices, in bucket order
   struct Slice { int i; uint64_t a, len; };
-  std::vector<Slice> stage;
+  std::vector<std::vector<Slice>> stages(1);
   uint64_t stage_elems = 0;
+  for (int k = 0; k < ntensors; ++k) {
+    const int i = L.order[k];
+    for (uint64_t a = 0; a < numels[i]; a += kSliceElems) {
+      const uint64_t len = std::min<uint64_t>(kSliceElems, numels[i] - a);
+      stages.back().push_back(Slice{i, a, len});
+      stage_elems += len;
+      if (stage_elems >= kStageElems) {
+        stages.emplace_back();
+        stage_elems = 0;
+      }
+    }
+  }
+  if (stages.back().empty()) stages.pop_back();
+  const size_t ns = stages.size();
+  std::vector<cudaEvent_t> in_done(ns), red_done(ns);
+  for (size_t k = 0; k < ns; ++k) {
+    in_done[k] = next_event();
+    red_done[k] = next_event();
+    if (!in_done[k] || !red_done[k]) return cudaErrorMemoryAllocation;
+  }
+  auto at = [](const void* p, uint64_t elems) { return static_cast<const char*>(p) + elems * 4; };
+  auto atw = [](void* p, uint64_t elems) { return static_cast<char*>(p) + elems * 4; };
+  // enqueue order: copies in of stage k+1, then the kernels and the copies out of stage k, so
+  // that each stream is fed just ahead of where the GPU is (a stream fed thousands of
+  // commands ahead blocks the enqueuing thread until its queue drains)
   std::vector<const void*> vg;
   std::vector<void*> vo;
   std::vector<BucketTensorDesc> vd;
   std::vector<int32_t> ids;
-  const int limit = bucket_group_limit(nranks);
-  auto at = [](const void* p, uint64_t elems) { return static_cast<const char*>(p) + elems * 4; };
-  auto atw = [](void* p, uint64_t elems) { return static_cast<char*>(p) + elems * 4; };
-
-  auto run_stage = [&]() -> cudaError_t {
-    cudaError_t err;
-    for (const Slice& c : stage)
+  const int limit = bucket_small_group_limit(nranks);
+  auto copies_in = [&](size_t k) -> cudaError_t {
+    for (const Slice& c : stages[k])
       for (int r = 0; r < nranks; ++r) {
         const size_t j = (size_t)r * ntensors + c.i;
-        if ((err = cudaMemcpyAsync(atw(dg[j], c.a), at(hg[j], c.a), c.len * 4, cudaMemcpyHostToDevice, P.in)) !=
-            cudaSuccess)
-          return err;
+        cudaError_t err = cudaMemcpyAsync(atw(dg[j], c.a), at(hg[j], c.a), c.len * 4, cudaMemcpyHostToDevice, P.in);
+        if (err != cudaSuccess) return err;
       }
-    cudaEvent_t in_done = next_event(), red_done = next_event();
-    if (!in_done || !red_done) return cudaErrorMemoryAllocation;
-    if ((err = cudaEventRecord(in_done, P.in)) != cudaSuccess) return err;
-    if ((err = cudaStreamWaitEvent(s, in_done, 0)) != cudaSuccess) return err;
-    // the stage's slices as tensors of their own, launched in groups that fit one launch
-    for (size_t g0 = 0; g0 < stage.size(); g0 += limit) {
-      const int nv = (int)std::min<size_t>(limit, stage.size() - g0);
+    return cudaEventRecord(in_done[k], P.in);
+  };
+  auto reduce_and_copy_out = [&](size_t k) -> cudaError_t {
+    cudaError_t err;
+    if ((err = cudaStreamWaitEvent(s, in_done[k], 0)) != cudaSuccess) return err;
+    const std::vector<Slice>& st = stages[k];
+    for (size_t g0 = 0; g0 < st.size(); g0 += limit) {
+      const int nv = (int)std::min<size_t>(limit, st.size() - g0);
       vg.assign((size_t)nranks * nv, nullptr);
       vo.assign((size_t)nranks * nv, nullptr);
       vd.resize(nv);
       ids.resize(nv);
       for (int v = 0; v < nv; ++v) {
-        const Slice& c = stage[g0 + v];
+        const Slice& c = st[g0 + v];
         const BucketTensorDesc& d = L.desc[c.i];
         vd[v] = BucketTensorDesc{c.len, d.bucket_off + c.a, d.bucket_count};
         ids[v] = v;
@@ -189,30 +211,22 @@ cudaError_t bucket_allreduce_pipelined(const void* const* hg, void* const* ho, v
           cudaSuccess)
         return err;
     }
-    if ((err = cudaEventRecord(red_done, s)) != cudaSuccess) return err;
-    if ((err = cudaStreamWaitEvent(P.out, red_done, 0)) != cudaSuccess) return err;
-    for (const Slice& c : stage)
+    if ((err = cudaEventRecord(red_done[k], s)) != cudaSuccess) return err;
+    if ((err = cudaStreamWaitEvent(P.out, red_done[k], 0)) != cudaSuccess) return err;
+    for (const Slice& c : st)
       for (int r = 0; r < nranks; ++r) {
         const size_t j = (size_t)r * ntensors + c.i;
         if ((err = cudaMemcpyAsync(atw(ho[j], c.a), at(dout[j], c.a), c.len * 4, cudaMemcpyDeviceToHost, P.out)) !=
             cudaSuccess)
           return err;
       }
-    stage.clear();
-    stage_elems = 0;
     return cudaSuccess;
   };
-
-  for (int k = 0; k < ntensors; ++k) {
-    const int i = L.order[k];
-    for (uint64_t a = 0; a < numels[i]; a += kSliceElems) {
-      const uint64_t len = std::min<uint64_t>(kSliceElems, numels[i] - a);
-      stage.push_back(Slice{i, a, len});
-      stage_elems += len;
-      if (stage_elems >= kStageElems && (e = run_stage()) != cudaSuccess) return e;
-    }
+  if ((e = copies_in(0)) != cudaSuccess) return e;
+  for (size_t k = 0; k < ns; ++k) {
+    if (k + 1 < ns && (e = copies_in(k + 1)) != cudaSuccess) return e;
+    if ((e = reduce_and_copy_out(k)) != cudaSuccess) return e;
   }
-  if (!stage.empty() && (e = run_stage()) != cudaSuccess) return e;
   cudaEvent_t end = next_event();
   if (!end) return cudaErrorMemoryAllocation;
   if ((e = cudaEventRecord(end, P.out)) != cudaSuccess) return e;

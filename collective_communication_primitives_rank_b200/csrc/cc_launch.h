@@ -24,7 +24,8 @@ struct BucketTensorDesc {
   uint64_t bucket_off;    // element offset of the tensor inside its bucket
   uint64_t bucket_count;  // elements in the tensor's bucket
 };
-int bucket_group_limit(int nranks);  // tensors one launch can take
+int bucket_group_limit(int nranks);        // tensors one launch can take
+int bucket_small_group_limit(int nranks);  // tensors a launch with a small (< 4 KB) parameter block takes
 cudaError_t launch_bucket_allreduce(const void* const* grads, void* const* out, int nranks,
                                     int ntensors_total, const int32_t* ids, int nids,
                                     const BucketTensorDesc* desc, FoldKind fold, float scale,

@@ -245,7 +245,11 @@ constexpr int kBucketMaxTensors = 192;
 constexpr int kBucketMaxPtrs = 1536;
 constexpr uint64_t kBucketTile = 8192;
 
-struct BucketParams {
+// Tables travel as kernel parameters: a large block (up to 192 tensors, 30 KB) for whole
+// tensor lists, and a small one (under 4 KB) for the short lists of the host-buffer
+// pipeline, whose many queued launches would otherwise hold the driver's parameter space.
+template <int MAXT, int MAXP> struct BucketParamsT {
+  static constexpr int kMaxT = MAXT, kMaxP = MAXP;
   int nranks;
   int ntensors;
   int fold;
@@ -253,15 +257,18 @@ struct BucketParams {
   float scale;
   int do_scale;
   FoldProgram prog;
-  uint32_t tile_prefix[kBucketMaxTensors + 1];
-  BucketTensorDesc t[kBucketMaxTensors];
-  const float* in[kBucketMaxPtrs];
-  float* out[kBucketMaxPtrs];
+  uint32_t tile_prefix[MAXT + 1];
+  BucketTensorDesc t[MAXT];
+  const float* in[MAXP];
+  float* out[MAXP];
 };
+using BucketParams = BucketParamsT<kBucketMaxTensors, kBucketMaxPtrs>;
+using BucketParamsSmall = BucketParamsT<8, 64>;
 static_assert(sizeof(BucketParams) <= 32000, "kernel parameter block too large");
+static_assert(sizeof(BucketParamsSmall) <= 4096, "small parameter block must stay under 4 KB");
 
-template <bool RING>
-__global__ void __launch_bounds__(kThreads, RING ? 3 : 2) bucket_allreduce_kernel(const __grid_constant__ BucketParams P) {
+template <bool RING, typename PT>
+__global__ void __launch_bounds__(kThreads, RING ? 3 : 2) bucket_allreduce_kernel(const __grid_constant__ PT P) {
   constexpr int IN = CC_F32, OP = CC_SUM;
   // the tile's per-rank pointers, staged once per tile: the fold reads them for every
   // 16-byte unit, and the parameter table is too large to stay in the constant cache
@@ -510,12 +517,14 @@ int bucket_group_limit(int nranks) {
   return std::max(1, std::min(kBucketMaxTensors, kBucketMaxPtrs / nranks));
 }
 
-cudaError_t launch_bucket_allreduce(const void* const* grads, void* const* out, int nranks, int ntensors_total,
-                                    const int32_t* ids, int nids, const BucketTensorDesc* desc, FoldKind fold,
-                                    float scale, cudaStream_t stream) {
-  static BucketParams P;  // large: keep it off the stack; calls are serialised by the caller's lock
-  static std::mutex mu;
-  std::lock_guard<std::mutex> lock(mu);
+int bucket_small_group_limit(int nranks) {
+  return std::max(1, std::min(BucketParamsSmall::kMaxT, BucketParamsSmall::kMaxP / nranks));
+}
+
+template <typename PT>
+static cudaError_t launch_bucket_with(PT& P, const void* const* grads, void* const* out, int nranks,
+                                      int ntensors_total, const int32_t* ids, int nids, const BucketTensorDesc* desc,
+                                      FoldKind fold, float scale, cudaStream_t stream) {
   P.nranks = nranks;
   P.ntensors = nids;
   P.fold = fold;
@@ -541,12 +550,25 @@ cudaError_t launch_bucket_allreduce(const void* const* grads, void* const* out, 
   if (fold == kFoldTree) tree_program(nranks, P.prog);
   if (tiles == 0) return cudaSuccess;
   const bool ring = fold == kFoldRing;
-  auto k = ring ? bucket_allreduce_kernel<true> : bucket_allreduce_kernel<false>;
-  static const int bps_ring = blocks_per_sm(bucket_allreduce_kernel<true>);
-  static const int bps_tree = blocks_per_sm(bucket_allreduce_kernel<false>);
+  auto k = ring ? bucket_allreduce_kernel<true, PT> : bucket_allreduce_kernel<false, PT>;
+  static const int bps_ring = blocks_per_sm(bucket_allreduce_kernel<true, PT>);
+  static const int bps_tree = blocks_per_sm(bucket_allreduce_kernel<false, PT>);
   const uint32_t grid = std::min<uint32_t>(tiles, (uint32_t)(2 * sm_count() * (ring ? bps_ring : bps_tree)));
   k<<<grid, kThreads, 0, stream>>>(P);
   return cudaGetLastError();
+}
+
+cudaError_t launch_bucket_allreduce(const void* const* grads, void* const* out, int nranks, int ntensors_total,
+                                    const int32_t* ids, int nids, const BucketTensorDesc* desc, FoldKind fold,
+                                    float scale, cudaStream_t stream) {
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  if (nids <= BucketParamsSmall::kMaxT && nids * nranks <= BucketParamsSmall::kMaxP) {
+    BucketParamsSmall P{};
+    return launch_bucket_with(P, grads, out, nranks, ntensors_total, ids, nids, desc, fold, scale, stream);
+  }
+  static BucketParams P;  // large: kept off the stack
+  return launch_bucket_with(P, grads, out, nranks, ntensors_total, ids, nids, desc, fold, scale, stream);
 }
 
 }  // namespace cc
