@@ -442,6 +442,11 @@ static cudaError_t run_reduce(ReduceParams& P, cudaStream_t s) {
   uint64_t upt = units / (resident * kThreads);
   upt = std::max<uint64_t>(1, std::min<uint64_t>(8, upt));
   P.tile = upt * kThreads * UE;
+  // a tile never spans much more than one fold group, so that the groups of a small
+  // buffer (N ring chunks of a few elements each) are folded by different CTAs in parallel
+  const uint64_t ngroups = P.fold == kFoldRing ? (uint64_t)P.nranks : (P.fold == kFoldTree ? 2 : 1);
+  const uint64_t per_group = ((P.count + ngroups - 1) / ngroups + 7) / 8 * 8;
+  P.tile = std::max<uint64_t>(8, std::min<uint64_t>(P.tile, per_group));
   const uint64_t ntiles = (P.count + P.tile - 1) / P.tile;
   const uint64_t grid = std::max<uint64_t>(1, std::min<uint64_t>(ntiles, 2 * resident));
   k<<<(unsigned)grid, kThreads, 0, s>>>(P);
