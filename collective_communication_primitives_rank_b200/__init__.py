@@ -36,6 +36,7 @@ _SIGS = {
     "cc_version": (_i, []),
     "cc_chunk": (_i, [_sz, _i, _i, _SZP, _SZP]),
     "cc_async_status": (_i, [_i, _vp]),
+    "cc_selftest_bounded_wait": (_i, [ctypes.c_uint, _vp]),
     "cc_allreduce": (_i, [_PP, _PP, _i, _sz, _i, _i, _i, _i, _f, _vp]),
     "cc_reduce_scatter": (_i, [_PP, _PP, _i, _sz, _i, _i, _i, _i, _f, _vp]),
     "cc_allgather": (_i, [_PP, _PP, _i, _sz, _i, _vp]),

@@ -256,6 +256,11 @@ cc_status cc_async_status(int reset, void* stream) {
   return v == CC_OK ? CC_OK : CC_ERR_TIMEOUT;
 }
 
+cc_status cc_selftest_bounded_wait(unsigned timeout_us, void* stream) {
+  if (timeout_us == 0 || timeout_us > 10000000u) return CC_ERR_INVALID_ARG;
+  return cuda_status(launch_bounded_wait_selftest((uint64_t)timeout_us * 1000ull, as_stream(stream)));
+}
+
 cc_status cc_chunk(size_t count, int nranks, int c, size_t* start, size_t* len) {
   if (!valid_ranks(nranks) || c < 0 || c >= nranks || !start || !len) return CC_ERR_INVALID_ARG;
   chunk_bounds(count, nranks, c, *start, *len);

@@ -45,6 +45,7 @@ cudaError_t launch_copy(const CopyEntry* entries, int nentries, void* const* dst
 // Device status word of the bounded waits (CC_OK or CC_ERR_TIMEOUT), read with a
 // stream synchronisation; `reset` clears it afterwards.
 cudaError_t read_async_status(int* out, bool reset, cudaStream_t stream);
+cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, cudaStream_t stream);
 
 // MoE
 cudaError_t launch_route_topk(const float* const* logits, int32_t* const* ids, int nranks, int tokens,

@@ -60,42 +60,54 @@ struct RouteParams {
   int tokens, experts, topk;
 };
 
-__device__ __forceinline__ bool better(float a, int ia, float b, int ib) {
-  return a > b || (a == b && ia < ib);
-}
-
-// One warp per token: topk rounds of a warp arg-max (larger value, then lower id).
+// One thread per token: the row's logits are scanned in expert order with a running,
+// descending top-k list in registers; a later expert enters only with a strictly larger
+// value, so equal values keep the lower expert id first.
 __global__ void __launch_bounds__(256) route_topk_kernel(const __grid_constant__ RouteParams P) {
-  const int lane = threadIdx.x & 31;
   const int s = blockIdx.y;
-  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= P.tokens) return;
   const float* row = P.logits[s] + (size_t)t * P.experts;
-  int chosen[kMaxTopk];
-  for (int j = 0; j < P.topk; ++j) {
-    float bv = 0.f;
-    int bi = -1;
-    for (int e = lane; e < P.experts; e += 32) {
-      bool taken = false;
-      for (int q = 0; q < j; ++q) taken |= (chosen[q] == e);
-      if (taken) continue;
-      const float v = __ldg(row + e);
-      if (bi < 0 || better(v, e, bv, bi)) { bv = v; bi = e; }
-    }
+  float val[kMaxTopk];
+  int idx[kMaxTopk];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-      if (oi >= 0 && (bi < 0 || better(ov, oi, bv, bi))) { bv = ov; bi = oi; }
+  for (int j = 0; j < kMaxTopk; ++j) { val[j] = -INFINITY; idx[j] = -1; }
+  auto insert = [&](float v, int e) {
+    if (idx[P.topk - 1] >= 0 && !(v > val[P.topk - 1])) return;
+    // shift down every entry v beats, then place v
+    bool placed = false;
+#pragma unroll
+    for (int j = kMaxTopk - 1; j >= 0; --j) {
+      if (j >= P.topk || placed) continue;
+      const bool beats = idx[j] < 0 || v > val[j];
+      if (beats && j > 0 && (idx[j - 1] < 0 || v > val[j - 1])) {
+        val[j] = val[j - 1];
+        idx[j] = idx[j - 1];
+      } else if (beats) {
+        val[j] = v;
+        idx[j] = e;
+        placed = true;
+      } else {
+        placed = true;
+      }
     }
-    chosen[j] = bi;
+  };
+  const bool vec = (P.experts % 4 == 0) && ((reinterpret_cast<uintptr_t>(P.logits[s]) & 15) == 0);
+  if (vec) {
+    for (int e = 0; e < P.experts; e += 4) {
+      const float4 v = __ldcs(reinterpret_cast<const float4*>(row + e));
+      insert(v.x, e);
+      insert(v.y, e + 1);
+      insert(v.z, e + 2);
+      insert(v.w, e + 3);
+    }
+  } else {
+    for (int e = 0; e < P.experts; ++e) insert(__ldcs(row + e), e);
   }
-  if (lane < P.topk) {
-    int v = chosen[0];
-    for (int q = 1; q < kMaxTopk; ++q)
-      if (q == lane) v = chosen[q];
-    P.ids[s][(size_t)t * P.topk + lane] = v;
-  }
+  int32_t* out = P.ids[s] + (size_t)t * P.topk;
+#pragma unroll
+  for (int j = 0; j < kMaxTopk; ++j)
+    if (j < P.topk) out[j] = idx[j];
 }
 
 cudaError_t launch_route_topk(const float* const* logits, int32_t* const* ids, int nranks, int tokens,
@@ -108,7 +120,7 @@ cudaError_t launch_route_topk(const float* const* logits, int32_t* const* ids, i
   P.tokens = tokens;
   P.experts = experts_total;
   P.topk = topk;
-  dim3 grid((tokens + 7) / 8, nranks);
+  dim3 grid((tokens + 255) / 256, nranks);
   route_topk_kernel<<<grid, 256, 0, stream>>>(P);
   return cudaGetLastError();
 }
@@ -226,20 +238,39 @@ __global__ void __launch_bounds__(256) a2a_copy_kernel(const __grid_constant__ A
     ok[k] = pos < P.capacity;
     ptr[k] = (P.direction == 0 ? P.recv[d] : const_cast<char*>(P.send[d])) + pos * P.row_bytes;
   }
+  // 8 loads per lane in flight before the stores that consume them
+  constexpr int B = 8;
   const uint64_t nvec = P.row_bytes / 16;
   if (P.direction == 0) {
-    const char* src = P.send[s] + (uint64_t)t * P.row_bytes;
-    for (uint64_t v = lane; v < nvec; v += 32) {
-      const uint4 x = __ldcs(reinterpret_cast<const uint4*>(src) + v);
-      for (int k = 0; k < P.topk; ++k)
-        if (ok[k]) __stcs(reinterpret_cast<uint4*>(ptr[k]) + v, x);
+    const uint4* src = reinterpret_cast<const uint4*>(P.send[s] + (uint64_t)t * P.row_bytes);
+    for (uint64_t v0 = lane; v0 < nvec; v0 += 32 * B) {
+      uint4 x[B];
+#pragma unroll
+      for (int b = 0; b < B; ++b)
+        if (v0 + 32 * b < nvec) x[b] = __ldcs(src + v0 + 32 * b);
+      for (int k = 0; k < P.topk; ++k) {
+        if (!ok[k]) continue;
+        uint4* d = reinterpret_cast<uint4*>(ptr[k]);
+#pragma unroll
+        for (int b = 0; b < B; ++b)
+          if (v0 + 32 * b < nvec) __stcs(d + v0 + 32 * b, x[b]);
+      }
     }
   } else {
     char* dst = P.recv[s] + (uint64_t)t * P.topk * P.row_bytes;
     for (int k = 0; k < P.topk; ++k) {
       if (!ok[k]) continue;
-      for (uint64_t v = lane; v < nvec; v += 32)
-        __stcs(reinterpret_cast<uint4*>(dst + k * P.row_bytes) + v, __ldcs(reinterpret_cast<const uint4*>(ptr[k]) + v));
+      const uint4* src = reinterpret_cast<const uint4*>(ptr[k]);
+      uint4* d = reinterpret_cast<uint4*>(dst + k * P.row_bytes);
+      for (uint64_t v0 = lane; v0 < nvec; v0 += 32 * B) {
+        uint4 x[B];
+#pragma unroll
+        for (int b = 0; b < B; ++b)
+          if (v0 + 32 * b < nvec) x[b] = __ldcs(src + v0 + 32 * b);
+#pragma unroll
+        for (int b = 0; b < B; ++b)
+          if (v0 + 32 * b < nvec) __stcs(d + v0 + 32 * b, x[b]);
+      }
     }
   }
 }

@@ -85,7 +85,8 @@ __device__ int g_async_status;  // CC_OK, or CC_ERR_TIMEOUT after a bounded wait
 
 constexpr int kBulkStages = 4;
 constexpr uint32_t kBulkTile = 32 * 1024;  // bytes; a multiple of 16
-constexpr long kWaitLimit = 1l << 26;      // try_wait polls before a wait gives up (seconds)
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // a wait gives up after 2 s (no load takes that long)
+constexpr long kWaitPolls = 1l << 30;             // and after this many polls, whatever the clock says
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -102,11 +103,32 @@ __device__ __forceinline__ bool mbar_test(uint64_t* m, uint32_t parity) {
       : "=r"(ok) : "r"(smem_addr(m)), "r"(parity) : "memory");
   return ok != 0;
 }
-__device__ __forceinline__ bool mbar_wait(uint64_t* m, uint32_t parity) {
-  for (long i = 0; i < kWaitLimit; ++i)
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait for the phase `parity` of an mbarrier; on giving up it records
+// CC_ERR_TIMEOUT in the device status word and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t* m, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
+  const uint64_t t0 = global_ns();
+  for (long i = 0; i < kWaitPolls; ++i) {
     if (mbar_test(m, parity)) return true;
+    if (global_ns() - t0 > limit_ns) break;
+  }
   atomicExch(&g_async_status, (int)CC_ERR_TIMEOUT);
   return false;
+}
+
+// Self-test of the bounded-wait path: one thread waits on an mbarrier that nothing will
+// ever arrive at, gives up after limit_ns and records CC_ERR_TIMEOUT. No fault, no trap:
+// the context stays usable.
+__global__ void bounded_wait_selftest_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bar)));
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  mbar_wait(&bar, 0, limit_ns);
 }
 __device__ __forceinline__ void bulk_load(void* smem, const void* gmem, uint32_t bytes, uint64_t* m) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
@@ -194,6 +216,11 @@ __global__ void __launch_bounds__(32) copy_bulk_kernel(const __grid_constant__ C
 }
 
 static bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, cudaStream_t stream) {
+  bounded_wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns);
+  return cudaGetLastError();
+}
 
 cudaError_t read_async_status(int* out, bool reset, cudaStream_t stream) {
   cudaError_t e = cudaMemcpyFromSymbolAsync(out, g_async_status, sizeof(int), 0, cudaMemcpyDeviceToHost, stream);

@@ -80,6 +80,12 @@ CC_API int cc_version(void);
  * device cannot be read. */
 CC_API cc_status cc_async_status(int reset, void* stream);
 
+/* Self-test of the device-side bounded waits: launches one thread that waits on a
+ * shared-memory barrier nothing will ever complete; after timeout_us (1 .. 10^7) it gives
+ * up and records CC_ERR_TIMEOUT in the status cc_async_status reads. Nothing faults or
+ * traps; the context stays usable. For tests of the failure path only. */
+CC_API cc_status cc_selftest_bounded_wait(unsigned timeout_us, void* stream);
+
 /* The chunk rule (host only): chunk c of a count-element buffer over nranks ranks
  * starts at *start and has *len elements (lecture 09 §7.1 splits the tensor into N equal
  * chunks; for a count N does not divide, the first count % N chunks get one more). */

@@ -216,3 +216,24 @@ def test_scatter_and_gather(n, count):
         out[r].check()
     _assert_same(to_host(back.t), x)
     back.check()
+
+
+# ---- failure detection on the device: a bounded wait that runs out reports, never hangs ----------
+
+def test_bounded_wait_timeout_is_reported_and_the_context_survives():
+    assert cc.cc_async_status(reset=True) in (cc.CC_OK, cc.CC_ERR_TIMEOUT)
+    assert cc.cc_async_status() == cc.CC_OK
+    st = cc.lib.cc_selftest_bounded_wait(20000, torch.cuda.current_stream().cuda_stream)  # 20 ms
+    assert st == cc.CC_OK
+    assert cc.cc_async_status() == cc.CC_ERR_TIMEOUT
+    assert cc.cc_async_status(reset=True) == cc.CC_ERR_TIMEOUT
+    assert cc.cc_async_status() == cc.CC_OK
+    # the context still runs collectives correctly
+    shards = [synth.uniform_f32(4, r, 1000) for r in range(4)]
+    out = [torch.empty(4000, device="cuda") for _ in range(4)]
+    cc.cc_allgather([to_dev(x) for x in shards], out)
+    want, _ = C.ring_allgather(shards)
+    torch.cuda.synchronize()
+    for r in range(4):
+        _assert_same(to_host(out[r]), want[r])
+    assert cc.cc_async_status() == cc.CC_OK
