@@ -260,6 +260,17 @@ def _prepared_allreduce(cc, x, y, algo, stream):
     return call
 
 
+def _prepared(cc, name, *args):
+    """A C entry point with its arguments marshalled once (timed spans hold only the call)."""
+    fn = getattr(cc.get_lib(), name)
+
+    def call():
+        st = fn(*args)
+        if st != cc.CC_OK:
+            raise RuntimeError(f"{name}: status {st}")
+    return call
+
+
 def _row_line(args, metric, value, unit, ms, config, roofline, launches, extra=None):
     peak, kind = measured_peak()
     line = {"metric": metric, "value": value, "unit": unit, "n_gpus": 1, "steps": args.steps,
@@ -288,17 +299,23 @@ def run_rows(args):
         shard = count // n
         rs = [torch.empty(shard, device="cuda") for _ in range(n)]
         ag = [torch.empty(count, device="cuda") for _ in range(n)]
+        st = torch.cuda.current_stream().cuda_stream
+        rs_call = _prepared(cc, "cc_reduce_scatter", cc._ptrs(x), cc._ptrs(rs), n, count, cc.CC_F32, cc.CC_F32,
+                            cc.CC_SUM, cc.CC_ALGO_RING, 1.0, st)
+        ag_call = _prepared(cc, "cc_allgather", cc._ptrs(rs), cc._ptrs(ag), n, count, cc.CC_F32, st)
         for _ in range(args.warmup):
-            cc.cc_reduce_scatter(x, rs)
-            cc.cc_allgather(rs, ag)
-        t_rs = _event_time_ms(torch, lambda: cc.cc_reduce_scatter(x, rs), iters) / iters
-        t_ag = _event_time_ms(torch, lambda: cc.cc_allgather(rs, ag), iters) / iters
-        del ag
+            rs_call()
+            ag_call()
+        t_rs = _event_time_ms(torch, rs_call, iters) / iters
+        t_ag = _event_time_ms(torch, ag_call, iters) / iters
+        del ag, ag_call
         xb = [t.to(torch.bfloat16) for t in x]
-        del x
+        del x, rs_call
+        bf_call = _prepared(cc, "cc_reduce_scatter", cc._ptrs(xb), cc._ptrs(rs), n, count, cc.CC_BF16, cc.CC_F32,
+                            cc.CC_SUM, cc.CC_ALGO_RING, 1.0, st)
         for _ in range(args.warmup):
-            cc.cc_reduce_scatter(xb, rs)
-        t_bf = _event_time_ms(torch, lambda: cc.cc_reduce_scatter(xb, rs), iters) / iters
+            bf_call()
+        t_bf = _event_time_ms(torch, bf_call, iters) / iters
         T = count * 4
         ms = t_rs + t_ag
         value = 2 * n * T / (ms * 1e-3) / 1e9
@@ -332,13 +349,20 @@ def run_rows(args):
         torch.cuda.synchronize()
         rows_recv = int(counts.sum().item())
         row = hidden * 2
+        st = torch.cuda.current_stream().cuda_stream
+        wsb = ws.numel() * 4
+        route = _prepared(cc, "cc_route_topk", cc._ptrs(logits), cc._ptrs(ids), n, tokens, E, topk, st)
+        disp = _prepared(cc, "cc_alltoallv", cc._ptrs(toks), cc._ptrs(recv), n, row, cc._ptrs(ids), tokens, topk, epr,
+                         cap, 0, ws.data_ptr(), wsb, st)
+        comb = _prepared(cc, "cc_alltoallv", cc._ptrs(recv), cc._ptrs(back), n, row, cc._ptrs(ids), tokens, topk, epr,
+                         cap, 1, ws.data_ptr(), wsb, st)
         for _ in range(args.warmup):
-            cc.cc_route_topk(logits, ids)
-            cc.cc_alltoallv(toks, recv, ids, epr, ws, direction=0)
-            cc.cc_alltoallv(recv, back, ids, epr, ws, direction=1)
-        t_route = _event_time_ms(torch, lambda: cc.cc_route_topk(logits, ids), iters) / iters
-        t_d = _event_time_ms(torch, lambda: cc.cc_alltoallv(toks, recv, ids, epr, ws, direction=0), iters) / iters
-        t_c = _event_time_ms(torch, lambda: cc.cc_alltoallv(recv, back, ids, epr, ws, direction=1), iters) / iters
+            route()
+            disp()
+            comb()
+        t_route = _event_time_ms(torch, route, iters) / iters
+        t_d = _event_time_ms(torch, disp, iters) / iters
+        t_c = _event_time_ms(torch, comb, iters) / iters
         b_d = n * tokens * row + rows_recv * row
         b_c = 2 * rows_recv * row
         ms = t_route + t_d + t_c
@@ -355,6 +379,7 @@ def run_rows(args):
         return 0
     # config 5: ring vs double-binary-tree allreduce, N in {2..64}, 1 KiB .. 256 MiB per rank
     flush_buf = torch.empty(256 * 1024 * 1024 // 4, device="cuda")
+    ws = torch.zeros(64, dtype=torch.int32, device="cuda")
     table = []
     best = None
     for n in (2, 4, 8, 16, 32, 64):
@@ -376,20 +401,32 @@ def run_rows(args):
                 ms = _event_time_ms(torch, call, reps, flush) / reps
                 row[algo + "_us"] = ms * 1e3
                 row[algo + "_GBps"] = 2 * n * size / (ms * 1e-3) / 1e9
+                # the same result by the schedule's dependent steps (grid barrier per step)
+                stepped = _prepared(cc, "cc_allreduce_stepped", cc._ptrs(x), cc._ptrs(y), n, count, cc.CC_F32,
+                                    cc.CC_F32, cc.CC_SUM, cc.CC_ALGO_RING if algo == "ring" else cc.CC_ALGO_TREE,
+                                    1.0, ws.data_ptr(), ws.numel() * 4, torch.cuda.current_stream().cuda_stream)
+                for _ in range(2):
+                    stepped()
+                sreps = max(2, reps // 4)
+                ms = _event_time_ms(torch, stepped, sreps, flush) / sreps
+                row[algo + "_stepped_us"] = ms * 1e3
+                row[algo + "_stepped_GBps"] = 2 * n * size / (ms * 1e-3) / 1e9
             if n == 8:
-                src = x[0]
-                ms = _event_time_ms(torch, lambda: cc.cc_broadcast(src, y, 0), reps, flush) / reps
+                bc = _prepared(cc, "cc_broadcast", x[0].data_ptr(), cc._ptrs(y), n, 0, count, cc.CC_F32,
+                               torch.cuda.current_stream().cuda_stream)
+                ms = _event_time_ms(torch, bc, reps, flush) / reps
                 row["broadcast_GBps"] = (n + 1) * size / (ms * 1e-3) / 1e9
             table.append(row)
             if n == 8 and size == 256 * 1024 * 1024:
                 best = row
             del x, y
-    cross = {}
+    cross, cross_stepped = {}, {}
     for n in (2, 4, 8, 16, 32, 64):
         pts = [r for r in table if r["n"] == n]
-        over = [r["bytes_per_rank"] for r in pts if r["ring_GBps"] > 1.03 * r["tree_GBps"]]
-        under = [r["bytes_per_rank"] for r in pts if r["tree_GBps"] > 1.03 * r["ring_GBps"]]
-        cross[str(n)] = {"ring_faster_by_3pct_at": over, "tree_faster_by_3pct_at": under}
+        for key, dst in (("", cross), ("_stepped", cross_stepped)):
+            over = [r["bytes_per_rank"] for r in pts if r["ring" + key + "_GBps"] > 1.03 * r["tree" + key + "_GBps"]]
+            under = [r["bytes_per_rank"] for r in pts if r["tree" + key + "_GBps"] > 1.03 * r["ring" + key + "_GBps"]]
+            dst[str(n)] = {"ring_faster_by_3pct_at": over, "tree_faster_by_3pct_at": under}
     lat = min(r["ring_us"] for r in table)
     _row_line(args, METRIC, best["ring_GBps"], "GB/s", best["ring_us"] / 1e3,
               {"workload": "sweep: ring vs double-binary-tree allreduce, N in {2,4,8,16,32,64}, fp32 U[-1,1] "
@@ -397,7 +434,7 @@ def run_rows(args):
                "l2": "L2 flushed (256 MiB write) before every timed call whose working set fits in L2"},
               {"achieved": best["ring_GBps"], "kernel": "reduce_kernel<f32,sum,ring>"},
               len(table) * 2,
-              {"sweep": table, "crossover": cross, "min_launch_latency_us": lat})
+              {"sweep": table, "crossover": cross, "crossover_stepped": cross_stepped, "min_launch_latency_us": lat})
     return 0
 
 

@@ -39,6 +39,7 @@ _SIGS = {
     "cc_selftest_bounded_wait": (_i, [ctypes.c_uint, _vp]),
     "cc_allreduce": (_i, [_PP, _PP, _i, _sz, _i, _i, _i, _i, _f, _vp]),
     "cc_reduce_scatter": (_i, [_PP, _PP, _i, _sz, _i, _i, _i, _i, _f, _vp]),
+    "cc_allreduce_stepped": (_i, [_PP, _PP, _i, _sz, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
     "cc_allgather": (_i, [_PP, _PP, _i, _sz, _i, _vp]),
     "cc_broadcast": (_i, [_vp, _PP, _i, _i, _sz, _i, _vp]),
     "cc_reduce": (_i, [_PP, _vp, _i, _i, _sz, _i, _i, _i, _f, _vp]),
@@ -173,6 +174,20 @@ def cc_allreduce(send, recv, *, op="sum", algo="ring", scale=1.0, stream=None) -
     _check(lib.cc_allreduce(_ptrs(send), _ptrs(recv), n, send[0].numel(), dtype_code(send[0]),
                             dtype_code(recv[0]), _OPS[op], _ALGOS[algo], float(scale), _stream(stream)),
            "cc_allreduce")
+
+
+def cc_allreduce_stepped(send, recv, workspace, *, op="sum", algo="ring", scale=1.0, stream=None) -> None:
+    """cc_allreduce's result, computed by executing the schedule step by step (grid barrier
+    between steps). `workspace`: a CUDA tensor of at least 256 bytes."""
+    n = _ranks(send, "cc_allreduce_stepped")
+    _same(send, send[0].numel(), send[0].dtype, "cc_allreduce_stepped send")
+    _same(recv, send[0].numel(), recv[0].dtype, "cc_allreduce_stepped recv")
+    if len(recv) != n:
+        raise ValueError("cc_allreduce_stepped: one output per rank")
+    _check(lib.cc_allreduce_stepped(_ptrs(send), _ptrs(recv), n, send[0].numel(), dtype_code(send[0]),
+                                    dtype_code(recv[0]), _OPS[op], _ALGOS[algo], float(scale), _dev_ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream)),
+           "cc_allreduce_stepped")
 
 
 def cc_reduce_scatter(send, recv, *, op="sum", algo="ring", scale=1.0, stream=None) -> None:

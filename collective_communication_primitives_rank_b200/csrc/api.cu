@@ -281,6 +281,22 @@ cc_status cc_allreduce(const void* const* send, void* const* recv, int nranks, s
                                    as_stream(stream)));
 }
 
+cc_status cc_allreduce_stepped(const void* const* send, void* const* recv, int nranks, size_t count, cc_dtype in_t,
+                               cc_dtype out_t, cc_op op, cc_algo algo, float scale, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  if (!valid_ranks(nranks) || !send || !recv) return CC_ERR_INVALID_ARG;
+  if (cc_status st = check_reduce(in_t, out_t, op, scale)) return st;
+  if (algo != CC_ALGO_RING && algo != CC_ALGO_TREE) return CC_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < 256 || (reinterpret_cast<uintptr_t>(workspace) & 255)) return CC_ERR_INVALID_ARG;
+  if (count == 0) return CC_OK;
+  if (!all_nonnull(send, nranks) || !all_nonnull((const void* const*)recv, nranks)) return CC_ERR_INVALID_ARG;
+  for (int r = 0; r < nranks; ++r)
+    if (recv[r] == send[r] && dtype_bytes(in_t) != dtype_bytes(out_t)) return CC_ERR_INVALID_ARG;
+  return cuda_status(launch_stepped_allreduce(send, recv, nranks, count, in_t, op,
+                                              algo == CC_ALGO_RING ? kFoldRing : kFoldTree, scale,
+                                              static_cast<unsigned*>(workspace), as_stream(stream)));
+}
+
 cc_status cc_reduce_scatter(const void* const* send, void* const* recv, int nranks, size_t count, cc_dtype in_t,
                             cc_dtype out_t, cc_op op, cc_algo algo, float scale, void* stream) {
   if (!valid_ranks(nranks) || !send || !recv) return CC_ERR_INVALID_ARG;

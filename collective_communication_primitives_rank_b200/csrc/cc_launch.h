@@ -46,6 +46,13 @@ cudaError_t launch_copy(const CopyEntry* entries, int nentries, void* const* dst
 // stream synchronisation; `reset` clears it afterwards.
 cudaError_t read_async_status(int* out, bool reset, cudaStream_t stream);
 cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, cudaStream_t stream);
+int* async_status_word();  // device address of that status word (current device), or null
+
+// Stepped (schedule-faithful) allreduce: one cooperative launch, a grid barrier between the
+// schedule's dependent steps; `barrier` is 4 bytes of caller device memory.
+cudaError_t launch_stepped_allreduce(const void* const* send, void* const* recv, int nranks, size_t count,
+                                     cc_dtype in_t, cc_op op, FoldKind fold, float scale, unsigned* barrier,
+                                     cudaStream_t s);
 
 // MoE
 cudaError_t launch_route_topk(const float* const* logits, int32_t* const* ids, int nranks, int tokens,

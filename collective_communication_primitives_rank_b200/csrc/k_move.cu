@@ -15,6 +15,7 @@
 // copy_kernel (any alignment): 128-bit streaming loads/stores per thread where an entry is
 // 16-byte aligned, element by element otherwise.
 #include <algorithm>
+#include <mutex>
 
 #include "cc_device.cuh"
 #include "cc_launch.h"
@@ -216,6 +217,18 @@ __global__ void __launch_bounds__(32) copy_bulk_kernel(const __grid_constant__ C
 }
 
 static bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int* async_status_word() {
+  static int* ptr[64];
+  static std::once_flag once[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::call_once(once[dev], [dev] {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_async_status) == cudaSuccess) ptr[dev] = static_cast<int*>(p);
+  });
+  return ptr[dev];
+}
 
 cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, cudaStream_t stream) {
   bounded_wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns);

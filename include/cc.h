@@ -102,6 +102,23 @@ CC_API cc_status cc_allreduce(const void* const* send, void* const* recv, int nr
                        cc_dtype in_t, cc_dtype out_t, cc_op op, cc_algo algo, float scale,
                        void* stream);
 
+/* Stepped AllReduce: the same result as cc_allreduce, bit for bit, obtained by executing the
+ * schedule's dependent steps one after another on the output buffers (ring: N-1
+ * reduce-scatter steps then N-1 allgather steps, lecture 09 §4.3 and experiment 1 §7.1;
+ * tree: the double binary tree reduced up one level per step and broadcast down one level
+ * per step, lecture 09 §5.2, multi-node page §4.3.2). One cooperative launch with a grid
+ * barrier between steps, so its time shows the schedule's latency (2(N-1) steps for the
+ * ring against about 2 log2 N for the tree) next to its bandwidth.
+ *   workspace: at least 256 bytes of device memory, 256-byte aligned, used for the grid
+ *   barrier (cleared by the call, stream-ordered); calls that overlap on the GPU need
+ *   separate workspaces.
+ *   A barrier that does not complete within 2 s makes the kernel stop and record
+ *   CC_ERR_TIMEOUT (see cc_async_status); outputs are then incomplete.
+ * Other arguments, layouts and errors as cc_allreduce. */
+CC_API cc_status cc_allreduce_stepped(const void* const* send, void* const* recv, int nranks, size_t count,
+                                      cc_dtype in_t, cc_dtype out_t, cc_op op, cc_algo algo, float scale,
+                                      void* workspace, size_t workspace_bytes, void* stream);
+
 /* ReduceScatter (lecture 09 §3.6; the from-scratch page's reduce_scatter as the first
  * half of the ring). Rank c receives, in recv[c], chunk c (chunk rule) of the ring
  * reduction: q + (c < r) elements of out_t. `count` is the per-rank INPUT length.

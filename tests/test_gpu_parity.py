@@ -237,3 +237,39 @@ def test_bounded_wait_timeout_is_reported_and_the_context_survives():
     for r in range(4):
         _assert_same(to_host(out[r]), want[r])
     assert cc.cc_async_status() == cc.CC_OK
+
+
+# ---- stepped (schedule-faithful) allreduce: the same bits as the fused kernels -------------------------
+
+@pytest.mark.parametrize("n,count", [(1, 37), (2, 4096), (3, 1001), (4, 4096), (5, 777), (8, 8 * 4096), (8, 999),
+                                     (13, 2000), (16, 65536), (64, 64 * 40), (64, 70)])
+@pytest.mark.parametrize("algo", ["ring", "tree"])
+@pytest.mark.parametrize("kind", ["spread", "i32", "bf16"])
+def test_stepped_allreduce_matches_oracle(n, count, algo, kind):
+    xs = _inputs(kind, n, count, seed=15)
+    scale = 1.0 if kind == "i32" else 1.0 / n
+    fn = C.ring_allreduce if algo == "ring" else C.tree_allreduce
+    want, _ = fn(xs, in_dtype=_IN[kind], scale=scale)
+    ws = torch.zeros(64, dtype=torch.int32, device="cuda")
+    out = [Guarded(count, _out_dtype(kind)) for _ in range(n)]
+    cc.cc_allreduce_stepped([to_dev(x) for x in xs], [o.t for o in out], ws, algo=algo, scale=scale)
+    torch.cuda.synchronize()
+    assert cc.cc_async_status() == cc.CC_OK
+    for r in range(n):
+        _assert_same(to_host(out[r].t), want[r], f"stepped {algo} {kind} N={n} rank {r}")
+        out[r].check()
+
+
+@pytest.mark.parametrize("op", ["max", "prod"])
+def test_stepped_in_place_other_ops(op):
+    n, count = 6, 4096
+    xs = [(1.0 + 0.01 * x).astype(np.float32) for x in _inputs("f32", n, count, seed=16)]
+    for algo in ("ring", "tree"):
+        fn = C.ring_allreduce if algo == "ring" else C.tree_allreduce
+        want, _ = fn(xs, op=op)
+        buf = [to_dev(x) for x in xs]
+        ws = torch.zeros(64, dtype=torch.int32, device="cuda")
+        cc.cc_allreduce_stepped(buf, buf, ws, op=op, algo=algo)
+        torch.cuda.synchronize()
+        for r in range(n):
+            _assert_same(to_host(buf[r]), want[r], f"stepped in place {op} {algo} rank {r}")
