@@ -40,6 +40,23 @@ PROFILE = os.path.join(ROOT, "profiles", "bucket_allreduce_ddp.txt")
 KERNEL_SRC = os.path.join(ROOT, "collective_communication_primitives_rank_b200", "csrc", "k_reduce.cu")
 
 
+def replica_seed(rank):
+    """Each GPU of a multi-GPU run holds its own replica of the workload (independent problem)."""
+    return SEED + 1000 * rank
+
+
+def max_over_ranks(dist, torch, value, device):
+    """The slowest rank's time (one float through the process group; not on the data path)."""
+    t = torch.tensor([float(value)], device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_gbps(world, bytes_per_step, ms_per_step):
+    """Whole-job throughput: every rank moves bytes_per_step in the (max-over-ranks) step time."""
+    return world * bytes_per_step / (ms_per_step * 1e-3) / 1e9
+
+
 def workload_desc(layers):
     return (f"ddp_bucket_allreduce: N={N_SIM} simulated ranks on one GPU, fp32 gradients of a "
             f"{layers}-layer d=768 ffn=3072 vocab=32000 transformer, 25 MiB buckets in reverse "
@@ -468,7 +485,7 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
 
-    w = build_workload(torch, args.layers, SEED + 1000 * rank, pinned_inputs=True)
+    w = build_workload(torch, args.layers, replica_seed(rank), pinned_inputs=True)
     bytes_step = 2 * N_SIM * w["total"] * 4
     stream = torch.cuda.current_stream()
 
@@ -498,11 +515,9 @@ def main():
         barrier()
     ms = start.elapsed_time(end)
     if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(dist, torch, ms, "cuda")
     ms_step = ms / args.steps
-    value = world * bytes_step / (ms_step * 1e-3) / 1e9
+    value = aggregate_gbps(world, bytes_step, ms_step)
 
     # end to end through the host-buffer entry point: H2D + fused allreduce + D2H per step
     host_out = [torch.empty(w["total"], dtype=torch.float32, pin_memory=True) for _ in range(N_SIM)]
@@ -524,10 +539,8 @@ def main():
     barrier()
     ems = s2.elapsed_time(e2)
     if world > 1:
-        t = torch.tensor([ems], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ems = float(t.item())
-    e2e_value = world * bytes_step / (ems / args.e2e_steps * 1e-3) / 1e9
+        ems = max_over_ranks(dist, torch, ems, "cuda")
+    e2e_value = aggregate_gbps(world, bytes_step, ems / args.e2e_steps)
 
     peak, peak_kind = measured_peak()
     achieved = bytes_step / launches_per_step / (ms_step / launches_per_step * 1e-3) / 1e9
