@@ -60,54 +60,94 @@ struct RouteParams {
   int tokens, experts, topk;
 };
 
-// One thread per token: the row's logits are scanned in expert order with a running,
-// descending top-k list in registers; a later expert enters only with a strictly larger
-// value, so equal values keep the lower expert id first.
+// Eight lanes per token. Lane g of a token's group scans the 4-expert chunks g, g+8, ... in
+// expert order with a running, descending top-k list in registers (a later expert enters
+// only with a strictly larger value, so equal values keep the lower id first); the eight
+// lists are then merged pairwise with shuffles (three butterfly steps), ordering by larger
+// value, then lower id. All lanes end with the token's top-k; lane 0 writes it.
+constexpr int kRouteLanes = 8;
+
+__device__ __forceinline__ bool route_better(float a, int ia, float b, int ib) {
+  return ib < 0 || (ia >= 0 && (a > b || (a == b && ia < ib)));
+}
+
 __global__ void __launch_bounds__(256) route_topk_kernel(const __grid_constant__ RouteParams P) {
   const int s = blockIdx.y;
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= P.tokens) return;
-  const float* row = P.logits[s] + (size_t)t * P.experts;
+  const int lane = threadIdx.x & 31;
+  const int g = lane % kRouteLanes;
+  const int t = (blockIdx.x * blockDim.x + threadIdx.x) / kRouteLanes;
+  const bool live = t < P.tokens;  // dead groups still take part in the shuffles
+  const int K = P.topk;
   float val[kMaxTopk];
   int idx[kMaxTopk];
 #pragma unroll
   for (int j = 0; j < kMaxTopk; ++j) { val[j] = -INFINITY; idx[j] = -1; }
   auto insert = [&](float v, int e) {
-    if (idx[P.topk - 1] >= 0 && !(v > val[P.topk - 1])) return;
-    // shift down every entry v beats, then place v
-    bool placed = false;
+    if (idx[K - 1] >= 0 && !(v > val[K - 1])) return;
+    int pos = K - 1;
 #pragma unroll
-    for (int j = kMaxTopk - 1; j >= 0; --j) {
-      if (j >= P.topk || placed) continue;
-      const bool beats = idx[j] < 0 || v > val[j];
-      if (beats && j > 0 && (idx[j - 1] < 0 || v > val[j - 1])) {
+    for (int j = kMaxTopk - 1; j >= 1; --j)
+      if (j <= K - 1 && pos == j && (idx[j - 1] < 0 || v > val[j - 1])) {
         val[j] = val[j - 1];
         idx[j] = idx[j - 1];
-      } else if (beats) {
-        val[j] = v;
-        idx[j] = e;
-        placed = true;
-      } else {
-        placed = true;
+        pos = j - 1;
       }
-    }
-  };
-  const bool vec = (P.experts % 4 == 0) && ((reinterpret_cast<uintptr_t>(P.logits[s]) & 15) == 0);
-  if (vec) {
-    for (int e = 0; e < P.experts; e += 4) {
-      const float4 v = __ldcs(reinterpret_cast<const float4*>(row + e));
-      insert(v.x, e);
-      insert(v.y, e + 1);
-      insert(v.z, e + 2);
-      insert(v.w, e + 3);
-    }
-  } else {
-    for (int e = 0; e < P.experts; ++e) insert(__ldcs(row + e), e);
-  }
-  int32_t* out = P.ids[s] + (size_t)t * P.topk;
 #pragma unroll
-  for (int j = 0; j < kMaxTopk; ++j)
-    if (j < P.topk) out[j] = idx[j];
+    for (int j = 0; j < kMaxTopk; ++j)
+      if (j == pos) { val[j] = v; idx[j] = e; }
+  };
+  if (live) {
+    const float* row = P.logits[s] + (size_t)t * P.experts;
+    const bool vec = (P.experts % 4 == 0) && ((reinterpret_cast<uintptr_t>(P.logits[s]) & 15) == 0);
+    if (vec) {
+      for (int e = 4 * g; e < P.experts; e += 4 * kRouteLanes) {
+        const float4 v = __ldcs(reinterpret_cast<const float4*>(row + e));
+        insert(v.x, e);
+        insert(v.y, e + 1);
+        insert(v.z, e + 2);
+        insert(v.w, e + 3);
+      }
+    } else {
+      for (int e = g; e < P.experts; e += kRouteLanes) insert(__ldcs(row + e), e);
+    }
+  }
+#pragma unroll
+  for (int off = kRouteLanes / 2; off >= 1; off >>= 1) {
+    float ov[kMaxTopk];
+    int oi[kMaxTopk];
+#pragma unroll
+    for (int j = 0; j < kMaxTopk; ++j) {
+      ov[j] = __shfl_xor_sync(0xffffffffu, val[j], off);
+      oi[j] = __shfl_xor_sync(0xffffffffu, idx[j], off);
+    }
+    // merge the two descending lists, keep the first K
+    float mv[kMaxTopk];
+    int mi[kMaxTopk];
+    int a = 0, b = 0;
+#pragma unroll
+    for (int j = 0; j < kMaxTopk; ++j) {
+      float va = -INFINITY, vb = -INFINITY;
+      int ia = -1, ib = -1;
+#pragma unroll
+      for (int x = 0; x < kMaxTopk; ++x) {
+        if (x == a) { va = val[x]; ia = idx[x]; }
+        if (x == b) { vb = ov[x]; ib = oi[x]; }
+      }
+      if (route_better(va, ia, vb, ib)) { mv[j] = va; mi[j] = ia; ++a; }
+      else { mv[j] = vb; mi[j] = ib; ++b; }
+    }
+#pragma unroll
+    for (int j = 0; j < kMaxTopk; ++j) {
+      val[j] = mv[j];
+      idx[j] = j < K ? mi[j] : -1;
+    }
+  }
+  if (live && g == 0) {
+    int32_t* out = P.ids[s] + (size_t)t * K;
+#pragma unroll
+    for (int j = 0; j < kMaxTopk; ++j)
+      if (j < K) out[j] = idx[j];
+  }
 }
 
 cudaError_t launch_route_topk(const float* const* logits, int32_t* const* ids, int nranks, int tokens,
@@ -120,7 +160,8 @@ cudaError_t launch_route_topk(const float* const* logits, int32_t* const* ids, i
   P.tokens = tokens;
   P.experts = experts_total;
   P.topk = topk;
-  dim3 grid((tokens + 255) / 256, nranks);
+  const long long threads = (long long)tokens * kRouteLanes;
+  dim3 grid((unsigned)((threads + 255) / 256), nranks);
   route_topk_kernel<<<grid, 256, 0, stream>>>(P);
   return cudaGetLastError();
 }
