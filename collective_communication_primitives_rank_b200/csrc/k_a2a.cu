@@ -71,29 +71,29 @@ __device__ __forceinline__ bool route_better(float a, int ia, float b, int ib) {
   return ib < 0 || (ia >= 0 && (a > b || (a == b && ia < ib)));
 }
 
+template <int K>
 __global__ void __launch_bounds__(256) route_topk_kernel(const __grid_constant__ RouteParams P) {
   const int s = blockIdx.y;
   const int lane = threadIdx.x & 31;
   const int g = lane % kRouteLanes;
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) / kRouteLanes;
   const bool live = t < P.tokens;  // dead groups still take part in the shuffles
-  const int K = P.topk;
-  float val[kMaxTopk];
-  int idx[kMaxTopk];
+  float val[K];
+  int idx[K];
 #pragma unroll
-  for (int j = 0; j < kMaxTopk; ++j) { val[j] = -INFINITY; idx[j] = -1; }
+  for (int j = 0; j < K; ++j) { val[j] = -INFINITY; idx[j] = -1; }
   auto insert = [&](float v, int e) {
     if (idx[K - 1] >= 0 && !(v > val[K - 1])) return;
     int pos = K - 1;
 #pragma unroll
-    for (int j = kMaxTopk - 1; j >= 1; --j)
-      if (j <= K - 1 && pos == j && (idx[j - 1] < 0 || v > val[j - 1])) {
+    for (int j = K - 1; j >= 1; --j)
+      if (pos == j && (idx[j - 1] < 0 || v > val[j - 1])) {
         val[j] = val[j - 1];
         idx[j] = idx[j - 1];
         pos = j - 1;
       }
 #pragma unroll
-    for (int j = 0; j < kMaxTopk; ++j)
+    for (int j = 0; j < K; ++j)
       if (j == pos) { val[j] = v; idx[j] = e; }
   };
   if (live) {
@@ -113,23 +113,23 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const __grid_constant__
   }
 #pragma unroll
   for (int off = kRouteLanes / 2; off >= 1; off >>= 1) {
-    float ov[kMaxTopk];
-    int oi[kMaxTopk];
+    float ov[K];
+    int oi[K];
 #pragma unroll
-    for (int j = 0; j < kMaxTopk; ++j) {
+    for (int j = 0; j < K; ++j) {
       ov[j] = __shfl_xor_sync(0xffffffffu, val[j], off);
       oi[j] = __shfl_xor_sync(0xffffffffu, idx[j], off);
     }
     // merge the two descending lists, keep the first K
-    float mv[kMaxTopk];
-    int mi[kMaxTopk];
+    float mv[K];
+    int mi[K];
     int a = 0, b = 0;
 #pragma unroll
-    for (int j = 0; j < kMaxTopk; ++j) {
+    for (int j = 0; j < K; ++j) {
       float va = -INFINITY, vb = -INFINITY;
       int ia = -1, ib = -1;
 #pragma unroll
-      for (int x = 0; x < kMaxTopk; ++x) {
+      for (int x = 0; x < K; ++x) {
         if (x == a) { va = val[x]; ia = idx[x]; }
         if (x == b) { vb = ov[x]; ib = oi[x]; }
       }
@@ -137,16 +137,12 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const __grid_constant__
       else { mv[j] = vb; mi[j] = ib; ++b; }
     }
 #pragma unroll
-    for (int j = 0; j < kMaxTopk; ++j) {
-      val[j] = mv[j];
-      idx[j] = j < K ? mi[j] : -1;
-    }
+    for (int j = 0; j < K; ++j) { val[j] = mv[j]; idx[j] = mi[j]; }
   }
   if (live && g == 0) {
     int32_t* out = P.ids[s] + (size_t)t * K;
 #pragma unroll
-    for (int j = 0; j < kMaxTopk; ++j)
-      if (j < K) out[j] = idx[j];
+    for (int j = 0; j < K; ++j) out[j] = idx[j];
   }
 }
 
@@ -162,7 +158,16 @@ cudaError_t launch_route_topk(const float* const* logits, int32_t* const* ids, i
   P.topk = topk;
   const long long threads = (long long)tokens * kRouteLanes;
   dim3 grid((unsigned)((threads + 255) / 256), nranks);
-  route_topk_kernel<<<grid, 256, 0, stream>>>(P);
+  switch (topk) {
+    case 1: route_topk_kernel<1><<<grid, 256, 0, stream>>>(P); break;
+    case 2: route_topk_kernel<2><<<grid, 256, 0, stream>>>(P); break;
+    case 3: route_topk_kernel<3><<<grid, 256, 0, stream>>>(P); break;
+    case 4: route_topk_kernel<4><<<grid, 256, 0, stream>>>(P); break;
+    case 5: route_topk_kernel<5><<<grid, 256, 0, stream>>>(P); break;
+    case 6: route_topk_kernel<6><<<grid, 256, 0, stream>>>(P); break;
+    case 7: route_topk_kernel<7><<<grid, 256, 0, stream>>>(P); break;
+    default: route_topk_kernel<8><<<grid, 256, 0, stream>>>(P); break;
+  }
   return cudaGetLastError();
 }
 
