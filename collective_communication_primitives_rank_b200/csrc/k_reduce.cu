@@ -23,6 +23,13 @@
 namespace cc {
 
 constexpr int kThreads = 256;
+// Grids are sized to one CTA per tile (capped at this many times the resident CTAs): with
+// the hardware handing tiles to CTAs as earlier ones finish, DRAM stayed busier than with
+// persistent CTAs looping over tiles (measured: 2x -> 93%, 8x -> 99.5%, one tile per CTA
+// -> 101% of the copy rate on the DDP step).
+#ifndef CC_REDUCE_OVERSUB
+#define CC_REDUCE_OVERSUB 1024
+#endif
 #ifndef CC_RING_MIN_BLOCKS
 #define CC_RING_MIN_BLOCKS 4  // resident 256-thread CTAs per SM the ring kernel is compiled for
 #endif
@@ -184,9 +191,9 @@ struct ReduceParams {
   int do_scale;
 };
 
-// Persistent CTAs take contiguous tiles round-robin (the grid is oversubscribed twice over
-// the resident CTAs, which measured faster than one wave); a tile is split where it crosses
-// a fold group (ring chunk or tree half) and each piece is folded by the whole CTA.
+// Each CTA folds contiguous tiles (normally exactly one: the grid is sized to the tile
+// count); a tile is split where it crosses a fold group (ring chunk or tree half) and each
+// piece is folded by the whole CTA.
 template <int IN, int OP, bool RING, int U>
 __global__ void __launch_bounds__(kThreads, (RING && U == 1) ? CC_RING_MIN_BLOCKS : 2) reduce_kernel(const __grid_constant__ ReduceParams P) {
   using In = typename Tr<IN>::In;
@@ -241,9 +248,18 @@ __global__ void __launch_bounds__(kThreads, (RING && U == 1) ? CC_RING_MIN_BLOCK
 // Every element is folded exactly as in flatten -> allreduce -> unflatten, with no flat
 // buffer: N·G bytes in, N·G bytes out.
 
+#ifndef CC_BUCKET_TILE
+#define CC_BUCKET_TILE 8192        // elements per tile
+#endif
+#ifndef CC_BUCKET_MIN_BLOCKS
+#define CC_BUCKET_MIN_BLOCKS 3     // resident 256-thread CTAs per SM the ring variant is compiled for
+#endif
+#ifndef CC_BUCKET_OVERSUB
+#define CC_BUCKET_OVERSUB 1024     // grid = tiles, capped at this many times the resident CTAs
+#endif
 constexpr int kBucketMaxTensors = 192;
 constexpr int kBucketMaxPtrs = 1536;
-constexpr uint64_t kBucketTile = 8192;
+constexpr uint64_t kBucketTile = CC_BUCKET_TILE;
 
 // Tables travel as kernel parameters: a large block (up to 192 tensors, 30 KB) for whole
 // tensor lists, and a small one (under 4 KB) for the short lists of the host-buffer
@@ -268,7 +284,7 @@ static_assert(sizeof(BucketParams) <= 32000, "kernel parameter block too large")
 static_assert(sizeof(BucketParamsSmall) <= 4096, "small parameter block must stay under 4 KB");
 
 template <bool RING, typename PT>
-__global__ void __launch_bounds__(kThreads, RING ? 3 : 2) bucket_allreduce_kernel(const __grid_constant__ PT P) {
+__global__ void __launch_bounds__(kThreads, RING ? CC_BUCKET_MIN_BLOCKS : 2) bucket_allreduce_kernel(const __grid_constant__ PT P) {
   constexpr int IN = CC_F32, OP = CC_SUM;
   // the tile's per-rank pointers, staged once per tile: the fold reads them for every
   // 16-byte unit, and the parameter table is too large to stay in the constant cache
@@ -448,7 +464,7 @@ static cudaError_t run_reduce(ReduceParams& P, cudaStream_t s) {
   const uint64_t per_group = ((P.count + ngroups - 1) / ngroups + 7) / 8 * 8;
   P.tile = std::max<uint64_t>(8, std::min<uint64_t>(P.tile, per_group));
   const uint64_t ntiles = (P.count + P.tile - 1) / P.tile;
-  const uint64_t grid = std::max<uint64_t>(1, std::min<uint64_t>(ntiles, 2 * resident));
+  const uint64_t grid = std::max<uint64_t>(1, std::min<uint64_t>(ntiles, CC_REDUCE_OVERSUB * resident));
   k<<<(unsigned)grid, kThreads, 0, s>>>(P);
   return cudaGetLastError();
 }
@@ -558,7 +574,8 @@ static cudaError_t launch_bucket_with(PT& P, const void* const* grads, void* con
   auto k = ring ? bucket_allreduce_kernel<true, PT> : bucket_allreduce_kernel<false, PT>;
   static const int bps_ring = blocks_per_sm(bucket_allreduce_kernel<true, PT>);
   static const int bps_tree = blocks_per_sm(bucket_allreduce_kernel<false, PT>);
-  const uint32_t grid = std::min<uint32_t>(tiles, (uint32_t)(2 * sm_count() * (ring ? bps_ring : bps_tree)));
+  const uint32_t grid =
+      std::min<uint32_t>(tiles, (uint32_t)(CC_BUCKET_OVERSUB * sm_count() * (ring ? bps_ring : bps_tree)));
   k<<<grid, kThreads, 0, stream>>>(P);
   return cudaGetLastError();
 }
