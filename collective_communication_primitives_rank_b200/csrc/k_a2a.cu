@@ -340,16 +340,6 @@ __global__ void __launch_bounds__(32) a2a_bulk_kernel(const __grid_constant__ A2
   const int s = blockIdx.y;
   const int t = blockIdx.x;
   const int rows = P.tokens * P.topk;
-  const uint32_t rb = (uint32_t)P.row_bytes;
-  if (lane == 0) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bar)));
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    if (P.direction == 0) {  // the token row does not depend on where it goes: fetch it first
-      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(&bar)), "r"(rb) : "memory");
-      asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                   ::"r"(smem_u32(smem)), "l"(P.send[s] + (uint64_t)t * rb), "r"(rb), "r"(smem_u32(&bar)) : "memory");
-    }
-  }
   // position of slot k = lane
   uint64_t pos = 0;
   int dst = -1;
@@ -370,15 +360,21 @@ __global__ void __launch_bounds__(32) a2a_bulk_kernel(const __grid_constant__ A2
     dstk[k] = __shfl_sync(0xffffffffu, dst, k);
   }
   if (lane != 0) return;
+  const uint32_t rb = (uint32_t)P.row_bytes;
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bar)));
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   uint32_t expect = 0;
   if (P.direction == 0) {
-    expect = rb;  // already in flight
+    expect = rb;
   } else {
     for (int k = 0; k < P.topk; ++k) expect += dstk[k] >= 0 ? rb : 0;
   }
   if (expect) {
-    if (P.direction == 1) {
-      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(&bar)), "r"(expect) : "memory");
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(&bar)), "r"(expect) : "memory");
+    if (P.direction == 0) {
+      asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                   ::"r"(smem_u32(smem)), "l"(P.send[s] + (uint64_t)t * rb), "r"(rb), "r"(smem_u32(&bar)) : "memory");
+    } else {
       for (int k = 0; k < P.topk; ++k)
         if (dstk[k] >= 0)
           asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
