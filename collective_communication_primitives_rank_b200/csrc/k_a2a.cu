@@ -321,98 +321,6 @@ __global__ void __launch_bounds__(256) a2a_copy_kernel(const __grid_constant__ A
   }
 }
 
-// ---- K4 with the tensor memory accelerator: one CTA (one warp) per token ------------------------------
-// Lanes 0..topk-1 compute the token's row positions; lane 0 bulk-loads the token row (dispatch)
-// or its topk expert-output rows (combine) into shared memory and bulk-stores them to their
-// destinations. The waits are bounded like every other wait of the library.
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-__device__ __forceinline__ uint64_t a2a_now() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-  return t;
-}
-
-__global__ void __launch_bounds__(32) a2a_bulk_kernel(const __grid_constant__ A2ACopyParams P, int* status) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ uint64_t bar;
-  const int lane = threadIdx.x;
-  const int s = blockIdx.y;
-  const int t = blockIdx.x;
-  const int rows = P.tokens * P.topk;
-  // position of slot k = lane
-  uint64_t pos = 0;
-  int dst = -1;
-  if (lane < P.topk) {
-    const int i = t * P.topk + lane;
-    const int e = P.ids[s][i];
-    if (e >= 0 && e < P.E) {
-      pos = (uint64_t)P.base[s * P.E + e] + P.tile_off[((size_t)s * P.ntiles + i / kTileRows) * P.E + e] +
-            P.row_rank[(size_t)s * rows + i];
-      if (pos < P.capacity) dst = e / P.epr;
-    }
-  }
-  uint64_t posk[kMaxTopk];
-  int dstk[kMaxTopk];
-#pragma unroll
-  for (int k = 0; k < kMaxTopk; ++k) {
-    posk[k] = __shfl_sync(0xffffffffu, pos, k);
-    dstk[k] = __shfl_sync(0xffffffffu, dst, k);
-  }
-  if (lane != 0) return;
-  const uint32_t rb = (uint32_t)P.row_bytes;
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bar)));
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  uint32_t expect = 0;
-  if (P.direction == 0) {
-    expect = rb;
-  } else {
-    for (int k = 0; k < P.topk; ++k) expect += dstk[k] >= 0 ? rb : 0;
-  }
-  if (expect) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(&bar)), "r"(expect) : "memory");
-    if (P.direction == 0) {
-      asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                   ::"r"(smem_u32(smem)), "l"(P.send[s] + (uint64_t)t * rb), "r"(rb), "r"(smem_u32(&bar)) : "memory");
-    } else {
-      for (int k = 0; k < P.topk; ++k)
-        if (dstk[k] >= 0)
-          asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                       ::"r"(smem_u32(smem + (size_t)k * rb)), "l"(P.send[dstk[k]] + posk[k] * rb), "r"(rb),
-                       "r"(smem_u32(&bar)) : "memory");
-    }
-    const uint64_t t0 = a2a_now();
-    for (;;) {
-      uint32_t ok;
-      asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0; selp.u32 %0, 1, 0, p; }"
-                   : "=r"(ok) : "r"(smem_u32(&bar)) : "memory");
-      if (ok) break;
-      if (a2a_now() - t0 > 2000000000ull) {
-        atomicExch(status, (int)CC_ERR_TIMEOUT);
-        return;
-      }
-    }
-    for (int k = 0; k < P.topk; ++k) {
-      if (dstk[k] < 0) continue;
-      void* gdst;
-      const unsigned char* ssrc;
-      if (P.direction == 0) {
-        gdst = P.recv[dstk[k]] + posk[k] * rb;
-        ssrc = smem;
-      } else {
-        gdst = P.recv[s] + ((uint64_t)t * P.topk + k) * rb;
-        ssrc = smem + (size_t)k * rb;
-      }
-      asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(ssrc)),
-                   "r"(rb) : "memory");
-    }
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-  }
-}
-
-constexpr size_t kA2ABulkSmemMax = 96 * 1024;
-
 cudaError_t launch_alltoallv(const void* const* send, void* const* recv, int nranks, size_t row_bytes,
                              const int32_t* const* ids, int tokens, int topk, int experts_per_rank,
                              size_t capacity_rows, int direction, void* workspace, cudaStream_t stream) {
@@ -454,16 +362,6 @@ cudaError_t launch_alltoallv(const void* const* send, void* const* recv, int nra
   P.E = E;
   P.ntiles = ntiles;
   P.direction = direction;
-  const size_t smem = row_bytes * (direction == 0 ? 1 : (size_t)topk);
-  int* status = async_status_word();
-  if (smem <= kA2ABulkSmemMax && status) {
-    static cudaError_t attr = cudaFuncSetAttribute(a2a_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (int)kA2ABulkSmemMax);
-    if (attr == cudaSuccess) {
-      a2a_bulk_kernel<<<dim3(tokens, nranks), 32, smem, stream>>>(P, status);
-      return cudaGetLastError();
-    }
-  }
   a2a_copy_kernel<<<dim3((tokens + 7) / 8, nranks), 256, 0, stream>>>(P);
   return cudaGetLastError();
 }
