@@ -183,6 +183,69 @@ def ring_allgather(shards: Sequence[np.ndarray], *, count: Optional[int] = None,
     return bufs, mesh
 
 
+# ---- hierarchical allreduce -------------------------------------------------------------------
+# Lecture 09 §9.3 design question 1 and appendix A Q4: with N = M nodes x G ranks per node
+# (rank = node * G + local), (1) each node runs a ring reduce-scatter over its G ranks,
+# (2) the G ranks that hold the same shard (one per node) run a ring allreduce across the M
+# nodes, G such rings in parallel, (3) each node runs a ring allgather over its G ranks.
+# Each phase is the ring of the section above on a sub-group (same send indices, same
+# "local (+) incoming" fold), so element e of local chunk c and of sub-chunk j (the chunk
+# rule applied to chunk c with M parts) folds, within every node, x_{m,c} (+) x_{m,c+1} ...
+# and across nodes, starting at node j: (S_j (+) S_{j+1}) (+) ... (reading: the nodes are
+# ordered by index, the inter-node ring is node j -> j + 1).
+
+def _group_ring_rs(ctx, group, pos, buf, sl, op, tag):
+    g = len(group)
+    right, left = group[(pos + 1) % g], group[(pos - 1) % g]
+    for s in range(g - 1):
+        ctx.send(right, buf[sl[(pos - s) % g]], tag=(tag, s))
+        c_in = (pos - s - 1) % g
+        incoming = yield from ctx.recv(left, tag=(tag, s))
+        buf[sl[c_in]] = combine(buf[sl[c_in]], incoming, op)
+
+
+def _group_ring_ag(ctx, group, pos, buf, sl, first_owned_offset, tag):
+    g = len(group)
+    right, left = group[(pos + 1) % g], group[(pos - 1) % g]
+    for s in range(g - 1):
+        ctx.send(right, buf[sl[(pos - s + first_owned_offset) % g]], tag=(tag, s))
+        c_in = (pos - s - 1 + first_owned_offset) % g
+        buf[sl[c_in]] = yield from ctx.recv(left, tag=(tag, s))
+
+
+def hierarchical_allreduce(xs: Sequence[np.ndarray], ranks_per_node: int, *, op: str = SUM, scale: float = 1.0,
+                           in_dtype: str = "f32", count: Optional[int] = None,
+                           positions: Optional[np.ndarray] = None, mesh: Optional[_MeshBase] = None):
+    n = len(xs)
+    G = ranks_per_node
+    if G < 1 or n % G:
+        raise ValueError("the rank count must be a multiple of ranks_per_node")
+    M = n // G
+    bufs = _prep(xs, in_dtype)
+    count = bufs[0].size if count is None else count
+    local_bounds = chunk_bounds(count, G)
+    sl_local = _local_slices(local_bounds, positions)
+    # sub-chunks of every local chunk, for the inter-node rings
+    sl_sub = [_local_slices([(a + p, a + q) for p, q in chunk_bounds(b - a, M)], positions) for a, b in local_bounds]
+    mesh = mesh or LockstepMesh(n, ranks_per_node=G)
+
+    def program(ctx):
+        m, l = divmod(ctx.rank, G)
+        buf = bufs[ctx.rank]
+        node = [m * G + k for k in range(G)]
+        yield from _group_ring_rs(ctx, node, l, buf, sl_local, op, "h1")
+        c = (l + 1) % G  # the local chunk this rank now holds complete for its node
+        peers = [k * G + l for k in range(M)]
+        yield from _group_ring_rs(ctx, peers, m, buf, sl_sub[c], op, "h2rs")
+        own = sl_sub[c][(m + 1) % M]
+        buf[own] = apply_scale(buf[own], scale)
+        yield from _group_ring_ag(ctx, peers, m, buf, sl_sub[c], 1, "h2ag")
+        yield from _group_ring_ag(ctx, node, l, buf, sl_local, 1, "h3")
+
+    mesh.run(program)
+    return bufs, mesh
+
+
 # ---- double binary tree allreduce -------------------------------------------------------------
 # Lecture 09 §5.2 (reduce leaves -> root, then broadcast root -> leaves; 2 log2 N steps) and
 # the multi-node page §4.3.2 (two trees, one per half of the data). Shapes: layout.BinaryTree.

@@ -58,12 +58,16 @@ class _Ctx:
 
 
 class _MeshBase:
-    def __init__(self, n: int):
+    def __init__(self, n: int, ranks_per_node: Optional[int] = None):
         if n < 1:
             raise ValueError("a mesh needs at least one rank")
         self.n = n
         self.sent = [0] * n
         self.recvd = [0] * n
+        # bytes a rank sends to ranks of other nodes (ranks r and s share a node when
+        # r // ranks_per_node == s // ranks_per_node; default: every rank is its own node)
+        self.ranks_per_node = ranks_per_node or 1
+        self.sent_off_node = [0] * n
         self.messages = 0
         self.delivered = 0
         self._seq_out: dict = defaultdict(int)
@@ -73,6 +77,8 @@ class _MeshBase:
         if src != dst:
             self.sent[src] += int(payload.nbytes)
             self.recvd[dst] += int(payload.nbytes)
+            if src // self.ranks_per_node != dst // self.ranks_per_node:
+                self.sent_off_node[src] += int(payload.nbytes)
         self.messages += 1
 
     def _check_seq(self, key, seq: int) -> None:
@@ -85,8 +91,8 @@ class _MeshBase:
 class LockstepMesh(_MeshBase):
     """Single-threaded round-robin driver (deterministic)."""
 
-    def __init__(self, n: int):
-        super().__init__(n)
+    def __init__(self, n: int, ranks_per_node: Optional[int] = None):
+        super().__init__(n, ranks_per_node)
         self._chan: dict = defaultdict(deque)
 
     def _send(self, src, dst, tag, payload):

@@ -368,3 +368,88 @@ def test_lockstep_deadlock_is_reported():
 
     with pytest.raises(ProtocolError):
         mesh.run(program)
+
+
+# ---- hierarchical allreduce (lecture 09 §9.3 Q1, appendix A Q4) ------------------------------------
+
+HIER = [(8, 4), (16, 8), (6, 2), (9, 3), (4, 1), (4, 4), (64, 8), (12, 4)]
+
+
+def _hier_expected(xs, G, count):
+    """Written from the two-level closed form: within each node a left fold over local ranks
+    starting at local chunk c; across nodes a left fold starting at sub-chunk j."""
+    n = len(xs)
+    M = n // G
+    out = np.empty(count, np.float32)
+    for e in range(count):
+        a_c = b_c = c = 0
+        for cc, (a, b) in enumerate(L.chunk_bounds(count, G)):
+            if a <= e < b:
+                c, a_c, b_c = cc, a, b
+        j = next(jj for jj, (p, q) in enumerate(L.chunk_bounds(b_c - a_c, M)) if p <= e - a_c < q)
+        outer = None
+        for dm in range(M):
+            m = (j + dm) % M
+            inner = np.float32(xs[m * G + c][e])
+            for dl in range(1, G):
+                inner = np.float32(inner + xs[m * G + (c + dl) % G][e])
+            outer = inner if outer is None else np.float32(outer + inner)
+        out[e] = outer
+    return out
+
+
+@pytest.mark.parametrize("n,G", HIER)
+def test_hierarchical_int32_equals_brute_force(n, G):
+    count = 3 * n + 5
+    xs = [synth.int32_uniform(31, r, count, -2**31, 2**31 - 1) for r in range(n)]
+    want = (np.sum(np.stack(xs).astype(np.int64), axis=0) & 0xFFFFFFFF).astype(np.uint32).view(np.int32)
+    out, _ = C.hierarchical_allreduce(xs, G, in_dtype="i32")
+    assert all(np.array_equal(o, want) for o in out)
+
+
+@pytest.mark.parametrize("n,G", [(8, 4), (6, 2), (9, 3), (12, 4)])
+def test_hierarchical_fold_is_the_two_level_closed_form(n, G):
+    count = 2 * n + 7
+    xs = _spread_f32(33, n, count)
+    out, _ = C.hierarchical_allreduce(xs, G)
+    want = _hier_expected(xs, G, count)
+    assert all(np.array_equal(_bits(o), _bits(want)) for o in out)
+    flat, _ = C.ring_allreduce(xs)
+    assert not np.array_equal(_bits(flat[0]), _bits(want))  # the probe tells the orders apart
+
+
+@pytest.mark.parametrize("n", [4, 8])
+def test_hierarchical_degenerates_to_the_flat_ring(n):
+    xs = _spread_f32(35, n, 5 * n + 3)
+    flat, _ = C.ring_allreduce(xs, scale=0.5)
+    for G in (1, n):  # one rank per node, or a single node
+        h, _ = C.hierarchical_allreduce(xs, G, scale=0.5)
+        assert all(np.array_equal(_bits(a), _bits(b)) for a, b in zip(h, flat))
+
+
+@pytest.mark.parametrize("n,G", [(16, 8), (64, 8), (8, 2)])
+def test_hierarchical_cuts_cross_node_bytes_per_nic(n, G):
+    """Appendix A Q4: per NIC, cross-node traffic falls by the node size: each rank sends
+    2(M-1)/M * T/G across nodes instead of the flat ring's 2(N-1)/N * T on the node-boundary
+    ranks."""
+    M = n // G
+    count = n * M * 4
+    T = 4 * count
+    xs = [np.ones(count, np.float32) for _ in range(n)]
+    _, mh = C.hierarchical_allreduce(xs, G)
+    assert mh.sent_off_node == [2 * (M - 1) * T // (M * G)] * n
+    _, mf = C.ring_allreduce(xs, mesh=LockstepMesh(n, ranks_per_node=G))
+    assert max(mf.sent_off_node) == 2 * (n - 1) * T // n
+    assert max(mf.sent_off_node) / max(mh.sent_off_node) == pytest.approx(G * (n - 1) * M / (n * (M - 1)))
+
+
+def test_hierarchical_within_fp64_bound_and_sampling():
+    n, G, count = 16, 4, 5003
+    xs = [synth.uniform_f32(36, r, count) for r in range(n)]
+    out, _ = C.hierarchical_allreduce(xs, G, scale=1.0 / n)
+    x64 = np.stack(xs).astype(np.float64)
+    bound = ((n - 1) * 2.0 ** -24 * np.abs(x64).sum(0) + 2.0 ** -24 * np.abs(x64.sum(0))) / n
+    assert np.all(np.abs(out[0].astype(np.float64) - x64.sum(0) / n) <= bound + 1e-30)
+    pos = np.unique(np.concatenate([[0, count - 1], np.arange(1, count, 97)]))
+    part, _ = C.hierarchical_allreduce([x[pos] for x in xs], G, scale=1.0 / n, count=count, positions=pos)
+    assert np.array_equal(_bits(out[5][pos]), _bits(part[5]))
