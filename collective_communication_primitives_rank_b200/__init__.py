@@ -40,6 +40,7 @@ _SIGS = {
     "cc_allreduce": (_i, [_PP, _PP, _i, _sz, _i, _i, _i, _i, _f, _vp]),
     "cc_reduce_scatter": (_i, [_PP, _PP, _i, _sz, _i, _i, _i, _i, _f, _vp]),
     "cc_allreduce_stepped": (_i, [_PP, _PP, _i, _sz, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
+    "cc_allreduce_hierarchical": (_i, [_PP, _PP, _i, _i, _sz, _i, _i, _i, _f, _vp]),
     "cc_allgather": (_i, [_PP, _PP, _i, _sz, _i, _vp]),
     "cc_broadcast": (_i, [_vp, _PP, _i, _i, _sz, _i, _vp]),
     "cc_reduce": (_i, [_PP, _vp, _i, _i, _sz, _i, _i, _i, _f, _vp]),
@@ -174,6 +175,18 @@ def cc_allreduce(send, recv, *, op="sum", algo="ring", scale=1.0, stream=None) -
     _check(lib.cc_allreduce(_ptrs(send), _ptrs(recv), n, send[0].numel(), dtype_code(send[0]),
                             dtype_code(recv[0]), _OPS[op], _ALGOS[algo], float(scale), _stream(stream)),
            "cc_allreduce")
+
+
+def cc_allreduce_hierarchical(send, recv, ranks_per_node: int, *, op="sum", scale=1.0, stream=None) -> None:
+    """recv[r] = what the intra-node RS -> inter-node ring AR -> intra-node AG schedule leaves."""
+    n = _ranks(send, "cc_allreduce_hierarchical")
+    _same(send, send[0].numel(), send[0].dtype, "cc_allreduce_hierarchical send")
+    _same(recv, send[0].numel(), recv[0].dtype, "cc_allreduce_hierarchical recv")
+    if len(recv) != n:
+        raise ValueError("cc_allreduce_hierarchical: one output per rank")
+    _check(lib.cc_allreduce_hierarchical(_ptrs(send), _ptrs(recv), n, int(ranks_per_node), send[0].numel(),
+                                         dtype_code(send[0]), dtype_code(recv[0]), _OPS[op], float(scale),
+                                         _stream(stream)), "cc_allreduce_hierarchical")
 
 
 def cc_allreduce_stepped(send, recv, workspace, *, op="sum", algo="ring", scale=1.0, stream=None) -> None:

@@ -12,8 +12,9 @@ namespace cc {
 
 // Reduction family: allreduce, reduce-scatter, reduce-to-root.
 enum ReduceMode { kAllReduce = 0, kReduceScatter = 1, kReduceRoot = 2 };
-enum FoldKind { kFoldRing = 0, kFoldTree = 1, kFoldBinomial = 2 };
+enum FoldKind { kFoldRing = 0, kFoldTree = 1, kFoldBinomial = 2, kFoldHier = 3 };
 
+// `root` is the root rank for kFoldBinomial and the ranks per node for kFoldHier.
 cudaError_t launch_reduce(const void* const* send, void* const* dst, int ndst, int nranks,
                           size_t count, cc_dtype in_t, cc_op op, FoldKind fold, ReduceMode mode,
                           int root, float scale, cudaStream_t stream);

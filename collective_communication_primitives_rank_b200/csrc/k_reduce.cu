@@ -56,19 +56,17 @@ __device__ __forceinline__ V ring_fold(int n, int c, Load ld, Widen widen) {
   return acc;
 }
 
-// Fold machine (tree / binomial): the position's rank is rmap[p], mirrored for tree B.
-template <int IN, int OP, typename V, typename X, int W, int S = kStackSlots, typename Load, typename Widen>
-__device__ __forceinline__ V machine_fold(int n, const FoldProgram& prog, bool mirror, Load ld, Widen widen) {
+// Fold machine (tree / binomial / hierarchical): position p holds rank rank_of(p).
+template <int IN, int OP, typename V, typename X, int W, int S = kStackSlots, typename RankOf, typename Load,
+          typename Widen>
+__device__ __forceinline__ V machine_fold(int n, const FoldProgram& prog, RankOf rank_of, Load ld, Widen widen) {
   V cur;
   FoldStack<V, S> st;
   for (int p0 = 0; p0 < n; p0 += W) {
     X x[W];
 #pragma unroll
     for (int k = 0; k < W; ++k)
-      if (p0 + k < n) {
-        const int rk = prog.rmap[p0 + k];
-        x[k] = ld(mirror ? n - 1 - rk : rk);
-      }
+      if (p0 + k < n) x[k] = ld(rank_of(p0 + k));
 #pragma unroll
     for (int k = 0; k < W; ++k)
       if (p0 + k < n) fold_step<IN, OP>(prog.code[p0 + k], widen(x[k]), cur, st);
@@ -84,8 +82,8 @@ template <int U> constexpr int stack_slots() { return U == 1 ? kStackSlots : (U 
 // every address is aligned, element-wise head and tail around them. Each thread folds U
 // units at once (units T apart, so warps stay coalesced) with windows of 8 / U positions:
 // about 8 loads in flight per thread for any rank count.
-template <int IN, int OP, bool RING, int U, typename Src, typename EmitU, typename EmitE>
-__device__ __forceinline__ void reduce_range(int n, int g, bool mirror, const FoldProgram& prog,
+template <int IN, int OP, bool RING, int U, typename RankOf, typename Src, typename EmitU, typename EmitE>
+__device__ __forceinline__ void reduce_range(int n, int g, RankOf rank_of, const FoldProgram& prog,
                                              uint64_t a, uint64_t b, uint64_t t, uint64_t T, bool vec,
                                              Src src, EmitU emit_unit, EmitE emit_elem) {
   using A = typename Tr<IN>::Acc;
@@ -95,7 +93,7 @@ __device__ __forceinline__ void reduce_range(int n, int g, bool mirror, const Fo
   auto fold_elem = [&](uint64_t e) -> A {
     auto ld = [&](int r) { return load_elem<IN>(src(r) + e); };
     if constexpr (RING) return ring_fold<IN, OP, A, A>(n, g, ld, same);
-    else return machine_fold<IN, OP, A, A, 8>(n, prog, mirror, ld, same);
+    else return machine_fold<IN, OP, A, A, 8>(n, prog, rank_of, ld, same);
   };
   if (vec) {
     uint64_t va = (a + UE - 1) / UE * UE;
@@ -119,7 +117,7 @@ __device__ __forceinline__ void reduce_range(int n, int g, bool mirror, const Fo
       };
       MU<IN, U> m;
       if constexpr (RING) m = ring_fold<IN, OP, MU<IN, U>, MX<U>, W>(n, g, ld, widen);
-      else m = machine_fold<IN, OP, MU<IN, U>, MX<U>, W, stack_slots<U>()>(n, prog, mirror, ld, widen);
+      else m = machine_fold<IN, OP, MU<IN, U>, MX<U>, W, stack_slots<U>()>(n, prog, rank_of, ld, widen);
 #pragma unroll
       for (int k = 0; k < U; ++k)
         if (k == 0 || e0 + k * step < vb) emit_unit(e0 + k * step, m.u[k]);
@@ -160,8 +158,18 @@ __device__ __forceinline__ int chunk_of(uint64_t count, int n, uint64_t o, uint6
 // The fold group of element o in a buffer of `count` elements: the ring chunk, the tree
 // half, or the single binomial group; returns the group and its [start, end).
 __device__ __forceinline__ int group_of(int fold, uint64_t count, int n, uint64_t o, uint64_t& start,
-                                        uint64_t& end) {
+                                        uint64_t& end, int per_node = 1) {
   if (fold == kFoldRing) return chunk_of(count, n, o, start, end);
+  if (fold == kFoldHier) {
+    // local chunk c of the node's G-way split, then sub-chunk j of that chunk's M-way split
+    const int G = per_node, M = n / per_node;
+    uint64_t ca, cb, ja, jb;
+    const int c = chunk_of(count, G, o, ca, cb);
+    const int j = chunk_of(cb - ca, M, o - ca, ja, jb);
+    start = ca + ja;
+    end = ca + jb;
+    return c * M + j;
+  }
   if (fold == kFoldTree) {
     const uint64_t mid = (count + 1) / 2;
     const int g = o >= mid;
@@ -184,6 +192,7 @@ struct ReduceParams {
   uint64_t tile;         // elements per tile (a multiple of 8)
   uint64_t dst_aligned;  // bit r: dst[r] is 16-byte aligned
   int nranks;
+  int per_node;  // ranks per node (hierarchical fold)
   int mode;
   int fold;
   int vec;  // every source (and every allreduce / root destination) is 16-byte aligned
@@ -208,9 +217,15 @@ __global__ void __launch_bounds__(kThreads, (RING && U == 1) ? CC_RING_MIN_BLOCK
     uint64_t s = ea;
     while (s < eb) {
       uint64_t ga, gb;
-      const int g = group_of(P.fold, P.count, n, s, ga, gb);
+      const int g = group_of(P.fold, P.count, n, s, ga, gb, P.per_node);
       const uint64_t se = min(eb, gb);
       const bool mirror = (P.fold == kFoldTree && g == 1);
+      const int G = P.per_node, M = n / P.per_node, hc = g / M, hj = g % M;
+      auto rank_of = [&](int p) {
+        if (P.fold == kFoldHier) return ((hj + p / G) % M) * G + (hc + p % G) % G;
+        const int rk = P.prog.rmap[p];
+        return mirror ? n - 1 - rk : rk;
+      };
       const bool shard_vec = ((P.dst_aligned >> g) & 1) && ((ga * sizeof(Out)) % 16 == 0);
       auto emit_unit = [&](uint64_t e, Unit<IN> u) {
         if (P.do_scale) scale_unit<IN>(u, P.scale);
@@ -233,8 +248,8 @@ __global__ void __launch_bounds__(kThreads, (RING && U == 1) ? CC_RING_MIN_BLOCK
           store_elem<IN>(static_cast<Out*>(P.dst[0]) + e, v);
         }
       };
-      reduce_range<IN, OP, RING, U>(n, g, mirror, P.prog, s, se, threadIdx.x, blockDim.x, P.vec != 0, src, emit_unit,
-                                    emit_elem);
+      reduce_range<IN, OP, RING, U>(n, g, rank_of, P.prog, s, se, threadIdx.x, blockDim.x, P.vec != 0, src,
+                                    emit_unit, emit_elem);
       s = se;
     }
   }
@@ -335,8 +350,13 @@ __global__ void __launch_bounds__(kThreads, RING ? CC_BUCKET_MIN_BLOCKS : 2) buc
         gend = g ? d.bucket_count : mid;
       }
       const uint64_t se = min(eb, gend - d.bucket_off);
-      reduce_range<IN, OP, RING, 1>(n, g, !RING && g == 1, P.prog, s, se, threadIdx.x, blockDim.x,
-                                    P.vec != 0, src, emit_unit, emit_elem);
+      const bool mirror = !RING && g == 1;
+      auto rank_of = [&](int p) {
+        const int rk = P.prog.rmap[p];
+        return mirror ? n - 1 - rk : rk;
+      };
+      reduce_range<IN, OP, RING, 1>(n, g, rank_of, P.prog, s, se, threadIdx.x, blockDim.x, P.vec != 0, src,
+                                    emit_unit, emit_elem);
       s = se;
     }
     __syncthreads();  // every thread is done with s_in / s_out before the next tile restages them
@@ -423,6 +443,25 @@ static void binomial_program(int n, int root, FoldProgram& fp) {
   }
 }
 
+// Hierarchical fold in machine codes: positions run node by node (G local ranks each); a
+// node's ranks are left-folded into cur; the first node's fold is pushed, each middle
+// node's is folded into it (top = top (+) cur), the last node's pops it (cur = top (+) cur).
+// The rank at each position depends on the element's group and is computed in the kernel.
+static void hier_program(int n, int G, FoldProgram& fp) {
+  const int M = n / G;
+  for (int p = 0; p < n; ++p) {
+    const int k = p / G, i = p % G;
+    uint8_t code = i > 0 ? kFoldCur : 0;
+    if (i == G - 1 && M > 1) {
+      if (k == 0) code |= kPush;
+      else if (k < M - 1) code |= kFoldTop;
+      else code |= (uint8_t)(1 << 2);  // one pop
+    }
+    fp.code[p] = code;
+    fp.rmap[p] = (uint8_t)p;
+  }
+}
+
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 int sm_count() {
@@ -460,7 +499,9 @@ static cudaError_t run_reduce(ReduceParams& P, cudaStream_t s) {
   P.tile = upt * kThreads * UE;
   // a tile never spans much more than one fold group, so that the groups of a small
   // buffer (N ring chunks of a few elements each) are folded by different CTAs in parallel
-  const uint64_t ngroups = P.fold == kFoldRing ? (uint64_t)P.nranks : (P.fold == kFoldTree ? 2 : 1);
+  const uint64_t ngroups = P.fold == kFoldRing ? (uint64_t)P.nranks
+                           : P.fold == kFoldTree ? 2
+                           : P.fold == kFoldHier ? (uint64_t)P.nranks : 1;
   const uint64_t per_group = ((P.count + ngroups - 1) / ngroups + 7) / 8 * 8;
   P.tile = std::max<uint64_t>(8, std::min<uint64_t>(P.tile, per_group));
   const uint64_t ntiles = (P.count + P.tile - 1) / P.tile;
@@ -515,8 +556,13 @@ cudaError_t launch_reduce(const void* const* send, void* const* dst, int ndst, i
     else if (mode != kReduceScatter) vec = false;
   }
   P.vec = vec;
+  P.per_node = 1;
   if (fold == kFoldTree) tree_program(nranks, P.prog);
   else if (fold == kFoldBinomial) binomial_program(nranks, root, P.prog);
+  else if (fold == kFoldHier) {
+    P.per_node = root;
+    hier_program(nranks, root, P.prog);
+  }
   const bool ring = fold == kFoldRing;
   // several columns per thread pay off for the fold machine (tree, binomial) at small N;
   // the ring's plain left fold is faster with one column and twice the resident CTAs

@@ -119,6 +119,20 @@ CC_API cc_status cc_allreduce_stepped(const void* const* send, void* const* recv
                                       cc_dtype in_t, cc_dtype out_t, cc_op op, cc_algo algo, float scale,
                                       void* workspace, size_t workspace_bytes, void* stream);
 
+/* Hierarchical AllReduce (lecture 09 §9.3 design question 1, appendix A Q4): the N ranks
+ * form N / ranks_per_node nodes of ranks_per_node consecutive ranks. The result is what the
+ * three-phase schedule leaves on every rank: a ring reduce-scatter inside every node, then
+ * for every shard a ring allreduce across the nodes (ranks_per_node rings in parallel), then
+ * a ring allgather inside every node. Element e of local chunk c (chunk rule over count with
+ * ranks_per_node parts) and of sub-chunk j (chunk rule over chunk c with N / ranks_per_node
+ * parts) folds x_{m,c} (+) x_{m,c+1} (+) ... inside each node m, and the node sums in node
+ * order starting at node j; then `scale`. One fused pass (N·T in, N·T out). ranks_per_node
+ * must divide nranks (else CC_ERR_INVALID_ARG); 1 or nranks give cc_allreduce's ring.
+ * Other arguments as cc_allreduce. */
+CC_API cc_status cc_allreduce_hierarchical(const void* const* send, void* const* recv, int nranks,
+                                           int ranks_per_node, size_t count, cc_dtype in_t,
+                                           cc_dtype out_t, cc_op op, float scale, void* stream);
+
 /* ReduceScatter (lecture 09 §3.6; the from-scratch page's reduce_scatter as the first
  * half of the ring). Rank c receives, in recv[c], chunk c (chunk rule) of the ring
  * reduction: q + (c < r) elements of out_t. `count` is the per-rank INPUT length.

@@ -273,3 +273,33 @@ def test_stepped_in_place_other_ops(op):
         torch.cuda.synchronize()
         for r in range(n):
             _assert_same(to_host(buf[r]), want[r], f"stepped in place {op} {algo} rank {r}")
+
+
+# ---- hierarchical allreduce: the two-level fold, fused ----------------------------------------------------
+
+@pytest.mark.parametrize("n,G,count", [(8, 4, 4096), (16, 8, 16 * 1000 + 7), (6, 2, 999), (9, 3, 3001), (4, 1, 77),
+                                       (4, 4, 4096), (64, 8, 64 * 50 + 13), (2, 1, 10), (12, 4, 12 * 4096)])
+@pytest.mark.parametrize("kind", ["spread", "i32", "bf16"])
+def test_hierarchical_allreduce_matches_oracle(n, G, count, kind):
+    xs = _inputs(kind, n, count, seed=40)
+    scale = 1.0 if kind == "i32" else 1.0 / n
+    want, _ = C.hierarchical_allreduce(xs, G, in_dtype=_IN[kind], scale=scale)
+    out = [Guarded(count, _out_dtype(kind)) for _ in range(n)]
+    cc.cc_allreduce_hierarchical([to_dev(x) for x in xs], [o.t for o in out], G, scale=scale)
+    torch.cuda.synchronize()
+    for r in range(n):
+        _assert_same(to_host(out[r].t), want[r], f"hierarchical {kind} N={n} G={G} rank {r}")
+        out[r].check()
+
+
+def test_hierarchical_in_place_and_large_sampled():
+    n, G, count = 64, 8, 4 * 1024 * 1024 + 5
+    xs = [synth.uniform_f32(41, r, count) for r in range(n)]
+    buf = [to_dev(x) for x in xs]
+    cc.cc_allreduce_hierarchical(buf, buf, G, scale=1.0 / n)
+    torch.cuda.synchronize()
+    pos = np.unique(np.concatenate([[0, count - 1], np.arange(3, count, 4099)]))
+    want, _ = C.hierarchical_allreduce([x[pos] for x in xs], G, scale=1.0 / n, count=count, positions=pos)
+    idx = torch.from_numpy(pos).cuda()
+    for r in (0, 37, n - 1):
+        _assert_same(buf[r][idx].cpu().numpy(), want[r], f"rank {r}")
