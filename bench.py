@@ -437,6 +437,20 @@ def run_rows(args):
             if n == 8 and size == 256 * 1024 * 1024:
                 best = row
             del x, y
+    # hierarchical allreduce (8 ranks per node) at the large sizes
+    hier = []
+    for n, mib in ((16, 256), (64, 64)):
+        count = mib * 1024 * 1024 // 4
+        x = [torch.rand(count, device="cuda", generator=gen) * 2 - 1 for _ in range(n)]
+        y = [torch.empty_like(t) for t in x]
+        call = _prepared(cc, "cc_allreduce_hierarchical", cc._ptrs(x), cc._ptrs(y), n, 8, count, cc.CC_F32,
+                         cc.CC_F32, cc.CC_SUM, 1.0, torch.cuda.current_stream().cuda_stream)
+        for _ in range(3):
+            call()
+        ms = _event_time_ms(torch, call, 5) / 5
+        hier.append({"n": n, "ranks_per_node": 8, "bytes_per_rank": count * 4, "us": ms * 1e3,
+                     "GBps": 2 * n * count * 4 / (ms * 1e-3) / 1e9})
+        del x, y
     cross, cross_stepped = {}, {}
     for n in (2, 4, 8, 16, 32, 64):
         pts = [r for r in table if r["n"] == n]
@@ -451,7 +465,8 @@ def run_rows(args):
                "l2": "L2 flushed (256 MiB write) before every timed call whose working set fits in L2"},
               {"achieved": best["ring_GBps"], "kernel": "reduce_kernel<f32,sum,ring>"},
               len(table) * 2,
-              {"sweep": table, "crossover": cross, "crossover_stepped": cross_stepped, "min_launch_latency_us": lat})
+              {"sweep": table, "crossover": cross, "crossover_stepped": cross_stepped, "hierarchical": hier,
+               "min_launch_latency_us": lat})
     return 0
 
 
