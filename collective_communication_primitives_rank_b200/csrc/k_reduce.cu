@@ -40,15 +40,19 @@ constexpr int kThreads = 256;
 // 128-bit loads per thread are in flight before the in-order folds consume them.
 // V is the accumulator (a unit or an element), X what one load returns (raw 16 bytes for a
 // unit, the element itself otherwise).
+// `up` false walks the ranks downwards (the left fold of a mirrored tree).
 template <int IN, int OP, typename V, typename X, int W = 8, typename Load, typename Widen>
-__device__ __forceinline__ V ring_fold(int n, int c, Load ld, Widen widen) {
+__device__ __forceinline__ V ring_fold(int n, int c, Load ld, Widen widen, bool up = true) {
   V acc = widen(ld(c));
   int r = c;
   for (int j0 = 1; j0 < n; j0 += W) {
     X x[W];
 #pragma unroll
     for (int k = 0; k < W; ++k)
-      if (j0 + k < n) { r = (r + 1 == n) ? 0 : r + 1; x[k] = ld(r); }
+      if (j0 + k < n) {
+        r = up ? (r + 1 == n ? 0 : r + 1) : (r == 0 ? n - 1 : r - 1);
+        x[k] = ld(r);
+      }
 #pragma unroll
     for (int k = 0; k < W; ++k)
       if (j0 + k < n) comb<IN, OP>(acc, x[k]);
@@ -85,14 +89,19 @@ template <int U> constexpr int stack_slots() { return U == 1 ? kStackSlots : (U 
 template <int IN, int OP, bool RING, int U, typename RankOf, typename Src, typename EmitU, typename EmitE>
 __device__ __forceinline__ void reduce_range(int n, int g, RankOf rank_of, const FoldProgram& prog,
                                              uint64_t a, uint64_t b, uint64_t t, uint64_t T, bool vec,
-                                             Src src, EmitU emit_unit, EmitE emit_elem) {
+                                             Src src, EmitU emit_unit, EmitE emit_elem,
+                                             bool linear_tree = false) {
   using A = typename Tr<IN>::Acc;
   constexpr int UE = Tr<IN>::UE;
   constexpr int W = 8 / U;
   auto same = [](const A& x) { return x; };
+  // a RING fold starts at rank g and walks up; a linear tree fold (g = 0 or 1 for tree A / B)
+  // starts at rank 0 and walks up, or at rank n-1 and walks down
+  const int start = linear_tree ? (g == 0 ? 0 : n - 1) : g;
+  const bool up = !linear_tree || g == 0;
   auto fold_elem = [&](uint64_t e) -> A {
     auto ld = [&](int r) { return load_elem<IN>(src(r) + e); };
-    if constexpr (RING) return ring_fold<IN, OP, A, A>(n, g, ld, same);
+    if constexpr (RING) return ring_fold<IN, OP, A, A>(n, start, ld, same, up);
     else return machine_fold<IN, OP, A, A, 8>(n, prog, rank_of, ld, same);
   };
   if (vec) {
@@ -116,7 +125,7 @@ __device__ __forceinline__ void reduce_range(int n, int g, RankOf rank_of, const
         return x;
       };
       MU<IN, U> m;
-      if constexpr (RING) m = ring_fold<IN, OP, MU<IN, U>, MX<U>, W>(n, g, ld, widen);
+      if constexpr (RING) m = ring_fold<IN, OP, MU<IN, U>, MX<U>, W>(n, start, ld, widen, up);
       else m = machine_fold<IN, OP, MU<IN, U>, MX<U>, W, stack_slots<U>()>(n, prog, rank_of, ld, widen);
 #pragma unroll
       for (int k = 0; k < U; ++k)
@@ -249,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, (RING && U == 1) ? CC_RING_MIN_BLOCK
         }
       };
       reduce_range<IN, OP, RING, U>(n, g, rank_of, P.prog, s, se, threadIdx.x, blockDim.x, P.vec != 0, src,
-                                    emit_unit, emit_elem);
+                                    emit_unit, emit_elem, RING && P.fold == kFoldTree);
       s = se;
     }
   }
@@ -400,6 +409,24 @@ static void tree_program(int n, FoldProgram& fp) {
     fp.code[p] = code;
     fp.rmap[p] = (uint8_t)p;
   }
+  // A right child that is a leaf is the very next position: instead of pushing
+  // (S_left (+) x) and popping it back after the leaf, fold the leaf into cur directly
+  // (((S_left (+) x) (+) leaf), the same operations in the same order).
+  for (int p = 0; p + 1 < n; ++p) {
+    const int q = p + 1;
+    if (right[q] == q + 1 && (fp.code[p] & kPush) && npop_of(fp.code[p + 1]) > 0) {
+      fp.code[p] &= (uint8_t)~kPush;
+      const int np = npop_of(fp.code[p + 1]) - 1;
+      fp.code[p + 1] = (uint8_t)((fp.code[p + 1] & ~(7 << 2)) | kFoldCur | (np << 2));
+    }
+  }
+}
+
+// A program without pushes, pops or fold-into-top is a left fold in position order.
+static bool program_is_linear(int n, const FoldProgram& fp) {
+  for (int p = 0; p < n; ++p)
+    if ((fp.code[p] & (kPush | kFoldTop)) || npop_of(fp.code[p])) return false;
+  return true;
 }
 
 // Binomial tree rooted at `root` (relative rank v = (r - root) mod n; parent v - 2^floor(log2 v);
@@ -563,7 +590,8 @@ cudaError_t launch_reduce(const void* const* send, void* const* dst, int ndst, i
     P.per_node = root;
     hier_program(nranks, root, P.prog);
   }
-  const bool ring = fold == kFoldRing;
+  // the ring, and a tree whose fold is a plain left fold (N <= 5), run the ring kernel
+  const bool ring = fold == kFoldRing || (fold == kFoldTree && program_is_linear(nranks, P.prog));
   // several columns per thread pay off for the fold machine (tree, binomial) at small N;
   // the ring's plain left fold is faster with one column and twice the resident CTAs
   int cols = ring ? 1 : (nranks <= 2 ? 4 : (nranks <= 4 ? 2 : 1));
