@@ -3,7 +3,7 @@
 // All of them are "copy entry k (src, bytes) to one destination, or to the same offset
 // of every rank's buffer" (fan-out). Each source byte is read once and written to each
 // destination: allgather reads T and writes N·T, the minimum. Entries are cut into tiles;
-// a CTA takes tiles round-robin (binary search in the tile prefix table).
+// a CTA finds its tile's entry by binary search in the tile prefix table.
 //
 // copy_bulk_tile_kernel (every entry 16-byte aligned): the tensor memory accelerator moves
 // the data. One CTA per 32 KiB tile; its one working thread issues a cp.async.bulk load of

@@ -266,9 +266,10 @@ __global__ void __launch_bounds__(kThreads, (RING && U == 1) ? CC_RING_MIN_BLOCK
 
 // ---- fused DDP bucket allreduce --------------------------------------------------------------------
 // One launch covers a group of gradient tensors. Work is cut into tiles of kBucketTile
-// elements that never cross a tensor; a CTA takes tiles round-robin, finds the tile's
-// tensor by binary search in the tile prefix table, and splits the tile at the fold-group
-// boundaries of the tensor's bucket (ring chunks or tree halves, in bucket coordinates).
+// elements that never cross a tensor, one CTA per tile; a CTA finds its tile's tensor by
+// binary search in the tile prefix table, stages that tensor's 2N pointers in shared
+// memory, and splits the tile at the fold-group boundaries of the tensor's bucket (ring
+// chunks or tree halves, in bucket coordinates).
 // Every element is folded exactly as in flatten -> allreduce -> unflatten, with no flat
 // buffer: N·G bytes in, N·G bytes out.
 
