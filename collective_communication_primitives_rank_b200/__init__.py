@@ -56,6 +56,7 @@ _SIGS = {
     "cc_bucket_unflatten": (_i, [_vp, _PP, _SZP, _i, _i, _vp]),
     "cc_bucket_allreduce": (_i, [_PP, _PP, _i, _i, _SZP, _sz, _i, _f, _vp]),
     "cc_bucket_allreduce_host": (_i, [_PP, _PP, _PP, _PP, _i, _i, _SZP, _sz, _i, _f, _vp]),
+    "cc_bucket_allreduce_buckets": (_i, [_PP, _PP, _i, _i, _SZP, _sz, _i, _i, _i, _f, _vp]),
 }
 
 
@@ -392,6 +393,14 @@ class BucketAllreducePlan:
                       _stream(stream))
         if st != CC_OK:
             raise CCError(st, "cc_bucket_allreduce")
+
+    def run_buckets(self, first: int, count: int = 1, stream=None) -> None:
+        """Only buckets [first, first + count) of the plan's assignment (for overlap with
+        backward: launch each bucket on a side stream once its gradients exist)."""
+        st = get_lib().cc_bucket_allreduce_buckets(self._in, self._out, self.n, self.nt, self._numels, self.cap_bytes,
+                                                   int(first), int(count), self.algo, self.scale, _stream(stream))
+        if st != CC_OK:
+            raise CCError(st, "cc_bucket_allreduce_buckets")
 
 
 class BucketAllreduceHostPlan:

@@ -514,6 +514,28 @@ cc_status cc_bucket_allreduce(const void* const* grads, void* const* out, int nr
   return CC_OK;
 }
 
+cc_status cc_bucket_allreduce_buckets(const void* const* grads, void* const* out, int nranks, int ntensors,
+                                      const size_t* numels, size_t cap_bytes, int first_bucket, int nbuckets,
+                                      cc_algo algo, float scale, void* stream) {
+  if (!valid_ranks(nranks) || ntensors < 0 || cap_bytes == 0 || !(scale == scale) || first_bucket < 0 ||
+      nbuckets < 0)
+    return CC_ERR_INVALID_ARG;
+  if (algo != CC_ALGO_RING && algo != CC_ALGO_TREE) return CC_ERR_INVALID_ARG;
+  if (ntensors == 0 || nbuckets == 0) return CC_OK;
+  if (!numels || !grads || !out) return CC_ERR_INVALID_ARG;
+  const BucketLayout L = bucket_layout(numels, ntensors, cap_bytes);
+  if (first_bucket + nbuckets > L.nb) return CC_ERR_INVALID_ARG;
+  for (int k = L.start[first_bucket]; k < L.start[first_bucket + nbuckets]; ++k)
+    for (int r = 0; r < nranks; ++r) {
+      const int i = L.order[k];
+      if (numels[i] && (!grads[(size_t)r * ntensors + i] || !out[(size_t)r * ntensors + i])) return CC_ERR_INVALID_ARG;
+    }
+  if (launch_bucket_range(grads, out, nranks, ntensors, L, L.start[first_bucket], L.start[first_bucket + nbuckets],
+                          algo == CC_ALGO_RING ? kFoldRing : kFoldTree, scale, as_stream(stream)) != cudaSuccess)
+    return CC_ERR_CUDA;
+  return CC_OK;
+}
+
 cc_status cc_bucket_allreduce_host(const void* const* host_grads, void* const* host_out, void* const* dev_grads,
                                    void* const* dev_out, int nranks, int ntensors, const size_t* numels,
                                    size_t cap_bytes, cc_algo algo, float scale, void* stream) {

@@ -246,6 +246,18 @@ CC_API cc_status cc_bucket_allreduce(const void* const* grads, void* const* out,
                               const size_t* numels, size_t cap_bytes, cc_algo algo, float scale,
                               void* stream);
 
+/* Buckets [first_bucket, first_bucket + nbuckets) of the assignment cc_bucket_assign makes
+ * for the whole tensor list, with the same results as cc_bucket_allreduce for their tensors
+ * (other tensors are not touched). This is how a training step overlaps the allreduce with
+ * backward (lecture 09 §6.1 bucket overlap; the from-scratch page's bucket-ready hooks):
+ * buckets come in the order backward produces gradients, so bucket b can be launched on a
+ * side stream as soon as its last gradient is written (cudaStreamWaitEvent on an event
+ * recorded after it). CC_ERR_INVALID_ARG if the range exceeds the bucket count. */
+CC_API cc_status cc_bucket_allreduce_buckets(const void* const* grads, void* const* out, int nranks,
+                                             int ntensors, const size_t* numels, size_t cap_bytes,
+                                             int first_bucket, int nbuckets, cc_algo algo, float scale,
+                                             void* stream);
+
 /* The same fused DDP step for gradients that live in host memory: every host_grads[j] is
  * copied to dev_grads[j] (host -> device), the fused allreduce runs on the device copies,
  * and every dev_out[j] is copied back to host_out[j] (device -> host). The work is cut in

@@ -168,3 +168,31 @@ def test_flatten_allreduce_unflatten_equals_fused():
     for r in range(n):
         for i in range(len(shapes)):
             assert np.array_equal(bits(to_host(outs[r][i])), bits(want[r][i]))
+
+
+def test_bucket_overlap_with_a_simulated_backward():
+    """Backward writes the gradients bucket by bucket on the compute stream; each bucket's
+    allreduce is launched on a side stream as soon as its gradients exist (event wait), while
+    backward goes on. The result equals the oracle's whole-step allreduce."""
+    n, cap = 8, 30_000
+    shapes, grads = _small_model(n, seed=11)
+    want, _ = ddp.ddp_allreduce(grads, cap_bytes=cap)
+    src = [[to_dev(g) for g in row] for row in grads]  # what backward will produce
+    d_in = [[torch.zeros_like(t) for t in row] for row in src]
+    out = [[torch.empty_like(t) for t in row] for row in src]
+    plan = cc.BucketAllreducePlan(d_in, out, cap_bytes=cap)
+    buckets = cc.cc_bucket_assign([g.size for g in grads[0]], 4, cap)
+    compute, comm = torch.cuda.current_stream(), torch.cuda.Stream()
+    for b, members in enumerate(buckets):
+        for r in range(n):
+            for i in members:
+                d_in[r][i].copy_(src[r][i])  # "backward" produces bucket b's gradients
+        ready = torch.cuda.Event()
+        ready.record(compute)
+        comm.wait_event(ready)
+        plan.run_buckets(b, 1, stream=comm)
+    compute.wait_stream(comm)
+    torch.cuda.synchronize()
+    for r in range(n):
+        for i in range(len(shapes)):
+            assert np.array_equal(bits(to_host(out[r][i])), bits(want[r][i])), f"rank {r} tensor {i}"
