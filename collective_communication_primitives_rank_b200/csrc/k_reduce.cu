@@ -78,6 +78,36 @@ __device__ __forceinline__ V machine_fold(int n, const FoldProgram& prog, RankOf
   return cur;
 }
 
+// Hierarchical fold: node by node, starting at node j, each node's G ranks left-folded
+// starting at local rank c (windows of 8 loads), the node sums left-folded in node order.
+template <int IN, int OP, typename V, typename X, typename Load, typename Widen>
+__device__ __forceinline__ V hier_fold(int n, int G, int c, int j, Load ld, Widen widen) {
+  const int M = n / G;
+  V outer;
+  int m = j;
+  for (int k = 0; k < M; ++k) {
+    const int base = m * G;
+    V inner = widen(ld(base + c));
+    int l = c;
+    for (int i0 = 1; i0 < G; i0 += 8) {
+      X x[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (i0 + q < G) {
+          l = (l + 1 == G) ? 0 : l + 1;
+          x[q] = ld(base + l);
+        }
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (i0 + q < G) comb<IN, OP>(inner, x[q]);
+    }
+    if (k == 0) outer = inner;
+    else comb<IN, OP>(outer, inner);
+    m = (m + 1 == M) ? 0 : m + 1;
+  }
+  return outer;
+}
+
 // Pending-partial slots the fold machine needs with U columns per thread: U > 1 is only
 // used for N <= 8 / U ranks, whose trees need at most 2 (U = 4) or 3 (U = 2) slots.
 template <int U> constexpr int stack_slots() { return U == 1 ? kStackSlots : (U == 2 ? 4 : 2); }
@@ -86,11 +116,16 @@ template <int U> constexpr int stack_slots() { return U == 1 ? kStackSlots : (U 
 // every address is aligned, element-wise head and tail around them. Each thread folds U
 // units at once (units T apart, so warps stay coalesced) with windows of 8 / U positions:
 // about 8 loads in flight per thread for any rank count.
-template <int IN, int OP, bool RING, int U, typename RankOf, typename Src, typename EmitU, typename EmitE>
+// KIND: kLinear (ring order or a linear tree), kMachine (tree / binomial programs),
+// kHier (two-level); hG / hc / hj describe the hierarchical group.
+constexpr int kLinear = 0, kMachine = 1, kHier = 2;
+
+template <int IN, int OP, int KIND, int U, typename RankOf, typename Src, typename EmitU, typename EmitE>
 __device__ __forceinline__ void reduce_range(int n, int g, RankOf rank_of, const FoldProgram& prog,
                                              uint64_t a, uint64_t b, uint64_t t, uint64_t T, bool vec,
                                              Src src, EmitU emit_unit, EmitE emit_elem,
-                                             bool linear_tree = false) {
+                                             bool linear_tree = false, int hG = 1, int hc = 0, int hj = 0) {
+  constexpr bool RING = KIND == kLinear;
   using A = typename Tr<IN>::Acc;
   constexpr int UE = Tr<IN>::UE;
   constexpr int W = 8 / U;
@@ -102,6 +137,7 @@ __device__ __forceinline__ void reduce_range(int n, int g, RankOf rank_of, const
   auto fold_elem = [&](uint64_t e) -> A {
     auto ld = [&](int r) { return load_elem<IN>(src(r) + e); };
     if constexpr (RING) return ring_fold<IN, OP, A, A>(n, start, ld, same, up);
+    else if constexpr (KIND == kHier) return hier_fold<IN, OP, A, A>(n, hG, hc, hj, ld, same);
     else return machine_fold<IN, OP, A, A, 8>(n, prog, rank_of, ld, same);
   };
   if (vec) {
@@ -126,6 +162,7 @@ __device__ __forceinline__ void reduce_range(int n, int g, RankOf rank_of, const
       };
       MU<IN, U> m;
       if constexpr (RING) m = ring_fold<IN, OP, MU<IN, U>, MX<U>, W>(n, start, ld, widen, up);
+      else if constexpr (KIND == kHier) m = hier_fold<IN, OP, MU<IN, U>, MX<U>>(n, hG, hc, hj, ld, widen);
       else m = machine_fold<IN, OP, MU<IN, U>, MX<U>, W, stack_slots<U>()>(n, prog, rank_of, ld, widen);
 #pragma unroll
       for (int k = 0; k < U; ++k)
@@ -212,8 +249,10 @@ struct ReduceParams {
 // Each CTA folds contiguous tiles (normally exactly one: the grid is sized to the tile
 // count); a tile is split where it crosses a fold group (ring chunk or tree half) and each
 // piece is folded by the whole CTA.
-template <int IN, int OP, bool RING, int U>
-__global__ void __launch_bounds__(kThreads, (RING && U == 1) ? CC_RING_MIN_BLOCKS : 2) reduce_kernel(const __grid_constant__ ReduceParams P) {
+template <int IN, int OP, int KIND, int U>
+__global__ void __launch_bounds__(kThreads, KIND == kLinear ? CC_RING_MIN_BLOCKS : KIND == kHier ? 3 : 2)
+    reduce_kernel(const __grid_constant__ ReduceParams P) {
+  constexpr bool RING = KIND == kLinear;
   using In = typename Tr<IN>::In;
   using Out = typename Tr<IN>::Out;
   using A = typename Tr<IN>::Acc;
@@ -257,8 +296,8 @@ __global__ void __launch_bounds__(kThreads, (RING && U == 1) ? CC_RING_MIN_BLOCK
           store_elem<IN>(static_cast<Out*>(P.dst[0]) + e, v);
         }
       };
-      reduce_range<IN, OP, RING, U>(n, g, rank_of, P.prog, s, se, threadIdx.x, blockDim.x, P.vec != 0, src,
-                                    emit_unit, emit_elem, RING && P.fold == kFoldTree);
+      reduce_range<IN, OP, KIND, U>(n, g, rank_of, P.prog, s, se, threadIdx.x, blockDim.x, P.vec != 0, src,
+                                    emit_unit, emit_elem, RING && P.fold == kFoldTree, G, hc, hj);
       s = se;
     }
   }
@@ -365,8 +404,8 @@ __global__ void __launch_bounds__(kThreads, RING ? CC_BUCKET_MIN_BLOCKS : 2) buc
         const int rk = P.prog.rmap[p];
         return mirror ? n - 1 - rk : rk;
       };
-      reduce_range<IN, OP, RING, 1>(n, g, rank_of, P.prog, s, se, threadIdx.x, blockDim.x, P.vec != 0, src,
-                                    emit_unit, emit_elem);
+      reduce_range<IN, OP, RING ? kLinear : kMachine, 1>(n, g, rank_of, P.prog, s, se, threadIdx.x, blockDim.x,
+                                                         P.vec != 0, src, emit_unit, emit_elem);
       s = se;
     }
     __syncthreads();  // every thread is done with s_in / s_out before the next tile restages them
@@ -513,9 +552,9 @@ static int blocks_per_sm(K kernel) {
   return b;
 }
 
-template <int IN, int OP, bool RING, int U>
+template <int IN, int OP, int KIND, int U>
 static cudaError_t run_reduce(ReduceParams& P, cudaStream_t s) {
-  auto k = reduce_kernel<IN, OP, RING, U>;
+  auto k = reduce_kernel<IN, OP, KIND, U>;
   static const int bps = blocks_per_sm(k);
   constexpr uint64_t UE = Tr<IN>::UE * U;
   const uint64_t resident = (uint64_t)sm_count() * bps;
@@ -540,16 +579,21 @@ static cudaError_t run_reduce(ReduceParams& P, cudaStream_t s) {
 
 // Columns per thread for SUM (the other operators fold one column).
 template <int IN>
-static cudaError_t dispatch_op(ReduceParams& P, cc_op op, bool ring, int cols, cudaStream_t s) {
+static cudaError_t dispatch_op(ReduceParams& P, cc_op op, int kind, int cols, cudaStream_t s) {
+#define CC_KINDS(OPV)                                                                         \
+  if (kind == kLinear) return run_reduce<IN, OPV, kLinear, 1>(P, s);                         \
+  if (kind == kHier) return run_reduce<IN, OPV, kHier, 1>(P, s);                             \
+  return run_reduce<IN, OPV, kMachine, 1>(P, s);
   switch (op) {
     case CC_SUM:
-      if (cols == 4) return ring ? run_reduce<IN, CC_SUM, true, 4>(P, s) : run_reduce<IN, CC_SUM, false, 4>(P, s);
-      if (cols == 2) return ring ? run_reduce<IN, CC_SUM, true, 2>(P, s) : run_reduce<IN, CC_SUM, false, 2>(P, s);
-      return ring ? run_reduce<IN, CC_SUM, true, 1>(P, s) : run_reduce<IN, CC_SUM, false, 1>(P, s);
-    case CC_MAX: return ring ? run_reduce<IN, CC_MAX, true, 1>(P, s) : run_reduce<IN, CC_MAX, false, 1>(P, s);
-    case CC_MIN: return ring ? run_reduce<IN, CC_MIN, true, 1>(P, s) : run_reduce<IN, CC_MIN, false, 1>(P, s);
-    case CC_PROD: return ring ? run_reduce<IN, CC_PROD, true, 1>(P, s) : run_reduce<IN, CC_PROD, false, 1>(P, s);
+      if (kind == kMachine && cols == 4) return run_reduce<IN, CC_SUM, kMachine, 4>(P, s);
+      if (kind == kMachine && cols == 2) return run_reduce<IN, CC_SUM, kMachine, 2>(P, s);
+      CC_KINDS(CC_SUM)
+    case CC_MAX: CC_KINDS(CC_MAX)
+    case CC_MIN: CC_KINDS(CC_MIN)
+    case CC_PROD: CC_KINDS(CC_PROD)
   }
+#undef CC_KINDS
   return cudaErrorInvalidValue;
 }
 
@@ -591,20 +635,23 @@ cudaError_t launch_reduce(const void* const* send, void* const* dst, int ndst, i
     P.per_node = root;
     hier_program(nranks, root, P.prog);
   }
-  // the ring, and a tree whose fold is a plain left fold (N <= 5), run the ring kernel
-  const bool ring = fold == kFoldRing || (fold == kFoldTree && program_is_linear(nranks, P.prog));
-  // several columns per thread pay off for the fold machine (tree, binomial) at small N;
-  // the ring's plain left fold is faster with one column and twice the resident CTAs
-  int cols = ring ? 1 : (nranks <= 2 ? 4 : (nranks <= 4 ? 2 : 1));
+  // the ring, and a tree whose fold is a plain left fold (N <= 5), run the linear fold; the
+  // hierarchical fold has its own nested loop; other trees and the binomial reduce run the
+  // fold machine
+  const int kind = (fold == kFoldRing || (fold == kFoldTree && program_is_linear(nranks, P.prog))) ? kLinear
+                   : fold == kFoldHier ? kHier : kMachine;
+  // several columns per thread pay off for the fold machine at small N; the linear fold is
+  // faster with one column and twice the resident CTAs
+  int cols = kind != kMachine ? 1 : (nranks <= 2 ? 4 : (nranks <= 4 ? 2 : 1));
   if (in_t == CC_BF16) cols = std::min(cols, 2);  // a bf16 column already holds 8 elements
-  if (!ring) {
+  if (kind == kMachine) {
     const int depth = program_depth(nranks, P.prog);
     if (depth > (cols == 4 ? 2 : cols == 2 ? 4 : kStackSlots)) cols = 1;
   }
   switch (in_t) {
-    case CC_F32: return dispatch_op<CC_F32>(P, op, ring, cols, stream);
-    case CC_BF16: return dispatch_op<CC_BF16>(P, op, ring, cols, stream);
-    case CC_I32: return dispatch_op<CC_I32>(P, op, ring, cols, stream);
+    case CC_F32: return dispatch_op<CC_F32>(P, op, kind, cols, stream);
+    case CC_BF16: return dispatch_op<CC_BF16>(P, op, kind, cols, stream);
+    case CC_I32: return dispatch_op<CC_I32>(P, op, kind, cols, stream);
   }
   return cudaErrorInvalidValue;
 }
