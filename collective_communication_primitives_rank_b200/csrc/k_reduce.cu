@@ -60,7 +60,7 @@ __device__ __forceinline__ V ring_fold(int n, int c, Load ld, Widen widen, bool 
   return acc;
 }
 
-// Fold machine (tree / binomial / hierarchical): position p holds rank rank_of(p).
+// Fold machine (tree / binomial): position p holds rank rank_of(p).
 template <int IN, int OP, typename V, typename X, int W, int S = kStackSlots, typename RankOf, typename Load,
           typename Widen>
 __device__ __forceinline__ V machine_fold(int n, const FoldProgram& prog, RankOf rank_of, Load ld, Widen widen) {
@@ -270,7 +270,6 @@ __global__ void __launch_bounds__(kThreads, KIND == kLinear ? CC_RING_MIN_BLOCKS
       const bool mirror = (P.fold == kFoldTree && g == 1);
       const int G = P.per_node, M = n / P.per_node, hc = g / M, hj = g % M;
       auto rank_of = [&](int p) {
-        if (P.fold == kFoldHier) return ((hj + p / G) % M) * G + (hc + p % G) % G;
         const int rk = P.prog.rmap[p];
         return mirror ? n - 1 - rk : rk;
       };
@@ -510,25 +509,6 @@ static void binomial_program(int n, int root, FoldProgram& fp) {
   }
 }
 
-// Hierarchical fold in machine codes: positions run node by node (G local ranks each); a
-// node's ranks are left-folded into cur; the first node's fold is pushed, each middle
-// node's is folded into it (top = top (+) cur), the last node's pops it (cur = top (+) cur).
-// The rank at each position depends on the element's group and is computed in the kernel.
-static void hier_program(int n, int G, FoldProgram& fp) {
-  const int M = n / G;
-  for (int p = 0; p < n; ++p) {
-    const int k = p / G, i = p % G;
-    uint8_t code = i > 0 ? kFoldCur : 0;
-    if (i == G - 1 && M > 1) {
-      if (k == 0) code |= kPush;
-      else if (k < M - 1) code |= kFoldTop;
-      else code |= (uint8_t)(1 << 2);  // one pop
-    }
-    fp.code[p] = code;
-    fp.rmap[p] = (uint8_t)p;
-  }
-}
-
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 int sm_count() {
@@ -631,10 +611,7 @@ cudaError_t launch_reduce(const void* const* send, void* const* dst, int ndst, i
   P.per_node = 1;
   if (fold == kFoldTree) tree_program(nranks, P.prog);
   else if (fold == kFoldBinomial) binomial_program(nranks, root, P.prog);
-  else if (fold == kFoldHier) {
-    P.per_node = root;
-    hier_program(nranks, root, P.prog);
-  }
+  else if (fold == kFoldHier) P.per_node = root;
   // the ring, and a tree whose fold is a plain left fold (N <= 5), run the linear fold; the
   // hierarchical fold has its own nested loop; other trees and the binomial reduce run the
   // fold machine
