@@ -11,7 +11,7 @@
 namespace cc {
 
 constexpr int kMaxRanks = CC_MAX_RANKS;
-constexpr int kStackSlots = 8;   // pending partials of a tree fold (depth <= 7 for N <= 64)
+constexpr int kStackSlots = 6;   // pending partials of a fold program (binomial N = 64 needs 6, trees <= 4)
 
 // ---- reduction operators (one binary32 / int32 operation, never contracted) ----------------
 
@@ -123,7 +123,7 @@ template <int IN> __device__ __forceinline__ void scale_unit(Unit<IN>& a, float 
 //   bit 5 FOLD_TOP : then top = top (+) cur
 // The double binary tree (in-order, ((S_left (+) x) (+) S_right)) uses FOLD_CUR / PUSH /
 // NPOP; the binomial reduce (x_v first, then each child's partial) uses PUSH / NPOP /
-// FOLD_TOP. The host builds the codes; a stack of at most 8 pending partials is kept in
+// FOLD_TOP. The host builds the codes; a stack of at most 6 pending partials is kept in
 // registers (each access is a warp-uniform switch, so nothing spills to local memory).
 
 constexpr uint8_t kFoldCur = 1, kPush = 2, kFoldTop = 32;
@@ -143,18 +143,6 @@ template <int IN, int OP> __device__ __forceinline__ void comb(typename Tr<IN>::
   a = op<IN, OP>(a, b);
 }
 
-// U units side by side (U columns of one thread), and U raw loads: small rank counts fold
-// several columns at once so that a thread still has about 8 loads in flight.
-template <int IN, int U> struct MU { Unit<IN> u[U]; };
-template <int U> struct MX { uint4 w[U]; };
-template <int IN, int OP, int U> __device__ __forceinline__ void comb(MU<IN, U>& a, const MU<IN, U>& b) {
-#pragma unroll
-  for (int k = 0; k < U; ++k) op_unit<IN, OP>(a.u[k], b.u[k]);
-}
-template <int IN, int OP, int U> __device__ __forceinline__ void comb(MU<IN, U>& a, const MX<U>& b) {
-#pragma unroll
-  for (int k = 0; k < U; ++k) op_unit<IN, OP>(a.u[k], to_unit<IN>(b.w[k]));
-}
 
 template <typename V, int S = kStackSlots> struct FoldStack {
   static_assert(S >= 1 && S <= 8, "1..8 stack slots");

@@ -33,6 +33,9 @@ constexpr int kThreads = 256;
 #ifndef CC_RING_MIN_BLOCKS
 #define CC_RING_MIN_BLOCKS 4  // resident 256-thread CTAs per SM the ring kernel is compiled for
 #endif
+#ifndef CC_SHALLOW_MIN_BLOCKS
+#define CC_SHALLOW_MIN_BLOCKS 3  // the same for the 2-slot fold machine
+#endif
 
 // ---- folds over the N ranks ---------------------------------------------------------------------
 
@@ -108,37 +111,32 @@ __device__ __forceinline__ V hier_fold(int n, int G, int c, int j, Load ld, Wide
   return outer;
 }
 
-// Pending-partial slots the fold machine needs with U columns per thread: U > 1 is only
-// used for N <= 8 / U ranks, whose trees need at most 2 (U = 4) or 3 (U = 2) slots.
-template <int U> constexpr int stack_slots() { return U == 1 ? kStackSlots : (U == 2 ? 4 : 2); }
 
 // Elements [a, b) of one fold group, spread over threads t = 0..T-1: 16-byte units where
-// every address is aligned, element-wise head and tail around them. Each thread folds U
-// units at once (units T apart, so warps stay coalesced) with windows of 8 / U positions:
-// about 8 loads in flight per thread for any rank count.
+// every address is aligned, element-wise head and tail around them. Each thread folds one
+// unit at a time (consecutive threads take consecutive units, so warps stay coalesced) with
+// windows of 8 positions: up to 8 loads in flight per thread.
 // KIND: kLinear (ring order or a linear tree), kMachine (tree / binomial programs),
-// kHier (two-level); hG / hc / hj describe the hierarchical group.
-constexpr int kLinear = 0, kMachine = 1, kHier = 2;
+// kHier (two-level), kShallow / kMid (the fold machine with 2 / 4 stack slots, for programs
+// that never hold more pending partials); hG / hc / hj describe the hierarchical group.
+constexpr int kLinear = 0, kMachine = 1, kHier = 2, kShallow = 3, kMid = 4;
 
-template <int IN, int OP, int KIND, int U, typename RankOf, typename Src, typename EmitU, typename EmitE>
+template <int IN, int OP, int KIND, typename RankOf, typename Src, typename EmitU, typename EmitE>
 __device__ __forceinline__ void reduce_range(int n, int g, RankOf rank_of, const FoldProgram& prog,
                                              uint64_t a, uint64_t b, uint64_t t, uint64_t T, bool vec,
                                              Src src, EmitU emit_unit, EmitE emit_elem,
-                                             bool linear_tree = false, int hG = 1, int hc = 0, int hj = 0) {
+                                             int start = 0, bool up = true, int hG = 1, int hc = 0, int hj = 0) {
   constexpr bool RING = KIND == kLinear;
+  constexpr int SLOTS = KIND == kShallow ? 2 : KIND == kMid ? 4 : kStackSlots;
   using A = typename Tr<IN>::Acc;
   constexpr int UE = Tr<IN>::UE;
-  constexpr int W = 8 / U;
   auto same = [](const A& x) { return x; };
-  // a RING fold starts at rank g and walks up; a linear tree fold (g = 0 or 1 for tree A / B)
-  // starts at rank 0 and walks up, or at rank n-1 and walks down
-  const int start = linear_tree ? (g == 0 ? 0 : n - 1) : g;
-  const bool up = !linear_tree || g == 0;
+  // a linear fold starts at rank `start` and walks up (or down) the ranks
   auto fold_elem = [&](uint64_t e) -> A {
     auto ld = [&](int r) { return load_elem<IN>(src(r) + e); };
     if constexpr (RING) return ring_fold<IN, OP, A, A>(n, start, ld, same, up);
     else if constexpr (KIND == kHier) return hier_fold<IN, OP, A, A>(n, hG, hc, hj, ld, same);
-    else return machine_fold<IN, OP, A, A, 8>(n, prog, rank_of, ld, same);
+    else return machine_fold<IN, OP, A, A, 8, SLOTS>(n, prog, rank_of, ld, same);
   };
   if (vec) {
     uint64_t va = (a + UE - 1) / UE * UE;
@@ -146,27 +144,14 @@ __device__ __forceinline__ void reduce_range(int n, int g, RankOf rank_of, const
     uint64_t vb = b / UE * UE;
     if (vb < va) vb = va;
     const uint64_t step = T * UE;
-    auto widen = [](const MX<U>& x) {
-      MU<IN, U> m;
-#pragma unroll
-      for (int k = 0; k < U; ++k) m.u[k] = to_unit<IN>(x.w[k]);
-      return m;
-    };
-    for (uint64_t e0 = va + t * UE; e0 < vb; e0 += step * U) {
-      auto ld = [&](int r) {
-        MX<U> x;
-#pragma unroll
-        for (int k = 0; k < U; ++k)
-          if (k == 0 || e0 + k * step < vb) x.w[k] = load_raw(src(r) + e0 + k * step);
-        return x;
-      };
-      MU<IN, U> m;
-      if constexpr (RING) m = ring_fold<IN, OP, MU<IN, U>, MX<U>, W>(n, start, ld, widen, up);
-      else if constexpr (KIND == kHier) m = hier_fold<IN, OP, MU<IN, U>, MX<U>>(n, hG, hc, hj, ld, widen);
-      else m = machine_fold<IN, OP, MU<IN, U>, MX<U>, W, stack_slots<U>()>(n, prog, rank_of, ld, widen);
-#pragma unroll
-      for (int k = 0; k < U; ++k)
-        if (k == 0 || e0 + k * step < vb) emit_unit(e0 + k * step, m.u[k]);
+    auto widen = [](const uint4& x) { return to_unit<IN>(x); };
+    for (uint64_t e0 = va + t * UE; e0 < vb; e0 += step) {
+      auto ld = [&](int r) { return load_raw(src(r) + e0); };
+      Unit<IN> m;
+      if constexpr (RING) m = ring_fold<IN, OP, Unit<IN>, uint4>(n, start, ld, widen, up);
+      else if constexpr (KIND == kHier) m = hier_fold<IN, OP, Unit<IN>, uint4>(n, hG, hc, hj, ld, widen);
+      else m = machine_fold<IN, OP, Unit<IN>, uint4, 8, SLOTS>(n, prog, rank_of, ld, widen);
+      emit_unit(e0, m);
     }
     const uint64_t nh = va - a, nt = b - vb;
     if (t < nh) emit_elem(a + t, fold_elem(a + t));
@@ -249,10 +234,11 @@ struct ReduceParams {
 // Each CTA folds contiguous tiles (normally exactly one: the grid is sized to the tile
 // count); a tile is split where it crosses a fold group (ring chunk or tree half) and each
 // piece is folded by the whole CTA.
-template <int IN, int OP, int KIND, int U>
-__global__ void __launch_bounds__(kThreads, KIND == kLinear ? CC_RING_MIN_BLOCKS : KIND == kHier ? 3 : 2)
+template <int IN, int OP, int KIND>
+__global__ void __launch_bounds__(kThreads, KIND == kLinear ? CC_RING_MIN_BLOCKS
+                                           : KIND == kHier ? 3
+                                           : KIND == kShallow || KIND == kMid ? CC_SHALLOW_MIN_BLOCKS : 2)
     reduce_kernel(const __grid_constant__ ReduceParams P) {
-  constexpr bool RING = KIND == kLinear;
   using In = typename Tr<IN>::In;
   using Out = typename Tr<IN>::Out;
   using A = typename Tr<IN>::Acc;
@@ -295,8 +281,13 @@ __global__ void __launch_bounds__(kThreads, KIND == kLinear ? CC_RING_MIN_BLOCKS
           store_elem<IN>(static_cast<Out*>(P.dst[0]) + e, v);
         }
       };
-      reduce_range<IN, OP, KIND, U>(n, g, rank_of, P.prog, s, se, threadIdx.x, blockDim.x, P.vec != 0, src,
-                                    emit_unit, emit_elem, RING && P.fold == kFoldTree, G, hc, hj);
+      // linear folds: a ring chunk starts at rank g and walks up; a linear tree (g = 0 or 1
+      // for tree A / B) starts at rank 0 and walks up, or at rank n-1 and walks down; a
+      // linear binomial program starts at the root and walks up
+      const int lstart = P.fold == kFoldRing ? g : P.fold == kFoldTree ? (g == 0 ? 0 : n - 1) : P.prog.rmap[0];
+      const bool lup = P.fold != kFoldTree || g == 0;
+      reduce_range<IN, OP, KIND>(n, g, rank_of, P.prog, s, se, threadIdx.x, blockDim.x, P.vec != 0, src,
+                                    emit_unit, emit_elem, lstart, lup, G, hc, hj);
       s = se;
     }
   }
@@ -312,10 +303,10 @@ __global__ void __launch_bounds__(kThreads, KIND == kLinear ? CC_RING_MIN_BLOCKS
 // buffer: N·G bytes in, N·G bytes out.
 
 #ifndef CC_BUCKET_TILE
-#define CC_BUCKET_TILE 8192        // elements per tile
+#define CC_BUCKET_TILE 1024        // elements per tile (one 16-byte unit per thread)
 #endif
 #ifndef CC_BUCKET_MIN_BLOCKS
-#define CC_BUCKET_MIN_BLOCKS 3     // resident 256-thread CTAs per SM the ring variant is compiled for
+#define CC_BUCKET_MIN_BLOCKS 4     // resident 256-thread CTAs per SM the ring variant is compiled for
 #endif
 #ifndef CC_BUCKET_OVERSUB
 #define CC_BUCKET_OVERSUB 1024     // grid = tiles, capped at this many times the resident CTAs
@@ -403,8 +394,8 @@ __global__ void __launch_bounds__(kThreads, RING ? CC_BUCKET_MIN_BLOCKS : 2) buc
         const int rk = P.prog.rmap[p];
         return mirror ? n - 1 - rk : rk;
       };
-      reduce_range<IN, OP, RING ? kLinear : kMachine, 1>(n, g, rank_of, P.prog, s, se, threadIdx.x, blockDim.x,
-                                                         P.vec != 0, src, emit_unit, emit_elem);
+      reduce_range<IN, OP, RING ? kLinear : kMachine>(n, g, rank_of, P.prog, s, se, threadIdx.x, blockDim.x,
+                                                         P.vec != 0, src, emit_unit, emit_elem, g, true);
       s = se;
     }
     __syncthreads();  // every thread is done with s_in / s_out before the next tile restages them
@@ -461,10 +452,14 @@ static void tree_program(int n, FoldProgram& fp) {
   }
 }
 
-// A program without pushes, pops or fold-into-top is a left fold in position order.
-static bool program_is_linear(int n, const FoldProgram& fp) {
-  for (int p = 0; p < n; ++p)
+// A program without pushes, pops or fold-into-top is a left fold in position order; it
+// runs as the linear fold when its positions walk the ranks upwards from rmap[0] (tree A
+// folds ranks 0, 1, ..., n-1; tree B is its mirror; a binomial program from its root).
+static bool program_is_rotation(int n, const FoldProgram& fp) {
+  for (int p = 0; p < n; ++p) {
     if ((fp.code[p] & (kPush | kFoldTop)) || npop_of(fp.code[p])) return false;
+    if (fp.rmap[p] != (fp.rmap[0] + p) % n) return false;
+  }
   return true;
 }
 
@@ -532,43 +527,47 @@ static int blocks_per_sm(K kernel) {
   return b;
 }
 
-template <int IN, int OP, int KIND, int U>
+template <int IN, int OP, int KIND>
 static cudaError_t run_reduce(ReduceParams& P, cudaStream_t s) {
-  auto k = reduce_kernel<IN, OP, KIND, U>;
+  auto k = reduce_kernel<IN, OP, KIND>;
   static const int bps = blocks_per_sm(k);
-  constexpr uint64_t UE = Tr<IN>::UE * U;
+  constexpr uint64_t UE = Tr<IN>::UE;
   const uint64_t resident = (uint64_t)sm_count() * bps;
-  // tiles of 1..8 units per thread: large buffers get 8 (long contiguous streams per CTA),
-  // small ones shrink the tile so that every resident CTA still gets work
-  const uint64_t units = (P.count + UE - 1) / UE;
-  uint64_t upt = units / (resident * kThreads);
-  upt = std::max<uint64_t>(1, std::min<uint64_t>(8, upt));
-  P.tile = upt * kThreads * UE;
   // a tile never spans much more than one fold group, so that the groups of a small
   // buffer (N ring chunks of a few elements each) are folded by different CTAs in parallel
   const uint64_t ngroups = P.fold == kFoldRing ? (uint64_t)P.nranks
                            : P.fold == kFoldTree ? 2
                            : P.fold == kFoldHier ? (uint64_t)P.nranks : 1;
   const uint64_t per_group = ((P.count + ngroups - 1) / ngroups + 7) / 8 * 8;
-  P.tile = std::max<uint64_t>(8, std::min<uint64_t>(P.tile, per_group));
+  // units per thread and tile (measured): the linear folds (ring, linear tree, hierarchical)
+  // run best with about 24 memory operations per thread and CTA (a unit costs N loads plus
+  // N stores for allreduce, one store otherwise), the small-stack tree machines with 16 / N
+  // units, the binomial and deep-stack machines with 8: many short-lived CTAs keep more
+  // loads in flight than long per-CTA streams. Small buffers take fewer, so that every
+  // resident CTA gets a tile.
+  const int ops = P.mode == kAllReduce ? 2 * P.nranks : P.nranks + 1;
+  const uint64_t target = (KIND == kMachine || P.fold == kFoldBinomial) ? 8
+                          : (KIND == kLinear || KIND == kHier) ? (uint64_t)std::max(1, std::min(8, 24 / ops))
+                          : (uint64_t)std::max(1, std::min(8, 16 / P.nranks));
+  const uint64_t units = (P.count + UE - 1) / UE;
+  const uint64_t upt = std::max<uint64_t>(1, std::min<uint64_t>(target, units / (resident * kThreads)));
+  P.tile = std::max<uint64_t>(8, std::min<uint64_t>(upt * kThreads * UE, per_group));
   const uint64_t ntiles = (P.count + P.tile - 1) / P.tile;
   const uint64_t grid = std::max<uint64_t>(1, std::min<uint64_t>(ntiles, CC_REDUCE_OVERSUB * resident));
   k<<<(unsigned)grid, kThreads, 0, s>>>(P);
   return cudaGetLastError();
 }
 
-// Columns per thread for SUM (the other operators fold one column).
 template <int IN>
-static cudaError_t dispatch_op(ReduceParams& P, cc_op op, int kind, int cols, cudaStream_t s) {
+static cudaError_t dispatch_op(ReduceParams& P, cc_op op, int kind, cudaStream_t s) {
 #define CC_KINDS(OPV)                                                                         \
-  if (kind == kLinear) return run_reduce<IN, OPV, kLinear, 1>(P, s);                         \
-  if (kind == kHier) return run_reduce<IN, OPV, kHier, 1>(P, s);                             \
-  return run_reduce<IN, OPV, kMachine, 1>(P, s);
+  if (kind == kLinear) return run_reduce<IN, OPV, kLinear>(P, s);                         \
+  if (kind == kHier) return run_reduce<IN, OPV, kHier>(P, s);                             \
+  if (kind == kShallow) return run_reduce<IN, OPV, kShallow>(P, s);                       \
+  if (kind == kMid) return run_reduce<IN, OPV, kMid>(P, s);                               \
+  return run_reduce<IN, OPV, kMachine>(P, s);
   switch (op) {
-    case CC_SUM:
-      if (kind == kMachine && cols == 4) return run_reduce<IN, CC_SUM, kMachine, 4>(P, s);
-      if (kind == kMachine && cols == 2) return run_reduce<IN, CC_SUM, kMachine, 2>(P, s);
-      CC_KINDS(CC_SUM)
+    case CC_SUM: CC_KINDS(CC_SUM)
     case CC_MAX: CC_KINDS(CC_MAX)
     case CC_MIN: CC_KINDS(CC_MIN)
     case CC_PROD: CC_KINDS(CC_PROD)
@@ -612,23 +611,22 @@ cudaError_t launch_reduce(const void* const* send, void* const* dst, int ndst, i
   if (fold == kFoldTree) tree_program(nranks, P.prog);
   else if (fold == kFoldBinomial) binomial_program(nranks, root, P.prog);
   else if (fold == kFoldHier) P.per_node = root;
-  // the ring, and a tree whose fold is a plain left fold (N <= 5), run the linear fold; the
-  // hierarchical fold has its own nested loop; other trees and the binomial reduce run the
-  // fold machine
-  const int kind = (fold == kFoldRing || (fold == kFoldTree && program_is_linear(nranks, P.prog))) ? kLinear
-                   : fold == kFoldHier ? kHier : kMachine;
-  // several columns per thread pay off for the fold machine at small N; the linear fold is
-  // faster with one column and twice the resident CTAs
-  int cols = kind != kMachine ? 1 : (nranks <= 2 ? 4 : (nranks <= 4 ? 2 : 1));
-  if (in_t == CC_BF16) cols = std::min(cols, 2);  // a bf16 column already holds 8 elements
-  if (kind == kMachine) {
+  // the ring, a tree whose fold is a plain left fold (N <= 5) and a binomial program that is
+  // one (N <= 3, ranks in order from the root) run the linear fold; the hierarchical fold has
+  // its own nested loop; other programs run the fold machine with the smallest stack that
+  // holds their pending partials (more resident CTAs for smaller stacks)
+  int kind = kMachine;
+  if (fold == kFoldRing || fold == kFoldHier) kind = fold == kFoldRing ? kLinear : kHier;
+  else if (program_is_rotation(nranks, P.prog)) kind = kLinear;
+  else {
     const int depth = program_depth(nranks, P.prog);
-    if (depth > (cols == 4 ? 2 : cols == 2 ? 4 : kStackSlots)) cols = 1;
+    if (depth > kStackSlots) return cudaErrorInvalidValue;  // not reached for N <= 64
+    kind = depth <= 2 ? kShallow : depth <= 4 ? kMid : kMachine;
   }
   switch (in_t) {
-    case CC_F32: return dispatch_op<CC_F32>(P, op, kind, cols, stream);
-    case CC_BF16: return dispatch_op<CC_BF16>(P, op, kind, cols, stream);
-    case CC_I32: return dispatch_op<CC_I32>(P, op, kind, cols, stream);
+    case CC_F32: return dispatch_op<CC_F32>(P, op, kind, stream);
+    case CC_BF16: return dispatch_op<CC_BF16>(P, op, kind, stream);
+    case CC_I32: return dispatch_op<CC_I32>(P, op, kind, stream);
   }
   return cudaErrorInvalidValue;
 }

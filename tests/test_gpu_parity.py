@@ -189,8 +189,10 @@ def test_broadcast(n, root, count):
         out[r].check()
 
 
-@pytest.mark.parametrize("n,root", [(1, 0), (4, 0), (8, 5), (13, 12), (64, 17)])
-@pytest.mark.parametrize("kind", ["spread", "i32"])
+# N = 2, 3: the binomial program is a left fold from the root (linear kernel); N = 4..31:
+# small-stack machines; N = 32, 64: the deep machine
+@pytest.mark.parametrize("n,root", [(1, 0), (2, 1), (3, 2), (4, 0), (8, 5), (13, 12), (32, 31), (64, 17)])
+@pytest.mark.parametrize("kind", ["spread", "i32", "bf16"])
 def test_reduce_to_root(n, root, kind):
     count = 2049
     xs = _inputs(kind, n, count, seed=12)
