@@ -284,8 +284,9 @@ __global__ void __launch_bounds__(256) a2a_copy_kernel(const __grid_constant__ A
     ok[k] = pos < P.capacity;
     ptr[k] = (P.direction == 0 ? P.recv[d] : const_cast<char*>(P.send[d])) + pos * P.row_bytes;
   }
-  // 8 loads per lane in flight before the stores that consume them
-  constexpr int B = 8;
+  // 16 loads per lane in flight before the stores that consume them (a whole 8 KiB row per
+  // warp; measured faster than 8 or 32)
+  constexpr int B = 16;
   const uint64_t nvec = P.row_bytes / 16;
   if (P.direction == 0) {
     const uint4* src = reinterpret_cast<const uint4*>(P.send[s] + (uint64_t)t * P.row_bytes);
