@@ -57,6 +57,13 @@ _SIGS = {
     "cc_bucket_allreduce": (_i, [_PP, _PP, _i, _i, _SZP, _sz, _i, _f, _vp]),
     "cc_bucket_allreduce_host": (_i, [_PP, _PP, _PP, _PP, _i, _i, _SZP, _sz, _i, _f, _vp]),
     "cc_bucket_allreduce_buckets": (_i, [_PP, _PP, _i, _i, _SZP, _sz, _i, _i, _i, _f, _vp]),
+    "cc_allreduce_slice": (_i, [_PP, _PP, _i, _i, _sz, _i, _i, _i, _i, _f, _vp]),
+    "cc_reduce_scatter_slice": (_i, [_PP, _vp, _i, _i, _sz, _i, _i, _i, _f, _vp]),
+    "cc_allgather_slice": (_i, [_vp, _PP, _i, _i, _sz, _i, _vp]),
+    "cc_ipc_handle_bytes": (_sz, []),
+    "cc_ipc_export": (_i, [_vp, ctypes.c_char_p, _SZP]),
+    "cc_ipc_open": (_i, [ctypes.c_char_p, _sz, _PP]),
+    "cc_ipc_close": (_i, [_vp]),
 }
 
 
@@ -465,6 +472,141 @@ def cc_bucket_allreduce_host(host_grads, host_out, dev_grads, dev_out, *, cap_by
                                         _ptrs([t for row in dev_out for t in row]), n, nt,
                                         _sizes([t.numel() for t in host_grads[0]]), cap_bytes, _ALGOS[algo],
                                         float(scale), _stream(stream)), "cc_bucket_allreduce_host")
+
+
+# ---- one rank per process: slices over peer-mapped buffers -----------------------------------
+
+class PeerGroup:
+    """Every rank's copy of some device tensors, mapped into this process.
+
+    Each process of the torch.distributed group `group` (one per GPU; any backend) passes its
+    own tensors, in the same order and of the same sizes on every rank. Their CUDA IPC
+    handles are exchanged over the group, and the other ranks' allocations are opened with
+    cc_ipc_open. buffers(i) is the list of the N ranks' copies of tensor i: this rank's
+    tensor at its own index, device pointers (ints) of the peers' elsewhere, which the slice
+    calls take. close() unmaps the peers; the tensors must stay alive until every rank has
+    closed its group."""
+
+    def __init__(self, tensors, group=None):
+        dist = _torch().distributed
+        self.rank = dist.get_rank(group)
+        self.nranks = dist.get_world_size(group)
+        self._tensors = list(tensors)
+        hb = int(lib.cc_ipc_handle_bytes())
+        mine = []
+        for t in self._tensors:
+            h = ctypes.create_string_buffer(hb)
+            off = ctypes.c_size_t()
+            _check(lib.cc_ipc_export(_dev_ptr(t), h, ctypes.byref(off)), "cc_ipc_export")
+            mine.append((h.raw, off.value, t.numel(), str(t.dtype)))
+        every = [None] * self.nranks
+        dist.all_gather_object(every, mine, group=group)
+        self._opened = []
+        self._bufs = []
+        try:
+            for i, t in enumerate(self._tensors):
+                row = []
+                for r in range(self.nranks):
+                    if r == self.rank:
+                        row.append(t)
+                        continue
+                    h, off, numel, dt = every[r][i]
+                    if numel != t.numel() or dt != str(t.dtype):
+                        raise ValueError(f"PeerGroup: tensor {i} differs on rank {r} ({numel} x {dt})")
+                    p = ctypes.c_void_p()
+                    _check(lib.cc_ipc_open(h, off, ctypes.byref(p)), "cc_ipc_open")
+                    self._opened.append(p.value)
+                    row.append(p.value)
+                self._bufs.append(row)
+        except Exception:
+            self.close()
+            raise
+
+    def buffers(self, i: int) -> list:
+        return list(self._bufs[i])
+
+    def close(self) -> None:
+        while self._opened:
+            lib.cc_ipc_close(self._opened.pop())
+
+
+def _slice_ptrs(bufs, rank: int, what: str):
+    """(pointer array, this rank's tensor) of N buffers: tensors of this process or peer
+    device pointers (ints); the entry at `rank` must be a tensor."""
+    torch = _torch()
+    n = _ranks(bufs, what)
+    if not 0 <= rank < n:
+        raise ValueError(f"{what}: rank {rank} outside 0..{n - 1}")
+    own = bufs[rank]
+    if not isinstance(own, torch.Tensor):
+        raise ValueError(f"{what}: entry {rank} (this rank) must be a tensor")
+    vals = []
+    for b in bufs:
+        if isinstance(b, torch.Tensor):
+            if b.numel() != own.numel() or b.dtype != own.dtype:
+                raise ValueError(f"{what}: every buffer must have {own.numel()} elements of {own.dtype}")
+            vals.append(_dev_ptr(b))
+        else:
+            vals.append(int(b))
+    return (ctypes.c_void_p * n)(*vals), own
+
+
+def cc_allreduce_slice(send, recv, rank: int, *, op="sum", algo="ring", scale=1.0, stream=None) -> None:
+    """Rank `rank`'s share of cc_allreduce over N ranks' buffers (see PeerGroup): folds chunk
+    `rank` from every send buffer and writes it into every recv buffer. After all N ranks
+    have run it (ordered by the caller's barriers), every recv equals cc_allreduce's."""
+    sp, s0 = _slice_ptrs(send, rank, "cc_allreduce_slice send")
+    rp, r0 = _slice_ptrs(recv, rank, "cc_allreduce_slice recv")
+    if len(recv) != len(send) or r0.numel() != s0.numel():
+        raise ValueError("cc_allreduce_slice: one output per rank, as long as the input")
+    _check(lib.cc_allreduce_slice(sp, rp, len(send), rank, s0.numel(), dtype_code(s0), dtype_code(r0), _OPS[op],
+                                  _ALGOS[algo], float(scale), _stream(stream)), "cc_allreduce_slice")
+
+
+def cc_reduce_scatter_slice(send, shard, rank: int, *, op="sum", scale=1.0, stream=None) -> None:
+    """Rank `rank`'s share of cc_reduce_scatter: folds chunk `rank` of every send buffer into
+    this rank's shard (a tensor of this process)."""
+    sp, s0 = _slice_ptrs(send, rank, "cc_reduce_scatter_slice send")
+    n = len(send)
+    _same([shard], cc_chunk(s0.numel(), n, rank)[1], shard.dtype, "cc_reduce_scatter_slice shard")
+    _check(lib.cc_reduce_scatter_slice(sp, _dev_ptr(shard), n, rank, s0.numel(), dtype_code(s0),
+                                       dtype_code(shard), _OPS[op], float(scale), _stream(stream)),
+           "cc_reduce_scatter_slice")
+
+
+def cc_allgather_slice(shard, recv, rank: int, *, stream=None) -> None:
+    """Rank `rank`'s share of cc_allgather: copies this rank's shard into chunk `rank` of
+    every recv buffer."""
+    rp, r0 = _slice_ptrs(recv, rank, "cc_allgather_slice recv")
+    n = len(recv)
+    _same([shard], cc_chunk(r0.numel(), n, rank)[1], r0.dtype, "cc_allgather_slice shard")
+    _check(lib.cc_allgather_slice(_dev_ptr(shard), rp, n, rank, r0.numel(), dtype_code(r0), _stream(stream)),
+           "cc_allgather_slice")
+
+
+class PeerAllreduce:
+    """Allreduce of one tensor per process across a torch.distributed group, one pass over
+    NVLink: each rank folds its own chunk from all peers' inputs and writes it into all
+    peers' outputs (cc_allreduce_slice). run() orders the ranks with a stream
+    synchronisation and a group barrier before and after the slice."""
+
+    def __init__(self, send, recv, group=None, *, op="sum", algo="ring", scale=1.0):
+        self.group = group
+        self.peers = PeerGroup([send, recv], group)
+        self.op, self.algo, self.scale = op, algo, scale
+
+    def run(self, stream=None) -> None:
+        torch = _torch()
+        s = stream if stream is not None else torch.cuda.current_stream()
+        s.synchronize()
+        torch.distributed.barrier(group=self.group)
+        cc_allreduce_slice(self.peers.buffers(0), self.peers.buffers(1), self.peers.rank, op=self.op,
+                           algo=self.algo, scale=self.scale, stream=s)
+        s.synchronize()
+        torch.distributed.barrier(group=self.group)
+
+    def close(self) -> None:
+        self.peers.close()
 
 
 def raw_call(name: str, *args) -> int:

@@ -552,4 +552,53 @@ cc_status cc_bucket_allreduce_host(const void* const* host_grads, void* const* h
                                                 as_stream(stream)));
 }
 
+// ---- one rank's slice (ranks in separate processes) -------------------------------------
+
+cc_status cc_allreduce_slice(const void* const* send, void* const* recv, int nranks, int rank, size_t count,
+                             cc_dtype in_t, cc_dtype out_t, cc_op op, cc_algo algo, float scale, void* stream) {
+  if (!valid_ranks(nranks) || !send || !recv || rank < 0 || rank >= nranks) return CC_ERR_INVALID_ARG;
+  if (cc_status st = check_reduce(in_t, out_t, op, scale)) return st;
+  if (algo != CC_ALGO_RING && algo != CC_ALGO_TREE) return CC_ERR_INVALID_ARG;
+  if (count == 0) return CC_OK;
+  if (!all_nonnull(send, nranks) || !all_nonnull((const void* const*)recv, nranks)) return CC_ERR_INVALID_ARG;
+  for (int r = 0; r < nranks; ++r)
+    if (recv[r] == send[r] && dtype_bytes(in_t) != dtype_bytes(out_t)) return CC_ERR_INVALID_ARG;
+  size_t a, len;
+  chunk_bounds(count, nranks, rank, a, len);
+  if (len == 0) return CC_OK;
+  return cuda_status(launch_reduce(send, recv, nranks, nranks, count, in_t, op,
+                                   algo == CC_ALGO_RING ? kFoldRing : kFoldTree, kAllReduce, 0, scale,
+                                   as_stream(stream), a, a + len));
+}
+
+cc_status cc_reduce_scatter_slice(const void* const* send, void* recv_shard, int nranks, int rank, size_t count,
+                                  cc_dtype in_t, cc_dtype out_t, cc_op op, float scale, void* stream) {
+  if (!valid_ranks(nranks) || !send || rank < 0 || rank >= nranks) return CC_ERR_INVALID_ARG;
+  if (cc_status st = check_reduce(in_t, out_t, op, scale)) return st;
+  if (count == 0) return CC_OK;
+  if (!all_nonnull(send, nranks)) return CC_ERR_INVALID_ARG;
+  size_t a, len;
+  chunk_bounds(count, nranks, rank, a, len);
+  if (len == 0) return CC_OK;
+  if (!recv_shard) return CC_ERR_INVALID_ARG;
+  // the reduce-scatter kernel writes chunk c to dst[c]; only chunk `rank` is folded here
+  std::vector<void*> dst(nranks, nullptr);
+  dst[rank] = recv_shard;
+  return cuda_status(launch_reduce(send, dst.data(), nranks, nranks, count, in_t, op, kFoldRing, kReduceScatter, 0,
+                                   scale, as_stream(stream), a, a + len));
+}
+
+cc_status cc_allgather_slice(const void* send_shard, void* const* recv, int nranks, int rank, size_t count,
+                             cc_dtype dtype, void* stream) {
+  if (!valid_ranks(nranks) || !recv || !valid_dtype(dtype) || rank < 0 || rank >= nranks) return CC_ERR_INVALID_ARG;
+  if (count == 0) return CC_OK;
+  if (!all_nonnull((const void* const*)recv, nranks)) return CC_ERR_INVALID_ARG;
+  size_t a, len;
+  chunk_bounds(count, nranks, rank, a, len);
+  if (len == 0) return CC_OK;
+  if (!send_shard) return CC_ERR_INVALID_ARG;
+  CopyEntry e{send_shard, nullptr, len, a};
+  return cuda_status(launch_copy(&e, 1, recv, nranks, true, -1, dtype_bytes(dtype), as_stream(stream), true));
+}
+
 }  // extern "C"

@@ -14,10 +14,12 @@ namespace cc {
 enum ReduceMode { kAllReduce = 0, kReduceScatter = 1, kReduceRoot = 2 };
 enum FoldKind { kFoldRing = 0, kFoldTree = 1, kFoldBinomial = 2, kFoldHier = 3 };
 
-// `root` is the root rank for kFoldBinomial and the ranks per node for kFoldHier.
+// `root` is the root rank for kFoldBinomial and the ranks per node for kFoldHier; only the
+// elements [lo, hi) of the count are folded and written (the whole buffer by default).
 cudaError_t launch_reduce(const void* const* send, void* const* dst, int ndst, int nranks,
                           size_t count, cc_dtype in_t, cc_op op, FoldKind fold, ReduceMode mode,
-                          int root, float scale, cudaStream_t stream);
+                          int root, float scale, cudaStream_t stream, size_t lo = 0,
+                          size_t hi = ~(size_t)0);
 
 // Fused DDP bucket allreduce over a tensor group (tables fit one launch).
 struct BucketTensorDesc {
@@ -33,7 +35,8 @@ cudaError_t launch_bucket_allreduce(const void* const* grads, void* const* out, 
                                     cudaStream_t stream);
 
 // Copies with fan-out: entry k copies numel[k] elements from src[k] either to every
-// dst_base[r] + dst_off[k] (fanout = true, r != skip) or to dst[k] + dst_off[k].
+// dst_base[r] + dst_off[k] (fanout = true, r != skip) or to dst[k] + dst_off[k]. `plain`
+// keeps to ordinary loads and stores (no bulk copies), for destinations in peer memory.
 struct CopyEntry {
   const void* src;
   void* dst;          // fanout == false
@@ -41,7 +44,7 @@ struct CopyEntry {
   uint64_t dst_off;   // elements
 };
 cudaError_t launch_copy(const CopyEntry* entries, int nentries, void* const* dst_base, int ndst,
-                        bool fanout, int skip, size_t elem_bytes, cudaStream_t stream);
+                        bool fanout, int skip, size_t elem_bytes, cudaStream_t stream, bool plain = false);
 
 // Device status word of the bounded waits (CC_OK or CC_ERR_TIMEOUT), read with a
 // stream synchronisation; `reset` clears it afterwards.

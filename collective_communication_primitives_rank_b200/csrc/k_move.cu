@@ -211,7 +211,7 @@ cudaError_t read_async_status(int* out, bool reset, cudaStream_t stream) {
 }
 
 cudaError_t launch_copy(const CopyEntry* entries, int nentries, void* const* dst_base, int ndst, bool fanout,
-                        int skip, size_t elem_bytes, cudaStream_t stream) {
+                        int skip, size_t elem_bytes, cudaStream_t stream, bool plain) {
   static int bps = 0;
   if (!bps && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, copy_kernel, kCopyThreads, 0) != cudaSuccess || bps <= 0))
     bps = 4;
@@ -250,7 +250,7 @@ cudaError_t launch_copy(const CopyEntry* entries, int nentries, void* const* dst
     if (tiles == 0) continue;
     bool all_vec = true;
     for (int k = 0; k < m; ++k) all_vec = all_vec && ((P.vec_mask[k >> 6] >> (k & 63)) & 1);
-    if (all_vec && bulk_attr == cudaSuccess) {
+    if (all_vec && !plain && bulk_attr == cudaSuccess) {
       // retile for the bulk kernel: kBulkTile-byte tiles, one CTA each
       uint32_t bt = 0;
       for (int k = 0; k < m; ++k) {

@@ -220,6 +220,7 @@ struct ReduceParams {
   void* dst[kMaxRanks];
   FoldProgram prog;
   uint64_t count;
+  uint64_t lo, hi;       // the elements this launch folds: [lo, hi) of the count
   uint64_t tile;         // elements per tile (a multiple of 8)
   uint64_t dst_aligned;  // bit r: dst[r] is 16-byte aligned
   int nranks;
@@ -244,10 +245,10 @@ __global__ void __launch_bounds__(kThreads, KIND == kLinear ? CC_RING_MIN_BLOCKS
   using A = typename Tr<IN>::Acc;
   const int n = P.nranks;
   const int mode = P.mode;
-  const uint64_t ntiles = (P.count + P.tile - 1) / P.tile;
+  const uint64_t ntiles = (P.hi - P.lo + P.tile - 1) / P.tile;
   auto src = [&](int r) { return static_cast<const In*>(P.src[r]); };
   for (uint64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    const uint64_t ea = tile * P.tile, eb = min(ea + P.tile, P.count);
+    const uint64_t ea = P.lo + tile * P.tile, eb = min(ea + P.tile, P.hi);
     uint64_t s = ea;
     while (s < eb) {
       uint64_t ga, gb;
@@ -549,10 +550,10 @@ static cudaError_t run_reduce(ReduceParams& P, cudaStream_t s) {
   const uint64_t target = (KIND == kMachine || P.fold == kFoldBinomial) ? 8
                           : (KIND == kLinear || KIND == kHier) ? (uint64_t)std::max(1, std::min(8, 24 / ops))
                           : (uint64_t)std::max(1, std::min(8, 16 / P.nranks));
-  const uint64_t units = (P.count + UE - 1) / UE;
+  const uint64_t units = (P.hi - P.lo + UE - 1) / UE;
   const uint64_t upt = std::max<uint64_t>(1, std::min<uint64_t>(target, units / (resident * kThreads)));
   P.tile = std::max<uint64_t>(8, std::min<uint64_t>(upt * kThreads * UE, per_group));
-  const uint64_t ntiles = (P.count + P.tile - 1) / P.tile;
+  const uint64_t ntiles = (P.hi - P.lo + P.tile - 1) / P.tile;
   const uint64_t grid = std::max<uint64_t>(1, std::min<uint64_t>(ntiles, CC_REDUCE_OVERSUB * resident));
   k<<<(unsigned)grid, kThreads, 0, s>>>(P);
   return cudaGetLastError();
@@ -588,9 +589,12 @@ static int program_depth(int n, const FoldProgram& fp) {
 
 cudaError_t launch_reduce(const void* const* send, void* const* dst, int ndst, int nranks, size_t count,
                           cc_dtype in_t, cc_op op, FoldKind fold, ReduceMode mode, int root, float scale,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, size_t lo, size_t hi) {
   ReduceParams P{};
   P.count = count;
+  P.hi = std::min<uint64_t>(hi, count);
+  P.lo = std::min<uint64_t>(lo, P.hi);
+  if (P.lo == P.hi) return cudaSuccess;
   P.nranks = nranks;
   P.mode = mode;
   P.fold = fold;

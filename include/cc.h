@@ -273,6 +273,55 @@ CC_API cc_status cc_bucket_allreduce_host(const void* const* host_grads, void* c
                                           int ntensors, const size_t* numels, size_t cap_bytes,
                                           cc_algo algo, float scale, void* stream);
 
+/* ---- One rank's slice, for ranks in separate processes (one per GPU) ----------------------
+ * The same schedules with the N ranks' buffers on N GPUs, one process each: every rank's
+ * buffers are mapped into each process (cc_ipc_open of the other processes' exports, or
+ * plain device pointers for this process's own), and rank `rank` does only its own share
+ * of the single-GPU call, loading peer inputs and storing into peer outputs directly over
+ * NVLink with ordinary loads and stores (no bulk or multicast copy touches peer memory).
+ * This is the ring's ownership split (lecture 09 §4.2-4.3: after the reduce-scatter, rank
+ * c holds the full sum of chunk c; the allgather then hands that chunk to everyone) run as
+ * one pass: rank c folds chunk c (chunk rule) from all N inputs and writes it to all N
+ * outputs, so the whole exchange is one fold per element and every byte crosses NVLink
+ * once each way.
+ * The caller orders the ranks: every input written (and every output no longer read)
+ * before any rank starts, and no output read before every rank has finished, e.g. a
+ * stream synchronisation plus a process-group barrier on both sides. Once all N ranks
+ * have made the call, the outputs hold exactly what the single-process call writes, bit
+ * for bit. `rank` outside [0, nranks) is CC_ERR_INVALID_ARG; other arguments, layouts and
+ * errors as the single-process call. */
+
+/* Allreduce: rank `rank` folds the elements of chunk `rank` (in the ring order of the
+ * chunk for CC_ALGO_RING, in the tree order of the half each element falls in for
+ * CC_ALGO_TREE) and writes them, scaled, into all N recv buffers. In-place allowed. */
+CC_API cc_status cc_allreduce_slice(const void* const* send, void* const* recv, int nranks, int rank,
+                                    size_t count, cc_dtype in_t, cc_dtype out_t, cc_op op, cc_algo algo,
+                                    float scale, void* stream);
+
+/* Reduce-scatter (ring order): rank `rank` folds chunk `rank` of all N send buffers into
+ * its own shard recv_shard (chunk `rank`'s length; may be NULL when that is 0). */
+CC_API cc_status cc_reduce_scatter_slice(const void* const* send, void* recv_shard, int nranks, int rank,
+                                         size_t count, cc_dtype in_t, cc_dtype out_t, cc_op op, float scale,
+                                         void* stream);
+
+/* Allgather: rank `rank` copies its shard (chunk `rank` of the count) into that chunk of
+ * all N recv buffers. */
+CC_API cc_status cc_allgather_slice(const void* send_shard, void* const* recv, int nranks, int rank,
+                                    size_t count, cc_dtype dtype, void* stream);
+
+/* CUDA IPC for the slice calls. cc_ipc_export writes an opaque handle (cc_ipc_handle_bytes()
+ * bytes, caller-owned) for the device allocation that holds dev_ptr, and the byte offset of
+ * dev_ptr inside it; any other process on the node passes both to cc_ipc_open to get a
+ * pointer to the same bytes (peer access is enabled on first use). Opening the same
+ * allocation several times in a process maps it once (reference-counted); cc_ipc_close
+ * undoes one cc_ipc_open. The exporting process must keep the allocation alive until every
+ * importer has closed it. Opening a handle in the process that exported it is
+ * CC_ERR_CUDA (use the local pointer). */
+CC_API size_t cc_ipc_handle_bytes(void);
+CC_API cc_status cc_ipc_export(const void* dev_ptr, void* handle, size_t* offset);
+CC_API cc_status cc_ipc_open(const void* handle, size_t offset, void** dev_ptr);
+CC_API cc_status cc_ipc_close(void* dev_ptr);
+
 #ifdef __cplusplus
 }
 #endif
