@@ -31,10 +31,10 @@ constexpr int kThreads = 256;
 #define CC_REDUCE_OVERSUB 1024
 #endif
 #ifndef CC_RING_MIN_BLOCKS
-#define CC_RING_MIN_BLOCKS 4  // resident 256-thread CTAs per SM the ring kernel is compiled for
+#define CC_RING_MIN_BLOCKS 4  // resident 256-thread CTAs per SM the linear-fold kernel is compiled for
 #endif
 #ifndef CC_SHALLOW_MIN_BLOCKS
-#define CC_SHALLOW_MIN_BLOCKS 3  // the same for the 2-slot fold machine
+#define CC_SHALLOW_MIN_BLOCKS 3  // the same for the 2- and 4-slot fold machines
 #endif
 
 // ---- folds over the N ranks ---------------------------------------------------------------------
