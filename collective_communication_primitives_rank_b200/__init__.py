@@ -55,7 +55,7 @@ _SIGS = {
     "cc_bucket_flatten": (_i, [_PP, _SZP, _i, _vp, _i, _vp]),
     "cc_bucket_unflatten": (_i, [_vp, _PP, _SZP, _i, _i, _vp]),
     "cc_bucket_allreduce": (_i, [_PP, _PP, _i, _i, _SZP, _sz, _i, _f, _vp]),
-    "cc_bucket_allreduce_host": (_i, [_PP, _PP, _PP, _PP, _i, _i, _SZP, _sz, _i, _f, _vp]),
+    "cc_bucket_allreduce_host": (_i, [_PP, _PP, _PP, _PP, _i, _i, _SZP, _sz, _i, _f, _i, _vp]),
     "cc_bucket_allreduce_buckets": (_i, [_PP, _PP, _i, _i, _SZP, _sz, _i, _i, _i, _f, _vp]),
     "cc_allreduce_slice": (_i, [_PP, _PP, _i, _i, _sz, _i, _i, _i, _i, _f, _vp]),
     "cc_reduce_scatter_slice": (_i, [_PP, _vp, _i, _i, _sz, _i, _i, _i, _f, _vp]),
@@ -410,6 +410,16 @@ class BucketAllreducePlan:
             raise CCError(st, "cc_bucket_allreduce_buckets")
 
 
+def _packed(*grids) -> int:
+    """1 when, in every table, each rank's tensors are views of one storage (one allocation),
+    the promise that lets cc_bucket_allreduce_host merge copies across tensors."""
+    for grid in grids:
+        for row in grid:
+            if len({t.untyped_storage().data_ptr() for t in row}) > 1:
+                return 0
+    return 1
+
+
 class BucketAllreduceHostPlan:
     """cc_bucket_allreduce_host with the marshalling done once (see BucketAllreducePlan)."""
 
@@ -437,11 +447,12 @@ class BucketAllreduceHostPlan:
         self._numels = _sizes([t.numel() for t in host_grads[0]])
         self.cap_bytes, self.algo = int(cap_bytes), _ALGOS[algo]
         self.scale = float(1.0 / n if scale is None else scale)
+        self.packed = _packed(host_grads, host_out, dev_grads, dev_out)
         self._fn = get_lib().cc_bucket_allreduce_host
 
     def run(self, stream=None) -> None:
         st = self._fn(self._hin, self._hout, self._din, self._dout, self.n, self.nt, self._numels, self.cap_bytes,
-                      self.algo, self.scale, _stream(stream))
+                      self.algo, self.scale, self.packed, _stream(stream))
         if st != CC_OK:
             raise CCError(st, "cc_bucket_allreduce_host")
 
@@ -471,7 +482,8 @@ def cc_bucket_allreduce_host(host_grads, host_out, dev_grads, dev_out, *, cap_by
                                         _ptrs([t for row in dev_grads for t in row]),
                                         _ptrs([t for row in dev_out for t in row]), n, nt,
                                         _sizes([t.numel() for t in host_grads[0]]), cap_bytes, _ALGOS[algo],
-                                        float(scale), _stream(stream)), "cc_bucket_allreduce_host")
+                                        float(scale), _packed(host_grads, host_out, dev_grads, dev_out),
+                                        _stream(stream)), "cc_bucket_allreduce_host")
 
 
 # ---- one rank per process: slices over peer-mapped buffers -----------------------------------

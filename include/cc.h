@@ -261,17 +261,23 @@ CC_API cc_status cc_bucket_allreduce_buckets(const void* const* grads, void* con
 /* The same fused DDP step for gradients that live in host memory: every host_grads[j] is
  * copied to dev_grads[j] (host -> device), the fused allreduce runs on the device copies,
  * and every dev_out[j] is copied back to host_out[j] (device -> host). The work is cut in
- * bucket order into slices (at most 2^20 elements per rank), and the copies in, the
- * kernels and the copies out of consecutive slices overlap on two library-owned streams
- * (created once per device) and `stream`; a slice keeps its bucket offset, so the results
- * equal cc_bucket_allreduce's. From the caller's view the call is ordered on `stream`
- * (it starts after earlier work on `stream`; later work on `stream` sees the host outputs
- * written). The caller owns the device staging buffers (dev_grads may equal dev_out);
- * host buffers must be pinned for the copies to overlap. Layouts as cc_bucket_allreduce. */
+ * bucket order into slices (at most 2^20 elements per rank) grouped into stages, and the
+ * copies in, the kernels and the copies out of consecutive stages overlap on two
+ * library-owned streams (created once per device) and `stream`; a slice keeps its bucket
+ * offset, so the results equal cc_bucket_allreduce's. From the caller's view the call is
+ * ordered on `stream` (it starts after earlier work on `stream`; later work on `stream`
+ * sees the host outputs written). The caller owns the device staging buffers (dev_grads
+ * may equal dev_out); host buffers must be pinned for the copies to overlap.
+ * packed != 0 promises that, for each rank and each of the four tables, the rank's
+ * tensors lie in one allocation (for instance views of one flat gradient buffer per
+ * rank): a stage's copies that are then contiguous on both sides are merged into one
+ * transfer. With packed == 0 a copy never spans two tensors (two allocations may happen
+ * to be adjacent, and one copy may not cross from one into the other). Layouts as
+ * cc_bucket_allreduce. */
 CC_API cc_status cc_bucket_allreduce_host(const void* const* host_grads, void* const* host_out,
                                           void* const* dev_grads, void* const* dev_out, int nranks,
                                           int ntensors, const size_t* numels, size_t cap_bytes,
-                                          cc_algo algo, float scale, void* stream);
+                                          cc_algo algo, float scale, int packed, void* stream);
 
 /* ---- One rank's slice, for ranks in separate processes (one per GPU) ----------------------
  * The same schedules with the N ranks' buffers on N GPUs, one process each: every rank's

@@ -144,6 +144,34 @@ def test_host_buffer_pipeline_matches_oracle(cap):
             assert np.array_equal(bits(h_out[r][i].numpy()), bits(want[r][i])), f"rank {r} tensor {i}"
 
 
+@pytest.mark.parametrize("cap", [30_000, 25 * 1024 * 1024])
+def test_host_buffer_pipeline_packed_matches_oracle(cap):
+    # each rank's tensors are views of one flat buffer per table: the pipeline merges a
+    # stage's contiguous copies across tensors; ~13.5M elements per rank make two stages
+    n = 8
+    shapes, grads = _small_model(n, seed=9, layers=3, d=512, ffn=2048, vocab=8000)
+    want, _ = ddp.ddp_allreduce(grads, cap_bytes=cap)
+    sizes = [g.size for g in grads[0]]
+    offs = np.concatenate([[0], np.cumsum(sizes)])
+
+    def views(flat):
+        return [flat[offs[i]:offs[i + 1]] for i in range(len(sizes))]
+
+    h_flat = [torch.from_numpy(np.concatenate([g.ravel() for g in row])).pin_memory() for row in grads]
+    ho_flat = [torch.full((int(offs[-1]),), float("nan")).pin_memory() for _ in range(n)]
+    d_flat = [torch.empty(int(offs[-1]), device="cuda") for _ in range(n)]
+    do_flat = [torch.empty(int(offs[-1]), device="cuda") for _ in range(n)]
+    plan = cc.BucketAllreduceHostPlan([views(h) for h in h_flat], [views(h) for h in ho_flat],
+                                      [views(d) for d in d_flat], [views(d) for d in do_flat], cap_bytes=cap)
+    assert plan.packed == 1
+    plan.run()
+    torch.cuda.synchronize()
+    for r in range(n):
+        got = views(ho_flat[r])
+        for i in range(len(shapes)):
+            assert np.array_equal(bits(got[i].numpy()), bits(want[r][i].ravel())), f"rank {r} tensor {i}"
+
+
 def test_flatten_allreduce_unflatten_equals_fused():
     n, cap = 8, 60_000
     shapes, grads = _small_model(n, seed=4)
