@@ -124,7 +124,8 @@ template <int IN> __device__ __forceinline__ void scale_unit(Unit<IN>& a, float 
 // The double binary tree (in-order, ((S_left (+) x) (+) S_right)) uses FOLD_CUR / PUSH /
 // NPOP; the binomial reduce (x_v first, then each child's partial) uses PUSH / NPOP /
 // FOLD_TOP. The host builds the codes; a stack of at most 6 pending partials is kept in
-// registers (each access is a warp-uniform switch, so nothing spills to local memory).
+// shared memory for 16-byte units (SmemStack) and in registers for single elements
+// (FoldStack: each access is a warp-uniform switch).
 
 constexpr uint8_t kFoldCur = 1, kPush = 2, kFoldTop = 32;
 __host__ __device__ constexpr int npop_of(uint8_t code) { return (code >> 2) & 7; }
@@ -176,9 +177,40 @@ template <typename V, int S = kStackSlots> struct FoldStack {
   }
 };
 
+// The same stack in shared memory, for units: each thread owns a column of kThreads-strided
+// 16-byte words (slot k, word w at base[(k * UW + w) * stride]; UW = 1 word per unit for
+// fp32 / int32, 2 for widened bf16), so a push or a pop is one shared-memory access at a
+// computed address instead of a switch over register slots.
+template <int IN> struct SmemStack {
+  static constexpr int UW = (int)(sizeof(Unit<IN>) / 16);
+  uint4* base;
+  int stride;
+  int depth = 0;
+  __device__ __forceinline__ void put(int k, const Unit<IN>& u) {
+#pragma unroll
+    for (int w = 0; w < UW; ++w) {
+      const uint32_t* b = reinterpret_cast<const uint32_t*>(u.v) + 4 * w;
+      base[(k * UW + w) * stride] = make_uint4(b[0], b[1], b[2], b[3]);
+    }
+  }
+  __device__ __forceinline__ Unit<IN> get(int k) const {
+    Unit<IN> u;
+#pragma unroll
+    for (int w = 0; w < UW; ++w) {
+      const uint4 q = base[(k * UW + w) * stride];
+      uint32_t* b = reinterpret_cast<uint32_t*>(u.v) + 4 * w;
+      b[0] = q.x; b[1] = q.y; b[2] = q.z; b[3] = q.w;
+    }
+    return u;
+  }
+  __device__ __forceinline__ void push(const Unit<IN>& u) { put(depth++, u); }
+  __device__ __forceinline__ Unit<IN> top() const { return get(depth - 1); }
+  __device__ __forceinline__ void set_top(const Unit<IN>& u) { put(depth - 1, u); }
+};
+
 // One position of the machine; `x` is the position's loaded value (a unit or an element).
-template <int IN, int OP, typename V, int S>
-__device__ __forceinline__ void fold_step(uint8_t code, const V& x, V& cur, FoldStack<V, S>& st) {
+template <int IN, int OP, typename V, typename St>
+__device__ __forceinline__ void fold_step(uint8_t code, const V& x, V& cur, St& st) {
   V node = x;
   if (code & kFoldCur) { node = cur; comb<IN, OP>(node, x); }
   if (code & kPush) st.push(node); else cur = node;

@@ -33,8 +33,14 @@ constexpr int kThreads = 256;
 #ifndef CC_RING_MIN_BLOCKS
 #define CC_RING_MIN_BLOCKS 4  // resident 256-thread CTAs per SM the linear-fold kernel is compiled for
 #endif
+// The fold machines keep their pending partials in shared memory, so they fit the same
+// register budget; measured against 3 (2- and 4-slot) and 2 (6-slot) resident CTAs:
+// reduce N=8 6392 vs 5570 GB/s, N=64 5788 vs 4542, trees within 1.3%.
 #ifndef CC_SHALLOW_MIN_BLOCKS
-#define CC_SHALLOW_MIN_BLOCKS 3  // the same for the 2- and 4-slot fold machines
+#define CC_SHALLOW_MIN_BLOCKS 4  // the same for the 2- and 4-slot fold machines
+#endif
+#ifndef CC_MACHINE_MIN_BLOCKS
+#define CC_MACHINE_MIN_BLOCKS 4  // the same for the 6-slot fold machine
 #endif
 
 // ---- folds over the N ranks ---------------------------------------------------------------------
@@ -63,12 +69,14 @@ __device__ __forceinline__ V ring_fold(int n, int c, Load ld, Widen widen, bool 
   return acc;
 }
 
-// Fold machine (tree / binomial): position p holds rank rank_of(p).
-template <int IN, int OP, typename V, typename X, int W, int S = kStackSlots, typename RankOf, typename Load,
+// Fold machine (tree / binomial): position p holds rank rank_of(p); `st` is an empty stack
+// of pending partials (registers or shared memory).
+template <int IN, int OP, typename V, typename X, int W, typename St, typename RankOf, typename Load,
           typename Widen>
-__device__ __forceinline__ V machine_fold(int n, const FoldProgram& prog, RankOf rank_of, Load ld, Widen widen) {
+__device__ __forceinline__ V machine_fold(int n, const FoldProgram& prog, RankOf rank_of, Load ld, Widen widen,
+                                          St& st) {
   V cur;
-  FoldStack<V, S> st;
+  st.depth = 0;
   for (int p0 = 0; p0 < n; p0 += W) {
     X x[W];
 #pragma unroll
@@ -124,7 +132,7 @@ constexpr int kLinear = 0, kMachine = 1, kHier = 2, kShallow = 3, kMid = 4;
 template <int IN, int OP, int KIND, typename RankOf, typename Src, typename EmitU, typename EmitE>
 __device__ __forceinline__ void reduce_range(int n, int g, RankOf rank_of, const FoldProgram& prog,
                                              uint64_t a, uint64_t b, uint64_t t, uint64_t T, bool vec,
-                                             Src src, EmitU emit_unit, EmitE emit_elem,
+                                             Src src, EmitU emit_unit, EmitE emit_elem, uint4* stk,
                                              int start = 0, bool up = true, int hG = 1, int hc = 0, int hj = 0) {
   constexpr bool RING = KIND == kLinear;
   constexpr int SLOTS = KIND == kShallow ? 2 : KIND == kMid ? 4 : kStackSlots;
@@ -136,7 +144,10 @@ __device__ __forceinline__ void reduce_range(int n, int g, RankOf rank_of, const
     auto ld = [&](int r) { return load_elem<IN>(src(r) + e); };
     if constexpr (RING) return ring_fold<IN, OP, A, A>(n, start, ld, same, up);
     else if constexpr (KIND == kHier) return hier_fold<IN, OP, A, A>(n, hG, hc, hj, ld, same);
-    else return machine_fold<IN, OP, A, A, 8, SLOTS>(n, prog, rank_of, ld, same);
+    else {
+      FoldStack<A, SLOTS> st;
+      return machine_fold<IN, OP, A, A, 8>(n, prog, rank_of, ld, same, st);
+    }
   };
   if (vec) {
     uint64_t va = (a + UE - 1) / UE * UE;
@@ -150,7 +161,10 @@ __device__ __forceinline__ void reduce_range(int n, int g, RankOf rank_of, const
       Unit<IN> m;
       if constexpr (RING) m = ring_fold<IN, OP, Unit<IN>, uint4>(n, start, ld, widen, up);
       else if constexpr (KIND == kHier) m = hier_fold<IN, OP, Unit<IN>, uint4>(n, hG, hc, hj, ld, widen);
-      else m = machine_fold<IN, OP, Unit<IN>, uint4, 8, SLOTS>(n, prog, rank_of, ld, widen);
+      else {
+        SmemStack<IN> st{stk, (int)T};
+        m = machine_fold<IN, OP, Unit<IN>, uint4, 8>(n, prog, rank_of, ld, widen, st);
+      }
       emit_unit(e0, m);
     }
     const uint64_t nh = va - a, nt = b - vb;
@@ -238,8 +252,12 @@ struct ReduceParams {
 template <int IN, int OP, int KIND>
 __global__ void __launch_bounds__(kThreads, KIND == kLinear ? CC_RING_MIN_BLOCKS
                                            : KIND == kHier ? 3
-                                           : KIND == kShallow || KIND == kMid ? CC_SHALLOW_MIN_BLOCKS : 2)
+                                           : KIND == kShallow || KIND == kMid ? CC_SHALLOW_MIN_BLOCKS
+                                                                              : CC_MACHINE_MIN_BLOCKS)
     reduce_kernel(const __grid_constant__ ReduceParams P) {
+  // the fold machines' pending partials, one column of 16-byte words per thread
+  constexpr int kSlots = KIND == kShallow ? 2 : KIND == kMid ? 4 : KIND == kMachine ? kStackSlots : 0;
+  __shared__ uint4 s_stk[kSlots > 0 ? kSlots * (int)(sizeof(Unit<IN>) / 16) * kThreads : 1];
   using In = typename Tr<IN>::In;
   using Out = typename Tr<IN>::Out;
   using A = typename Tr<IN>::Acc;
@@ -288,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, KIND == kLinear ? CC_RING_MIN_BLOCKS
       const int lstart = P.fold == kFoldRing ? g : P.fold == kFoldTree ? (g == 0 ? 0 : n - 1) : P.prog.rmap[0];
       const bool lup = P.fold != kFoldTree || g == 0;
       reduce_range<IN, OP, KIND>(n, g, rank_of, P.prog, s, se, threadIdx.x, blockDim.x, P.vec != 0, src,
-                                    emit_unit, emit_elem, lstart, lup, G, hc, hj);
+                                    emit_unit, emit_elem, s_stk + threadIdx.x, lstart, lup, G, hc, hj);
       s = se;
     }
   }
@@ -308,6 +326,9 @@ __global__ void __launch_bounds__(kThreads, KIND == kLinear ? CC_RING_MIN_BLOCKS
 #endif
 #ifndef CC_BUCKET_MIN_BLOCKS
 #define CC_BUCKET_MIN_BLOCKS 4     // resident 256-thread CTAs per SM the ring variant is compiled for
+#endif
+#ifndef CC_BUCKET_TREE_MIN_BLOCKS
+#define CC_BUCKET_TREE_MIN_BLOCKS 4  // the same for the tree variant (fold machine; DDP step 6022 vs 5313 GB/s at 2)
 #endif
 #ifndef CC_BUCKET_OVERSUB
 #define CC_BUCKET_OVERSUB 1024     // grid = tiles, capped at this many times the resident CTAs
@@ -339,13 +360,15 @@ static_assert(sizeof(BucketParams) <= 32000, "kernel parameter block too large")
 static_assert(sizeof(BucketParamsSmall) <= 4096, "small parameter block must stay under 4 KB");
 
 template <bool RING, typename PT>
-__global__ void __launch_bounds__(kThreads, RING ? CC_BUCKET_MIN_BLOCKS : 2) bucket_allreduce_kernel(const __grid_constant__ PT P) {
+__global__ void __launch_bounds__(kThreads, RING ? CC_BUCKET_MIN_BLOCKS : CC_BUCKET_TREE_MIN_BLOCKS)
+    bucket_allreduce_kernel(const __grid_constant__ PT P) {
   constexpr int IN = CC_F32, OP = CC_SUM;
   // the tile's per-rank pointers, staged once per tile: the fold reads them for every
   // 16-byte unit, and the parameter table is too large to stay in the constant cache
   __shared__ const float* s_in[kMaxRanks];
   __shared__ float* s_out[kMaxRanks];
   __shared__ int s_tensor;
+  __shared__ uint4 s_stk[RING ? 1 : kStackSlots * kThreads];  // the tree's pending partials
   const int n = P.nranks, nt = P.ntensors;
   const uint32_t ntiles = P.tile_prefix[nt];
   for (uint32_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
@@ -396,7 +419,8 @@ __global__ void __launch_bounds__(kThreads, RING ? CC_BUCKET_MIN_BLOCKS : 2) buc
         return mirror ? n - 1 - rk : rk;
       };
       reduce_range<IN, OP, RING ? kLinear : kMachine>(n, g, rank_of, P.prog, s, se, threadIdx.x, blockDim.x,
-                                                         P.vec != 0, src, emit_unit, emit_elem, g, true);
+                                                         P.vec != 0, src, emit_unit, emit_elem, s_stk + threadIdx.x,
+                                                         g, true);
       s = se;
     }
     __syncthreads();  // every thread is done with s_in / s_out before the next tile restages them
