@@ -135,3 +135,16 @@ def test_binding_refuses_cpu_tensors():
     x = [torch.zeros(8) for _ in range(2)]
     with pytest.raises(ValueError):
         cc.cc_allreduce(x, x)
+
+
+def test_packed_detection_for_the_host_pipeline():
+    # the host-buffer DDP step may merge copies across tensors only when, in every table, each
+    # rank's tensors are views of one storage (one allocation)
+    import torch
+    flat = [torch.zeros(100) for _ in range(2)]
+    views = [[f[0:30], f[30:100]] for f in flat]
+    assert cc._packed(views, views) == 1
+    separate = [[torch.zeros(30), torch.zeros(70)] for _ in range(2)]
+    assert cc._packed(views, separate) == 0
+    mixed = [[flat[0][0:30], torch.zeros(70)], [flat[1][0:30], flat[1][30:100]]]
+    assert cc._packed(mixed) == 0
