@@ -518,15 +518,43 @@ static void tree_program(int n, FoldProgram& fp) {
   }
 }
 
-// A program without pushes, pops or fold-into-top is a left fold in position order; it
-// runs as the linear fold when its positions walk the ranks upwards from rmap[0] (tree A
-// folds ranks 0, 1, ..., n-1; tree B is its mirror; a binomial program from its root).
+// Whether a program computes a plain left fold of its positions in order,
+// ((x_0 (+) x_1) (+) x_2) ..., and walks the ranks upwards from rmap[0] (tree A folds ranks
+// 0, 1, ..., n-1; tree B is its mirror; a binomial program from its root): it then runs as
+// the linear fold. The program is run symbolically: a value is "the left fold of positions
+// 0..k" (k >= 0; a single x_0 is k = 0), "position p alone", or anything else; one (+) of
+// the left fold of 0..k and position k+1 (in either operand order: each operator is
+// commutative) is the left fold of 0..k+1. Binomial programs for 2 and 3 ranks use a push
+// and a pop and still reduce to the left fold.
 static bool program_is_rotation(int n, const FoldProgram& fp) {
-  for (int p = 0; p < n; ++p) {
-    if ((fp.code[p] & (kPush | kFoldTop)) || npop_of(fp.code[p])) return false;
+  for (int p = 0; p < n; ++p)
     if (fp.rmap[p] != (fp.rmap[0] + p) % n) return false;
+  // value encoding: v >= 0 left fold of 0..v; v = -2 - p position p alone; kOther otherwise
+  constexpr int kOther = -1;
+  auto leaf = [](int p) { return p == 0 ? 0 : -2 - p; };
+  auto comb = [&](int a, int b) {
+    if (a >= 0 && b <= -2 && -2 - b == a + 1) return a + 1;
+    if (b >= 0 && a <= -2 && -2 - a == b + 1) return b + 1;
+    return kOther;
+  };
+  int cur = kOther;
+  std::vector<int> st;
+  for (int p = 0; p < n; ++p) {
+    const uint8_t c = fp.code[p];
+    int node = leaf(p);
+    if (c & kFoldCur) node = comb(cur, node);
+    if (c & kPush) st.push_back(node); else cur = node;
+    for (int k = npop_of(c); k > 0; --k) {
+      if (st.empty()) return false;
+      cur = comb(st.back(), cur);
+      st.pop_back();
+    }
+    if (c & kFoldTop) {
+      if (st.empty()) return false;
+      st.back() = comb(st.back(), cur);
+    }
   }
-  return true;
+  return st.empty() && cur == n - 1;
 }
 
 // Binomial tree rooted at `root` (relative rank v = (r - root) mod n; parent v - 2^floor(log2 v);
