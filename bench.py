@@ -301,6 +301,77 @@ def _row_line(args, metric, value, unit, ms, config, roofline, launches, extra=N
     print(json.dumps(line))
 
 
+def run_peer(args):
+    """One rank per GPU (torchrun): a 256 MiB fp32 allreduce per rank through libcc's slice
+    calls over CUDA IPC peer mappings (each rank folds its own chunk from every GPU and writes
+    it to every GPU, ordered by host barriers), timed beside NCCL's all_reduce of the same
+    buffer. Bus bandwidth = 2(N-1)/N * T / t per GPU (every byte of a rank's chunk leaves it
+    once each way). Parity of the slice path is covered by the GPU tests."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    import collective_communication_primitives_rank_b200 as cc
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ.setdefault("MASTER_PORT", "29531")
+    os.environ.setdefault("RANK", str(rank))
+    os.environ.setdefault("WORLD_SIZE", str(world))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    count = 64 * 1024 * 1024
+    T = count * 4
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(replica_seed(rank))
+    send = torch.randn(count, device="cuda", generator=gen)
+    recv = torch.empty_like(send)
+    stream = torch.cuda.current_stream()
+    ar = cc.PeerAllreduce(send, recv, scale=1.0 / world)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        dist.barrier()
+        return max_over_ranks(dist, torch, a.elapsed_time(b) / args.steps, "cuda")
+
+    with Clocks(local) as clocks:
+        ms = timed(ar.run)
+    x = send.clone()
+    ms_nccl = timed(lambda: dist.all_reduce(x))
+    ar.close()
+    dist.barrier()
+    factor = 2.0 * (world - 1) / world
+    bus, bus_nccl = factor * T / (ms * 1e-3) / 1e9, factor * T / (ms_nccl * 1e-3) / 1e9
+    if rank == 0:
+        peak = 770.0  # measured peer copy per direction per GPU on this pool's NVLink 5
+        print(json.dumps({
+            "metric": "allreduce bus bandwidth per GPU, 2(N-1)/N * T / t (one rank per GPU over NVLink)",
+            "value": bus, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": "peer: 256 MiB fp32 per rank, one rank per GPU, ring-order one-shot allreduce "
+                                   "(scale 1/N) through cc_allreduce_slice over CUDA IPC, host barriers included; "
+                                   "NCCL all_reduce (sum) of the same buffer as the comparator",
+                       "bytes_per_rank": T, "parallelism": f"ranks x{world}"},
+            "algbw": T / (ms * 1e-3) / 1e9,
+            "nccl": {"ms_per_step": ms_nccl, "busbw": bus_nccl, "algbw": T / (ms_nccl * 1e-3) / 1e9},
+            "roofline": {"bound": "nvlink", "achieved": bus, "peak": peak, "unit": "GB/s",
+                         "frac": bus / peak, "peak_kind": "measured peer copy (per direction)", "traffic": None,
+                         "note": "no NVLink traffic at one GPU" if world == 1 else ""},
+            "gpu_launches": args.steps, "clocks": clocks.summary()}))
+    dist.destroy_process_group()
+    return 0
+
+
 def run_rows(args):
     import torch
     import collective_communication_primitives_rank_b200 as cc
@@ -480,11 +551,14 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--oracle-buckets", type=int, default=8)
-    ap.add_argument("--workload", default="ddp", choices=["ddp", "zero", "moe", "sweep"],
-                    help="ddp = the headline step; the others measure the remaining hot-path rows")
+    ap.add_argument("--workload", default="ddp", choices=["ddp", "zero", "moe", "sweep", "peer"],
+                    help="ddp = the headline step; zero, moe, sweep measure the remaining hot-path rows; "
+                         "peer = one rank per GPU over NVLink against NCCL (run under torchrun)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "peer":
+        return run_peer(args)
     if args.workload != "ddp":
         return run_rows(args)
 
