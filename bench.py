@@ -36,7 +36,6 @@ NOMINAL_HBM_GBS = 8000.0
 N_SIM = 8
 CAP = 25 * 1024 * 1024
 SEED = 0x5EED
-PROFILE = os.path.join(ROOT, "profiles", "bucket_allreduce_ddp.txt")
 KERNEL_SRC = os.path.join(ROOT, "collective_communication_primitives_rank_b200", "csrc", "k_reduce.cu")
 
 
@@ -72,13 +71,15 @@ def measured_peak():
         return 6650.0, "fallback"
 
 
-def profile_traffic():
-    """DRAM bytes per launch of the fused kernel from the committed ncu summary, or None
-    when the kernel source changed since the counters were taken."""
+def profile_traffic(name="bucket_allreduce_ddp.txt"):
+    """DRAM bytes per launch of a line's dominant kernel from a committed ncu summary in
+    profiles/, or None when the kernel's source file changed since the counters were taken
+    (the summary records the file and its SHA-256)."""
     try:
-        lines = dict(l.split(":", 1) for l in open(PROFILE).read().splitlines() if ":" in l)
-        src = hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()
-        if lines.get("kernel_source_sha256", "").strip() != src:
+        text = open(os.path.join(ROOT, "profiles", name)).read()
+        lines = dict(l.split(":", 1) for l in text.splitlines() if ":" in l and not l.startswith(" "))
+        src = os.path.join(ROOT, lines.get("kernel_source", os.path.relpath(KERNEL_SRC, ROOT)).strip())
+        if lines.get("kernel_source_sha256", "").strip() != hashlib.sha256(open(src, "rb").read()).hexdigest():
             return None
         return int(float(lines["dram_bytes_per_launch_full_workload"].strip()))
     except Exception:
@@ -294,7 +295,7 @@ def _row_line(args, metric, value, unit, ms, config, roofline, launches, extra=N
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": config.pop("dtype", "f32"), "data": "synthetic", "config": config,
             "roofline": dict(roofline, peak=peak, peak_kind=kind, unit="GB/s",
-                             frac=roofline["achieved"] / peak, bound="hbm", traffic=None),
+                             frac=roofline["achieved"] / peak, bound="hbm", traffic=roofline.get("traffic")),
             "gpu_launches": launches}
     if extra:
         line.update(extra)
@@ -411,7 +412,8 @@ def run_rows(args):
                   {"workload": "zero: N=8 simulated ranks, 300M fp32 per rank normal(0,1e-2), ring reduce-scatter "
                                "to 37.5M-element shards, then allgather of the shards (device-seeded inputs)",
                    "l2": "inputs larger than L2; no flush"},
-                  {"achieved": (n + 1) * T / (t_rs * 1e-3) / 1e9, "kernel": "reduce_kernel<f32,sum,ring> (RS)"},
+                  {"achieved": (n + 1) * T / (t_rs * 1e-3) / 1e9, "kernel": "reduce_kernel<f32,sum,ring> (RS)",
+                   "traffic": profile_traffic("reduce_scatter_allgather_zero.txt")},
                   2 * iters,
                   {"rows": {"reduce_scatter_f32": {"ms": t_rs, "bytes": (n + 1) * T, "GBps": (n + 1) * T / t_rs / 1e6},
                             "allgather_f32": {"ms": t_ag, "bytes": (n + 1) * T, "GBps": (n + 1) * T / t_ag / 1e6},
@@ -459,7 +461,8 @@ def run_rows(args):
                   {"workload": "moe: N=8 simulated ranks, 8192 tokens x 4096 bf16 per rank, 64 experts (8 per rank), "
                                "top-2 routing from normal logits, dispatch then combine (device-seeded inputs)",
                    "dtype": "bf16 (bit copy)", "l2": "inputs larger than L2; no flush"},
-                  {"achieved": b_d / (t_d * 1e-3) / 1e9, "kernel": "a2a dispatch (count + scan + base + copy)"},
+                  {"achieved": b_d / (t_d * 1e-3) / 1e9, "kernel": "a2a dispatch (count + scan + base + copy)",
+                   "traffic": profile_traffic("alltoallv_dispatch_moe.txt")},
                   iters * (1 + 4 + 4),
                   {"rows": {"route_topk": {"ms": t_route},
                             "dispatch": {"ms": t_d, "bytes": b_d, "GBps": b_d / t_d / 1e6},
