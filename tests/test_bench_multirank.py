@@ -64,3 +64,25 @@ def test_reference_arm_under_torchrun_prints_once():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_profile_traffic_goes_null_when_the_kernel_source_changes(tmp_path):
+    # a committed ncu summary carries the SHA-256 of the kernel source it measured; bench.py
+    # reports its DRAM traffic only while that source is unchanged
+    import hashlib
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    src = tmp_path / "k.cu"
+    src.write_text("kernel v1\n")
+    (tmp_path / "profiles").mkdir()
+    sha = hashlib.sha256(b"kernel v1\n").hexdigest()
+    (tmp_path / "profiles" / "p.txt").write_text(
+        f"kernel_source: k.cu\nkernel_source_sha256: {sha}\ndram_bytes_per_launch_full_workload: 1234\n"
+        "  launch  0  1.0 us\n")
+    b.ROOT = str(tmp_path)
+    assert b.profile_traffic("p.txt") == 1234
+    src.write_text("kernel v2\n")
+    assert b.profile_traffic("p.txt") is None
+    assert b.profile_traffic("missing.txt") is None
