@@ -22,8 +22,10 @@ Modules:
 Pins (tests/test_oracle_*.py): the pages' worked examples (tests/golden/), the per-rank
 byte counts the pages derive, allreduce == allgather(reduce_scatter) bit for bit, the
 N = 1 identity, int32 against brute-force sums, fp32 against an independent left-fold /
-recursive evaluator and against an fp64 error bound, tree-shape invariants, alltoallv
-round trip and count conservation, and gloo (int32) on CPU processes.
+recursive evaluator and against an fp64 error bound, tree-shape invariants and hand-derived
+tree shapes for N = 5, 6, 8, 13 (tests/golden/tree_shapes.json), the binomial reduce's
+bracketing against an evaluator built from the broadcast's rounds, alltoallv round trip and
+count conservation, and gloo (int32) on CPU processes.
 Parity unpinned: the per-rank byte figures the pages give for the tree (they disagree with
 one another; the oracle counts what its own schedule moves).
 """
