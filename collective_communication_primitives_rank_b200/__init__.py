@@ -25,6 +25,13 @@ CC_F32, CC_BF16, CC_I32 = 0, 1, 2
 CC_SUM, CC_MAX, CC_MIN, CC_PROD = 0, 1, 2, 3
 CC_ALGO_RING, CC_ALGO_TREE = 0, 1
 MAX_RANKS = 64
+# `scale` value that asks the library for the average over the ranks (it multiplies by
+# fl(1/N) itself); the bucket calls pass it when scale is None
+CC_SCALE_MEAN = float("nan")
+
+
+def _scale(scale) -> float:
+    return CC_SCALE_MEAN if scale is None else float(scale)
 
 _vp, _sz, _i, _f = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_float
 _PP = ctypes.POINTER(ctypes.c_void_p)
@@ -181,7 +188,7 @@ def cc_allreduce(send, recv, *, op="sum", algo="ring", scale=1.0, stream=None) -
     if len(recv) != n:
         raise ValueError("cc_allreduce: one output per rank")
     _check(lib.cc_allreduce(_ptrs(send), _ptrs(recv), n, send[0].numel(), dtype_code(send[0]),
-                            dtype_code(recv[0]), _OPS[op], _ALGOS[algo], float(scale), _stream(stream)),
+                            dtype_code(recv[0]), _OPS[op], _ALGOS[algo], _scale(scale), _stream(stream)),
            "cc_allreduce")
 
 
@@ -193,7 +200,7 @@ def cc_allreduce_hierarchical(send, recv, ranks_per_node: int, *, op="sum", scal
     if len(recv) != n:
         raise ValueError("cc_allreduce_hierarchical: one output per rank")
     _check(lib.cc_allreduce_hierarchical(_ptrs(send), _ptrs(recv), n, int(ranks_per_node), send[0].numel(),
-                                         dtype_code(send[0]), dtype_code(recv[0]), _OPS[op], float(scale),
+                                         dtype_code(send[0]), dtype_code(recv[0]), _OPS[op], _scale(scale),
                                          _stream(stream)), "cc_allreduce_hierarchical")
 
 
@@ -206,7 +213,7 @@ def cc_allreduce_stepped(send, recv, workspace, *, op="sum", algo="ring", scale=
     if len(recv) != n:
         raise ValueError("cc_allreduce_stepped: one output per rank")
     _check(lib.cc_allreduce_stepped(_ptrs(send), _ptrs(recv), n, send[0].numel(), dtype_code(send[0]),
-                                    dtype_code(recv[0]), _OPS[op], _ALGOS[algo], float(scale), _dev_ptr(workspace),
+                                    dtype_code(recv[0]), _OPS[op], _ALGOS[algo], _scale(scale), _dev_ptr(workspace),
                                     workspace.numel() * workspace.element_size(), _stream(stream)),
            "cc_allreduce_stepped")
 
@@ -220,7 +227,7 @@ def cc_reduce_scatter(send, recv, *, op="sum", algo="ring", scale=1.0, stream=No
     for c in range(n):
         _same([recv[c]], cc_chunk(send[0].numel(), n, c)[1], recv[0].dtype, f"cc_reduce_scatter recv[{c}]")
     _check(lib.cc_reduce_scatter(_ptrs(send), _ptrs(recv), n, send[0].numel(), dtype_code(send[0]),
-                                 dtype_code(recv[0]), _OPS[op], _ALGOS[algo], float(scale), _stream(stream)),
+                                 dtype_code(recv[0]), _OPS[op], _ALGOS[algo], _scale(scale), _stream(stream)),
            "cc_reduce_scatter")
 
 
@@ -248,7 +255,7 @@ def cc_reduce(send, recv_root, root: int = 0, *, op="sum", scale=1.0, stream=Non
     _same(send, send[0].numel(), send[0].dtype, "cc_reduce send")
     _same([recv_root], send[0].numel(), recv_root.dtype, "cc_reduce recv_root")
     _check(lib.cc_reduce(_ptrs(send), _dev_ptr(recv_root), len(send), root, send[0].numel(), dtype_code(send[0]),
-                         dtype_code(recv_root), _OPS[op], float(scale), _stream(stream)), "cc_reduce")
+                         dtype_code(recv_root), _OPS[op], _scale(scale), _stream(stream)), "cc_reduce")
 
 
 def cc_scatter(src, recv, root: int = 0, *, stream=None) -> None:
@@ -365,11 +372,10 @@ def cc_bucket_allreduce(grads, out, *, cap_bytes: int = 25 * 1024 * 1024, algo="
     for i in range(nt):
         _same([grads[r][i] for r in range(n)] + [out[r][i] for r in range(n)], grads[0][i].numel(),
               torch.float32, f"cc_bucket_allreduce tensor {i}")
-    scale = 1.0 / n if scale is None else scale
     flat_in = [t for row in grads for t in row]
     flat_out = [t for row in out for t in row]
     _check(lib.cc_bucket_allreduce(_ptrs(flat_in), _ptrs(flat_out), n, nt, _sizes([t.numel() for t in grads[0]]),
-                                   cap_bytes, _ALGOS[algo], float(scale), _stream(stream)), "cc_bucket_allreduce")
+                                   cap_bytes, _ALGOS[algo], _scale(scale), _stream(stream)), "cc_bucket_allreduce")
 
 
 class BucketAllreducePlan:
@@ -392,7 +398,7 @@ class BucketAllreducePlan:
         self._numels = _sizes([t.numel() for t in grads[0]])
         self.cap_bytes = int(cap_bytes)
         self.algo = _ALGOS[algo]
-        self.scale = float(1.0 / n if scale is None else scale)
+        self.scale = _scale(scale)
         self._fn = get_lib().cc_bucket_allreduce
 
     def run(self, stream=None) -> None:
@@ -446,7 +452,7 @@ class BucketAllreduceHostPlan:
         self._dout = _ptrs([t for row in dev_out for t in row])
         self._numels = _sizes([t.numel() for t in host_grads[0]])
         self.cap_bytes, self.algo = int(cap_bytes), _ALGOS[algo]
-        self.scale = float(1.0 / n if scale is None else scale)
+        self.scale = _scale(scale)
         self.packed = _packed(host_grads, host_out, dev_grads, dev_out)
         self._fn = get_lib().cc_bucket_allreduce_host
 
@@ -476,13 +482,12 @@ def cc_bucket_allreduce_host(host_grads, host_out, dev_grads, dev_out, *, cap_by
                 raise ValueError("cc_bucket_allreduce_host: host tables must hold CPU tensors")
             if not (host_grads[r][i].is_contiguous() and host_out[r][i].is_contiguous()):
                 raise ValueError("cc_bucket_allreduce_host: contiguous tensors only")
-    scale = 1.0 / n if scale is None else scale
     hp = lambda grid: (ctypes.c_void_p * (n * nt))(*[t.data_ptr() for row in grid for t in row])
     _check(lib.cc_bucket_allreduce_host(hp(host_grads), hp(host_out),
                                         _ptrs([t for row in dev_grads for t in row]),
                                         _ptrs([t for row in dev_out for t in row]), n, nt,
                                         _sizes([t.numel() for t in host_grads[0]]), cap_bytes, _ALGOS[algo],
-                                        float(scale), _packed(host_grads, host_out, dev_grads, dev_out),
+                                        _scale(scale), _packed(host_grads, host_out, dev_grads, dev_out),
                                         _stream(stream)), "cc_bucket_allreduce_host")
 
 
@@ -572,7 +577,7 @@ def cc_allreduce_slice(send, recv, rank: int, *, op="sum", algo="ring", scale=1.
     if len(recv) != len(send) or r0.numel() != s0.numel():
         raise ValueError("cc_allreduce_slice: one output per rank, as long as the input")
     _check(lib.cc_allreduce_slice(sp, rp, len(send), rank, s0.numel(), dtype_code(s0), dtype_code(r0), _OPS[op],
-                                  _ALGOS[algo], float(scale), _stream(stream)), "cc_allreduce_slice")
+                                  _ALGOS[algo], _scale(scale), _stream(stream)), "cc_allreduce_slice")
 
 
 def cc_reduce_scatter_slice(send, shard, rank: int, *, op="sum", scale=1.0, stream=None) -> None:
@@ -582,7 +587,7 @@ def cc_reduce_scatter_slice(send, shard, rank: int, *, op="sum", scale=1.0, stre
     n = len(send)
     _same([shard], cc_chunk(s0.numel(), n, rank)[1], shard.dtype, "cc_reduce_scatter_slice shard")
     _check(lib.cc_reduce_scatter_slice(sp, _dev_ptr(shard), n, rank, s0.numel(), dtype_code(s0),
-                                       dtype_code(shard), _OPS[op], float(scale), _stream(stream)),
+                                       dtype_code(shard), _OPS[op], _scale(scale), _stream(stream)),
            "cc_reduce_scatter_slice")
 
 

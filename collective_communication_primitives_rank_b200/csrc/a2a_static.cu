@@ -10,6 +10,7 @@
 // the process exits.
 #include <mutex>
 
+#include "cc_args.h"
 #include "cc_launch.h"
 
 namespace {
@@ -20,11 +21,12 @@ constexpr int kMaxDevices = 64;
 __device__ __align__(256) unsigned char g_a2a_scratch[kStaticScratchBytes];
 
 // In host code g_a2a_scratch names a host-side stand-in, not device memory: the device
-// address is looked up once per device, with that device current.
+// address is looked up with the device current, and only a successful lookup is kept, so a
+// call that failed (for instance one made while a stream was being captured) leaves the
+// next call free to try again.
 struct DeviceScratch {
-  std::once_flag once;
+  std::mutex mu;
   void* ptr = nullptr;
-  cudaError_t err = cudaSuccess;
 };
 DeviceScratch g_scratch[kMaxDevices];
 
@@ -34,19 +36,18 @@ cudaError_t scratch_for_current_device(void** out) {
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   DeviceScratch& s = g_scratch[dev];
-  std::call_once(s.once, [&s] { s.err = cudaGetSymbolAddress(&s.ptr, g_a2a_scratch); });
-  if (s.err != cudaSuccess) return s.err;
+  std::lock_guard<std::mutex> lock(s.mu);
+  if (!s.ptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_a2a_scratch);
+    if (e != cudaSuccess) {
+      cudaGetLastError();  // do not leave the failed lookup pending for the caller
+      return e;
+    }
+    s.ptr = p;
+  }
   *out = s.ptr;
   return cudaSuccess;
-}
-
-bool ranks_ok(int n) { return n >= 1 && n <= CC_MAX_RANKS; }
-
-bool nonnull(const void* const* p, int n) {
-  if (!p) return false;
-  for (int i = 0; i < n; ++i)
-    if (!p[i]) return false;
-  return true;
 }
 
 }  // namespace
@@ -55,15 +56,8 @@ extern "C" cc_status cc_alltoallv_noalloc(const void* const* send, void* const* 
                                           const int32_t* const* expert_ids, int tokens, int topk,
                                           int experts_per_rank, size_t recv_capacity_rows, int direction,
                                           int32_t* recv_rows, void* stream) {
-  if (!ranks_ok(nranks) || tokens < 0 || topk < 1 || topk > 8 || experts_per_rank < 1 ||
-      (long long)nranks * experts_per_rank > 1024 || (long long)tokens * topk >= (1ll << 31))
+  if (!cc::a2a_args_ok(send, recv, nranks, row_bytes, expert_ids, tokens, topk, experts_per_rank, direction))
     return CC_ERR_INVALID_ARG;
-  if (!nonnull(send, nranks) || !nonnull((const void* const*)recv, nranks) ||
-      !nonnull((const void* const*)expert_ids, nranks))
-    return CC_ERR_INVALID_ARG;
-  if (row_bytes == 0 || row_bytes % 16 != 0 || (direction != 0 && direction != 1)) return CC_ERR_INVALID_ARG;
-  for (int r = 0; r < nranks; ++r)
-    if ((reinterpret_cast<uintptr_t>(send[r]) | reinterpret_cast<uintptr_t>(recv[r])) & 15) return CC_ERR_INVALID_ARG;
   // the routing scratch must fit the fixed array
   if (cc::a2a_workspace_bytes(nranks, tokens, topk, experts_per_rank) > kStaticScratchBytes) return CC_ERR_INVALID_ARG;
   void* scratch = nullptr;

@@ -6,6 +6,7 @@
 #include <mutex>
 #include <vector>
 
+#include "cc_args.h"
 #include "cc_launch.h"
 
 using namespace cc;
@@ -18,15 +19,6 @@ size_t dtype_bytes(cc_dtype t) { return t == CC_BF16 ? 2 : 4; }
 
 bool valid_dtype(int t) { return t == CC_F32 || t == CC_BF16 || t == CC_I32; }
 
-bool valid_ranks(int nranks) { return nranks >= 1 && nranks <= CC_MAX_RANKS; }
-
-bool all_nonnull(const void* const* p, int n) {
-  if (!p) return false;
-  for (int i = 0; i < n; ++i)
-    if (!p[i]) return false;
-  return true;
-}
-
 // The reduction dtype pairs: (F32, F32), (BF16, F32), (I32, I32).
 cc_status check_reduce(int in_t, int out_t, int op, float scale) {
   if (!valid_dtype(in_t) || !valid_dtype(out_t)) return CC_ERR_INVALID_ARG;
@@ -34,10 +26,13 @@ cc_status check_reduce(int in_t, int out_t, int op, float scale) {
                        (in_t == CC_I32 && out_t == CC_I32);
   if (!pair_ok) return CC_ERR_INVALID_ARG;
   if (op < CC_SUM || op > CC_PROD) return CC_ERR_INVALID_ARG;
-  if (in_t == CC_I32 && scale != 1.0f) return CC_ERR_INVALID_ARG;
-  if (!(scale == scale)) return CC_ERR_INVALID_ARG;  // NaN scale
+  if (in_t == CC_I32 && scale != 1.0f) return CC_ERR_INVALID_ARG;  // CC_SCALE_MEAN included
   return CC_OK;
 }
+
+// CC_SCALE_MEAN (any NaN) asks for the average over the N ranks: one binary32 multiply of
+// the folded sum by fl(1/N), the DDP average of lecture 09 §3.5 / §6.1.
+float resolve_scale(float scale, int nranks) { return scale == scale ? scale : 1.0f / (float)nranks; }
 
 void chunk_bounds(size_t count, int n, int c, size_t& a, size_t& len) {
   const size_t q = count / n, r = count % n;
@@ -307,8 +302,8 @@ cc_status cc_allreduce(const void* const* send, void* const* recv, int nranks, s
   for (int r = 0; r < nranks; ++r)
     if (recv[r] == send[r] && dtype_bytes(in_t) != dtype_bytes(out_t)) return CC_ERR_INVALID_ARG;
   return cuda_status(launch_reduce(send, recv, nranks, nranks, count, in_t, op,
-                                   algo == CC_ALGO_RING ? kFoldRing : kFoldTree, kAllReduce, 0, scale,
-                                   as_stream(stream)));
+                                   algo == CC_ALGO_RING ? kFoldRing : kFoldTree, kAllReduce, 0,
+                                   resolve_scale(scale, nranks), as_stream(stream)));
 }
 
 cc_status cc_allreduce_stepped(const void* const* send, void* const* recv, int nranks, size_t count, cc_dtype in_t,
@@ -323,8 +318,9 @@ cc_status cc_allreduce_stepped(const void* const* send, void* const* recv, int n
   for (int r = 0; r < nranks; ++r)
     if (recv[r] == send[r] && dtype_bytes(in_t) != dtype_bytes(out_t)) return CC_ERR_INVALID_ARG;
   return cuda_status(launch_stepped_allreduce(send, recv, nranks, count, in_t, op,
-                                              algo == CC_ALGO_RING ? kFoldRing : kFoldTree, scale,
-                                              static_cast<unsigned*>(workspace), as_stream(stream)));
+                                              algo == CC_ALGO_RING ? kFoldRing : kFoldTree,
+                                              resolve_scale(scale, nranks), static_cast<unsigned*>(workspace),
+                                              as_stream(stream)));
 }
 
 cc_status cc_allreduce_hierarchical(const void* const* send, void* const* recv, int nranks, int ranks_per_node,
@@ -337,7 +333,7 @@ cc_status cc_allreduce_hierarchical(const void* const* send, void* const* recv, 
   for (int r = 0; r < nranks; ++r)
     if (recv[r] == send[r] && dtype_bytes(in_t) != dtype_bytes(out_t)) return CC_ERR_INVALID_ARG;
   return cuda_status(launch_reduce(send, recv, nranks, nranks, count, in_t, op, kFoldHier, kAllReduce, ranks_per_node,
-                                   scale, as_stream(stream)));
+                                   resolve_scale(scale, nranks), as_stream(stream)));
 }
 
 cc_status cc_reduce_scatter(const void* const* send, void* const* recv, int nranks, size_t count, cc_dtype in_t,
@@ -354,7 +350,7 @@ cc_status cc_reduce_scatter(const void* const* send, void* const* recv, int nran
     if (len && !recv[c]) return CC_ERR_INVALID_ARG;  // an empty shard may be null
   }
   return cuda_status(launch_reduce(send, recv, nranks, nranks, count, in_t, op, kFoldRing, kReduceScatter, 0,
-                                   scale, as_stream(stream)));
+                                   resolve_scale(scale, nranks), as_stream(stream)));
 }
 
 cc_status cc_reduce(const void* const* send, void* recv_root, int nranks, int root, size_t count, cc_dtype in_t,
@@ -364,8 +360,8 @@ cc_status cc_reduce(const void* const* send, void* recv_root, int nranks, int ro
   if (count == 0) return CC_OK;
   if (!all_nonnull(send, nranks) || !recv_root) return CC_ERR_INVALID_ARG;
   void* dst[1] = {recv_root};
-  return cuda_status(launch_reduce(send, dst, 1, nranks, count, in_t, op, kFoldBinomial, kReduceRoot, root, scale,
-                                   as_stream(stream)));
+  return cuda_status(launch_reduce(send, dst, 1, nranks, count, in_t, op, kFoldBinomial, kReduceRoot, root,
+                                   resolve_scale(scale, nranks), as_stream(stream)));
 }
 
 cc_status cc_allgather(const void* const* send, void* const* recv, int nranks, size_t count, cc_dtype dtype,
@@ -439,11 +435,6 @@ cc_status cc_route_topk(const float* const* logits, int32_t* const* expert_ids, 
   return cuda_status(launch_route_topk(logits, expert_ids, nranks, tokens, experts_total, topk, as_stream(stream)));
 }
 
-static bool a2a_shape_ok(int nranks, int tokens, int topk, int experts_per_rank) {
-  return valid_ranks(nranks) && tokens >= 0 && topk >= 1 && topk <= 8 && experts_per_rank >= 1 &&
-         (long long)nranks * experts_per_rank <= 1024 && (long long)tokens * topk < (1ll << 31);
-}
-
 size_t cc_alltoallv_workspace_size(int nranks, int tokens, int topk, int experts_per_rank) {
   if (!a2a_shape_ok(nranks, tokens, topk, experts_per_rank)) return 0;
   return a2a_workspace_bytes(nranks, tokens, topk, experts_per_rank);
@@ -453,16 +444,11 @@ cc_status cc_alltoallv(const void* const* send, void* const* recv, int nranks, s
                        const int32_t* const* expert_ids, int tokens, int topk, int experts_per_rank,
                        size_t recv_capacity_rows, int direction, void* workspace, size_t workspace_bytes,
                        void* stream) {
-  if (!a2a_shape_ok(nranks, tokens, topk, experts_per_rank)) return CC_ERR_INVALID_ARG;
-  if (!all_nonnull(send, nranks) || !all_nonnull((const void* const*)recv, nranks) ||
-      !all_nonnull((const void* const*)expert_ids, nranks))
+  if (!a2a_args_ok(send, recv, nranks, row_bytes, expert_ids, tokens, topk, experts_per_rank, direction))
     return CC_ERR_INVALID_ARG;
-  if (row_bytes == 0 || row_bytes % 16 != 0 || (direction != 0 && direction != 1)) return CC_ERR_INVALID_ARG;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255) ||
       workspace_bytes < a2a_workspace_bytes(nranks, tokens, topk, experts_per_rank))
     return CC_ERR_INVALID_ARG;
-  for (int r = 0; r < nranks; ++r)
-    if ((reinterpret_cast<uintptr_t>(send[r]) | reinterpret_cast<uintptr_t>(recv[r])) & 15) return CC_ERR_INVALID_ARG;
   return cuda_status(launch_alltoallv(send, recv, nranks, row_bytes, expert_ids, tokens, topk, experts_per_rank,
                                       recv_capacity_rows, direction, workspace, as_stream(stream)));
 }
@@ -529,10 +515,11 @@ cc_status cc_bucket_unflatten(const void* bucket, void* const* tensors, const si
 
 cc_status cc_bucket_allreduce(const void* const* grads, void* const* out, int nranks, int ntensors,
                               const size_t* numels, size_t cap_bytes, cc_algo algo, float scale, void* stream) {
-  if (!valid_ranks(nranks) || ntensors < 0 || cap_bytes == 0 || !(scale == scale)) return CC_ERR_INVALID_ARG;
+  if (!valid_ranks(nranks) || ntensors < 0 || cap_bytes == 0) return CC_ERR_INVALID_ARG;
   if (algo != CC_ALGO_RING && algo != CC_ALGO_TREE) return CC_ERR_INVALID_ARG;
   if (ntensors == 0) return CC_OK;
   if (!numels || !grads || !out) return CC_ERR_INVALID_ARG;
+  scale = resolve_scale(scale, nranks);
   for (int r = 0; r < nranks; ++r)
     for (int i = 0; i < ntensors; ++i)
       if (numels[i] && (!grads[(size_t)r * ntensors + i] || !out[(size_t)r * ntensors + i]))
@@ -547,9 +534,9 @@ cc_status cc_bucket_allreduce(const void* const* grads, void* const* out, int nr
 cc_status cc_bucket_allreduce_buckets(const void* const* grads, void* const* out, int nranks, int ntensors,
                                       const size_t* numels, size_t cap_bytes, int first_bucket, int nbuckets,
                                       cc_algo algo, float scale, void* stream) {
-  if (!valid_ranks(nranks) || ntensors < 0 || cap_bytes == 0 || !(scale == scale) || first_bucket < 0 ||
-      nbuckets < 0)
+  if (!valid_ranks(nranks) || ntensors < 0 || cap_bytes == 0 || first_bucket < 0 || nbuckets < 0)
     return CC_ERR_INVALID_ARG;
+  scale = resolve_scale(scale, nranks);
   if (algo != CC_ALGO_RING && algo != CC_ALGO_TREE) return CC_ERR_INVALID_ARG;
   if (ntensors == 0 || nbuckets == 0) return CC_OK;
   if (!numels || !grads || !out) return CC_ERR_INVALID_ARG;
@@ -569,7 +556,8 @@ cc_status cc_bucket_allreduce_buckets(const void* const* grads, void* const* out
 cc_status cc_bucket_allreduce_host(const void* const* host_grads, void* const* host_out, void* const* dev_grads,
                                    void* const* dev_out, int nranks, int ntensors, const size_t* numels,
                                    size_t cap_bytes, cc_algo algo, float scale, int packed, void* stream) {
-  if (!valid_ranks(nranks) || ntensors < 0 || cap_bytes == 0 || !(scale == scale)) return CC_ERR_INVALID_ARG;
+  if (!valid_ranks(nranks) || ntensors < 0 || cap_bytes == 0) return CC_ERR_INVALID_ARG;
+  scale = resolve_scale(scale, nranks);
   if (algo != CC_ALGO_RING && algo != CC_ALGO_TREE) return CC_ERR_INVALID_ARG;
   if (ntensors == 0) return CC_OK;
   if (!host_grads || !host_out || !dev_grads || !dev_out || !numels) return CC_ERR_INVALID_ARG;
@@ -597,8 +585,8 @@ cc_status cc_allreduce_slice(const void* const* send, void* const* recv, int nra
   chunk_bounds(count, nranks, rank, a, len);
   if (len == 0) return CC_OK;
   return cuda_status(launch_reduce(send, recv, nranks, nranks, count, in_t, op,
-                                   algo == CC_ALGO_RING ? kFoldRing : kFoldTree, kAllReduce, 0, scale,
-                                   as_stream(stream), a, a + len));
+                                   algo == CC_ALGO_RING ? kFoldRing : kFoldTree, kAllReduce, 0,
+                                   resolve_scale(scale, nranks), as_stream(stream), a, a + len));
 }
 
 cc_status cc_reduce_scatter_slice(const void* const* send, void* recv_shard, int nranks, int rank, size_t count,
@@ -615,7 +603,7 @@ cc_status cc_reduce_scatter_slice(const void* const* send, void* recv_shard, int
   std::vector<void*> dst(nranks, nullptr);
   dst[rank] = recv_shard;
   return cuda_status(launch_reduce(send, dst.data(), nranks, nranks, count, in_t, op, kFoldRing, kReduceScatter, 0,
-                                   scale, as_stream(stream), a, a + len));
+                                   resolve_scale(scale, nranks), as_stream(stream), a, a + len));
 }
 
 cc_status cc_allgather_slice(const void* send_shard, void* const* recv, int nranks, int rank, size_t count,

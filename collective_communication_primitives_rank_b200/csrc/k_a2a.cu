@@ -341,7 +341,9 @@ cudaError_t launch_alltoallv(const void* const* send, void* const* recv, int nra
     a2a_count_kernel<<<dim3(ntiles, nranks), kTileRows, sizeof(int) * 8 * E, stream>>>(I, rows, E, tile_cnt, row_rank);
     a2a_tile_scan_kernel<<<dim3(E, nranks), 32, 0, stream>>>(ntiles, E, tile_cnt, totals);
   } else {
-    cudaMemsetAsync(totals, 0, sizeof(int) * nranks * E, stream);
+    // no rows: the bases read zero totals (the only write to this scratch before K3)
+    const cudaError_t e = cudaMemsetAsync(totals, 0, sizeof(int) * nranks * E, stream);
+    if (e != cudaSuccess) return e;
   }
   a2a_base_kernel<<<1, 1024, 0, stream>>>(nranks, experts_per_rank, totals, base, recv_count);
   cudaError_t err = cudaGetLastError();

@@ -21,7 +21,10 @@
  * (+) is one IEEE binary32 operation rounded to nearest even (SUM add, PROD multiply,
  * MAX / MIN with -0 ordered below +0), or the wrapping int32 operation. bf16 inputs are
  * widened exactly to binary32 before the first operation. `scale` multiplies the final
- * result once (binary32); it must be 1 for int32.
+ * result once (binary32); it must be 1 for int32. CC_SCALE_MEAN (any NaN) asks for the
+ * average over the N ranks, the DDP step of lecture 09 §3.5 / §6.1 (AllReduce(SUM), then
+ * divide by the card count): the library then multiplies by fl(1/N), computed in binary32
+ * (exactly 1/N for N a power of two); for int32 it is CC_ERR_INVALID_ARG.
  *
  * Conventions for every call:
  *   - send / recv are HOST arrays of nranks DEVICE pointers (1 <= nranks <= 64), one per
@@ -40,6 +43,7 @@
 #ifndef CC_H_
 #define CC_H_
 
+#include <math.h>
 #include <stddef.h>
 #include <stdint.h>
 
@@ -60,6 +64,9 @@ typedef enum { CC_SUM = 0, CC_MAX = 1, CC_MIN = 2, CC_PROD = 3 } cc_op;
 typedef enum { CC_ALGO_RING = 0, CC_ALGO_TREE = 1 } cc_algo;
 
 #define CC_MAX_RANKS 64
+
+/* `scale` argument of the reductions meaning "the mean over the ranks": fl(1/N). */
+#define CC_SCALE_MEAN (NAN)
 
 #if defined(__GNUC__)
 #define CC_API __attribute__((visibility("default")))
@@ -97,7 +104,7 @@ CC_API cc_status cc_chunk(size_t count, int nranks, int c, size_t* start, size_t
  *   send[r]: count elements of in_t;  recv[r]: count elements of out_t.
  *   In place allowed (recv[r] == send[r] for every r, same dtype width).
  * Errors: CC_ERR_INVALID_ARG for null arrays/pointers, nranks outside [1, 64], a dtype
- * pair not listed above, op outside cc_op, scale != 1 for I32. */
+ * pair not listed above, op outside cc_op, scale != 1 for I32 (CC_SCALE_MEAN included). */
 CC_API cc_status cc_allreduce(const void* const* send, void* const* recv, int nranks, size_t count,
                        cc_dtype in_t, cc_dtype out_t, cc_op op, cc_algo algo, float scale,
                        void* stream);

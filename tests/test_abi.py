@@ -83,7 +83,7 @@ FAKE = [0x10000 * (i + 1) for i in range(65)]  # never dereferenced: every call 
     (dict(in_t=cc.CC_I32, out_t=cc.CC_I32, scale=0.5), cc.CC_ERR_INVALID_ARG),
     (dict(op=7), cc.CC_ERR_INVALID_ARG),
     (dict(algo=5), cc.CC_ERR_INVALID_ARG),
-    (dict(scale=float("nan")), cc.CC_ERR_INVALID_ARG),
+    (dict(in_t=cc.CC_I32, out_t=cc.CC_I32, scale=cc.CC_SCALE_MEAN), cc.CC_ERR_INVALID_ARG),  # no int mean
     (dict(null_at=2), cc.CC_ERR_INVALID_ARG),
     (dict(count=0), cc.CC_OK),
 ])

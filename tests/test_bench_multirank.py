@@ -86,3 +86,54 @@ def test_profile_traffic_goes_null_when_the_kernel_source_changes(tmp_path):
     src.write_text("kernel v2\n")
     assert b.profile_traffic("p.txt") is None
     assert b.profile_traffic("missing.txt") is None
+
+
+def _layout_worker(rank, world, port, q):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    numels = [synth.numel(s) for _, s in synth.transformer_grad_shapes(layers=2)]
+    offs, ranges = bench.bucket_order_layout(numels, cap=4 * 1024 * 1024)
+    every = [None] * world
+    dist.all_gather_object(every, (offs, ranges))
+    # fake peer base addresses: every rank's flat buffer at its own address
+    bases = [0x7000_0000_0000 + r * 0x1_0000_0000 for r in range(world)]
+    ptrs = [bench.offset_ptrs(bases, start) for start, _ in ranges]
+    q.put((rank, every, offs, ranges, numels, ptrs, bases))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.timeout(120)
+def test_multi_gpu_bucket_layout_agrees_across_ranks_and_tiles_the_buffer():
+    """The one-rank-per-GPU path: every rank derives the same flat bucket-order layout, each
+    bucket is one contiguous range holding exactly its tensors, the ranges tile the buffer,
+    and a bucket's pointers are every rank's base advanced by the bucket's start."""
+    import torch.multiprocessing as mp
+    sys.path.insert(0, ROOT)
+    import collective_communication_primitives_rank_b200 as cc
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _port()
+    procs = [ctx.Process(target=_layout_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = [q.get(timeout=90) for _ in range(2)]
+    for p in procs:
+        p.join(timeout=30)
+        assert p.exitcode == 0
+    for rank, every, offs, ranges, numels, ptrs, bases in got:
+        assert every[0] == every[1]
+        assert ranges[0][0] == 0 and sum(c for _, c in ranges) == sum(numels)
+        for (s0, c0), (s1, _) in zip(ranges, ranges[1:]):
+            assert s0 + c0 == s1
+        buckets = cc.cc_bucket_assign(numels, 4, 4 * 1024 * 1024)
+        assert len(buckets) == len(ranges)
+        for members, (start, count) in zip(buckets, ranges):
+            assert sorted(offs[i] for i in members) == [offs[i] for i in members]  # in the order taken
+            assert offs[members[0]] == start and sum(numels[i] for i in members) == count
+        for (start, _), p in zip(ranges, ptrs):
+            assert p == [b + 4 * start for b in bases]

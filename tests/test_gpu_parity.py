@@ -305,3 +305,30 @@ def test_hierarchical_in_place_and_large_sampled():
     idx = torch.from_numpy(pos).cuda()
     for r in (0, 37, n - 1):
         _assert_same(buf[r][idx].cpu().numpy(), want[r], f"rank {r}")
+
+
+# ---- CC_SCALE_MEAN: the library takes the average itself (fl(1/N) in binary32) -------------------------
+
+@pytest.mark.parametrize("n", [3, 5, 6, 7, 8])
+def test_scale_mean_sentinel_equals_explicit_reciprocal(n):
+    count = 3 * 1024 + 5
+    xs = _inputs("spread", n, count, seed=50)
+    inv = float(np.float32(1) / np.float32(n))  # fl(1/N), one correctly rounded binary32 division
+    send = [to_dev(x) for x in xs]
+    for algo, fn in (("ring", C.ring_allreduce), ("tree", C.tree_allreduce)):
+        want, _ = fn(xs, scale=inv)
+        out = [torch.empty(count, device="cuda") for _ in range(n)]
+        cc.cc_allreduce(send, out, algo=algo, scale=None)
+        torch.cuda.synchronize()
+        for r in range(n):
+            _assert_same(to_host(out[r]), want[r], f"mean {algo} N={n} rank {r}")
+    want_rs, _ = C.ring_reduce_scatter(xs, scale=inv)
+    shards = [torch.empty(cc.cc_chunk(count, n, c)[1], device="cuda") for c in range(n)]
+    cc.cc_reduce_scatter(send, shards, scale=None)
+    want_red, _ = C.reduce(xs, n - 1)
+    red = torch.empty(count, device="cuda")
+    cc.cc_reduce(send, red, n - 1, scale=None)
+    torch.cuda.synchronize()
+    for c in range(n):
+        _assert_same(to_host(shards[c]), want_rs[c], f"mean reduce-scatter N={n} shard {c}")
+    _assert_same(to_host(red), (want_red * np.float32(inv)).astype(np.float32), f"mean reduce N={n}")

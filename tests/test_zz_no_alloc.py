@@ -81,3 +81,46 @@ def test_noalloc_rejects_shapes_beyond_its_scratch():
     st = cc.lib.cc_alltoallv_noalloc(_pp(t), _pp(t), n, 16, _pp(ids), tokens, 2, epr, 16, 0, None,
                                      torch.cuda.current_stream().cuda_stream)
     assert st == cc.CC_ERR_INVALID_ARG
+
+
+def test_noalloc_with_no_tokens_reports_zero_rows():
+    """tokens = 0: nothing is copied; the receive counts come back as zeros (the scratch is
+    cleared by the call, whatever an earlier call left there)."""
+    n, epr = 4, 2
+    ids, tok = _case(n, 64, 16, epr, 5)  # an earlier call leaves non-zero tables in the scratch
+    got = [torch.zeros(64 * 2 * n, 16, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+    _noalloc(tok, got, ids, epr, 64 * 2 * n, 0, None)
+    empty_ids = [torch.zeros(1, 2, dtype=torch.int32, device="cuda") for _ in range(n)]
+    cnt = torch.full((n,), -1, dtype=torch.int32, device="cuda")
+    st = cc.lib.cc_alltoallv_noalloc(_pp(tok), _pp(got), n, 32, _pp(empty_ids), 0, 2, epr, 16, 0, cnt.data_ptr(),
+                                     torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert st == cc.CC_OK
+    assert cnt.tolist() == [0] * n
+
+
+def test_noalloc_accepts_the_largest_shape_that_fits_and_rejects_the_next():
+    """The 1 MiB limit at its edge: the largest token count whose routing scratch fits gives
+    exactly cc_alltoallv's result; one token more is rejected before anything runs."""
+    n, epr, hidden = 8, 8, 8
+    size = lambda t: cc.cc_alltoallv_workspace_size(n, t, 2, epr)
+    lo, hi = 1, 1 << 16
+    assert size(lo) <= (1 << 20) < size(hi)
+    while hi - lo > 1:  # the size grows with the token count
+        mid = (lo + hi) // 2
+        lo, hi = (mid, hi) if size(mid) <= (1 << 20) else (lo, mid)
+    ids, tok = _case(n, lo, hidden, epr, 6)
+    cap = lo * 2 * n
+    ws = torch.empty(size(lo) // 4 + 64, dtype=torch.int32, device="cuda")
+    ref = [torch.zeros(cap, hidden, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+    cc.cc_alltoallv(tok, ref, ids, epr, ws, direction=0)
+    got = [torch.zeros(cap, hidden, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+    _noalloc(tok, got, ids, epr, cap, 0, None)
+    torch.cuda.synchronize()
+    for d in range(n):
+        assert torch.equal(got[d].view(torch.int16), ref[d].view(torch.int16)), f"dispatch rank {d}"
+    ids2, tok2 = _case(n, hi, hidden, epr, 7)  # buffers sized for the larger shape
+    out2 = [torch.zeros(hi * 2, hidden, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+    st = cc.lib.cc_alltoallv_noalloc(_pp(tok2), _pp(out2), n, hidden * 2, _pp(ids2), hi, 2, epr, hi * 2, 0, None,
+                                     torch.cuda.current_stream().cuda_stream)
+    assert st == cc.CC_ERR_INVALID_ARG
