@@ -246,6 +246,66 @@ def hierarchical_allreduce(xs: Sequence[np.ndarray], ranks_per_node: int, *, op:
     return bufs, mesh
 
 
+# ---- multi-ring allreduce ---------------------------------------------------------------------
+# Lecture 09 §5.3: for large cross-node messages the library runs several rings side by side,
+# one per NIC rail. Reading (the page names the algorithm only): K rings; the message is cut
+# into K contiguous parts by the chunk rule (K parts) and ring k runs the ring allreduce of
+# §4.3 on part k, with the chunk rule over N inside the part. Even-numbered rings pass chunks
+# to rank r + 1 exactly as above; odd-numbered rings run the same schedule the other way round:
+# in reduce-scatter step s rank r sends chunk (r + s) mod N to rank r - 1, which folds it, so
+# chunk c completes on rank c + 1 and its allgather starts there. With K >= 2 both directions
+# of every link carry traffic. Chunk c of part k folds
+#   ((x_c (+) x_{c+1}) (+) ...) (+) x_{c-1}   for even k,
+#   ((x_c (+) x_{c-1}) (+) ...) (+) x_{c+1}   for odd k.
+# The rings touch disjoint elements and use their own message tags, so running them one
+# after another, as below, gives the same values and byte counts as running them side by side.
+
+def _ring_rs_dir(ctx, buf, sl, op, d, tag):
+    """Reduce-scatter phase of a ring whose chunks travel from rank r to rank r + d."""
+    r, n = ctx.rank, ctx.n
+    to, frm = (r + d) % n, (r - d) % n
+    for s in range(n - 1):
+        ctx.send(to, buf[sl[(r - d * s) % n]], tag=(tag, "rs", s))
+        c_in = (r - d * s - d) % n
+        incoming = yield from ctx.recv(frm, tag=(tag, "rs", s))
+        buf[sl[c_in]] = combine(buf[sl[c_in]], incoming, op)
+
+
+def _ring_ag_dir(ctx, buf, sl, d, tag):
+    """Allgather phase after _ring_rs_dir: rank r starts with chunk r + d, complete."""
+    r, n = ctx.rank, ctx.n
+    to, frm = (r + d) % n, (r - d) % n
+    for s in range(n - 1):
+        ctx.send(to, buf[sl[(r - d * s + d) % n]], tag=(tag, "ag", s))
+        c_in = (r - d * s) % n
+        buf[sl[c_in]] = yield from ctx.recv(frm, tag=(tag, "ag", s))
+
+
+def multiring_allreduce(xs: Sequence[np.ndarray], nrings: int, *, op: str = SUM, scale: float = 1.0,
+                        in_dtype: str = "f32", count: Optional[int] = None,
+                        positions: Optional[np.ndarray] = None, mesh: Optional[_MeshBase] = None):
+    n = len(xs)
+    if nrings < 1:
+        raise ValueError("at least one ring")
+    bufs = _prep(xs, in_dtype)
+    count = bufs[0].size if count is None else count
+    parts = chunk_bounds(count, nrings)
+    sls = [_local_slices([(a + p, a + q) for p, q in chunk_bounds(b - a, n)], positions) for a, b in parts]
+    mesh = mesh or LockstepMesh(n)
+
+    def program(ctx):
+        buf = bufs[ctx.rank]
+        for k in range(nrings):
+            d = 1 if k % 2 == 0 else -1
+            yield from _ring_rs_dir(ctx, buf, sls[k], op, d, ("mr", k))
+            own = sls[k][(ctx.rank + d) % n]
+            buf[own] = apply_scale(buf[own], scale)
+            yield from _ring_ag_dir(ctx, buf, sls[k], d, ("mr", k))
+
+    mesh.run(program)
+    return bufs, mesh
+
+
 # ---- double binary tree allreduce -------------------------------------------------------------
 # Lecture 09 §5.2 (reduce leaves -> root, then broadcast root -> leaves; 2 log2 N steps) and
 # the multi-node page §4.3.2 (two trees, one per half of the data). Shapes: layout.BinaryTree.

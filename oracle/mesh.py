@@ -68,6 +68,8 @@ class _MeshBase:
         # r // ranks_per_node == s // ranks_per_node; default: every rank is its own node)
         self.ranks_per_node = ranks_per_node or 1
         self.sent_off_node = [0] * n
+        # bytes per directed link (src, dst)
+        self.link_bytes: dict = defaultdict(int)
         self.messages = 0
         self.delivered = 0
         self._seq_out: dict = defaultdict(int)
@@ -77,6 +79,7 @@ class _MeshBase:
         if src != dst:
             self.sent[src] += int(payload.nbytes)
             self.recvd[dst] += int(payload.nbytes)
+            self.link_bytes[(src, dst)] += int(payload.nbytes)
             if src // self.ranks_per_node != dst // self.ranks_per_node:
                 self.sent_off_node[src] += int(payload.nbytes)
         self.messages += 1
