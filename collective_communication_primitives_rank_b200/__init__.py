@@ -48,6 +48,7 @@ _SIGS = {
     "cc_reduce_scatter": (_i, [_PP, _PP, _i, _sz, _i, _i, _i, _i, _f, _vp]),
     "cc_allreduce_stepped": (_i, [_PP, _PP, _i, _sz, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
     "cc_allreduce_hierarchical": (_i, [_PP, _PP, _i, _i, _sz, _i, _i, _i, _f, _vp]),
+    "cc_allreduce_multiring": (_i, [_PP, _PP, _i, _i, _sz, _i, _i, _i, _f, _vp]),
     "cc_allgather": (_i, [_PP, _PP, _i, _sz, _i, _vp]),
     "cc_broadcast": (_i, [_vp, _PP, _i, _i, _sz, _i, _vp]),
     "cc_reduce": (_i, [_PP, _vp, _i, _i, _sz, _i, _i, _i, _f, _vp]),
@@ -202,6 +203,19 @@ def cc_allreduce_hierarchical(send, recv, ranks_per_node: int, *, op="sum", scal
     _check(lib.cc_allreduce_hierarchical(_ptrs(send), _ptrs(recv), n, int(ranks_per_node), send[0].numel(),
                                          dtype_code(send[0]), dtype_code(recv[0]), _OPS[op], _scale(scale),
                                          _stream(stream)), "cc_allreduce_hierarchical")
+
+
+def cc_allreduce_multiring(send, recv, nrings: int, *, op="sum", scale=1.0, stream=None) -> None:
+    """recv[r] = what nrings rings side by side leave (part k of the buffer on ring k, odd
+    rings in the opposite direction), times scale."""
+    n = _ranks(send, "cc_allreduce_multiring")
+    _same(send, send[0].numel(), send[0].dtype, "cc_allreduce_multiring send")
+    _same(recv, send[0].numel(), recv[0].dtype, "cc_allreduce_multiring recv")
+    if len(recv) != n:
+        raise ValueError("cc_allreduce_multiring: one output per rank")
+    _check(lib.cc_allreduce_multiring(_ptrs(send), _ptrs(recv), n, int(nrings), send[0].numel(), dtype_code(send[0]),
+                                      dtype_code(recv[0]), _OPS[op], _scale(scale), _stream(stream)),
+           "cc_allreduce_multiring")
 
 
 def cc_allreduce_stepped(send, recv, workspace, *, op="sum", algo="ring", scale=1.0, stream=None) -> None:

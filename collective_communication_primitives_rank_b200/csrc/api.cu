@@ -336,6 +336,18 @@ cc_status cc_allreduce_hierarchical(const void* const* send, void* const* recv, 
                                    resolve_scale(scale, nranks), as_stream(stream)));
 }
 
+cc_status cc_allreduce_multiring(const void* const* send, void* const* recv, int nranks, int nrings, size_t count,
+                                 cc_dtype in_t, cc_dtype out_t, cc_op op, float scale, void* stream) {
+  if (!valid_ranks(nranks) || !send || !recv || nrings < 1 || nrings > CC_MAX_RINGS) return CC_ERR_INVALID_ARG;
+  if (cc_status st = check_reduce(in_t, out_t, op, scale)) return st;
+  if (count == 0) return CC_OK;
+  if (!all_nonnull(send, nranks) || !all_nonnull((const void* const*)recv, nranks)) return CC_ERR_INVALID_ARG;
+  for (int r = 0; r < nranks; ++r)
+    if (recv[r] == send[r] && dtype_bytes(in_t) != dtype_bytes(out_t)) return CC_ERR_INVALID_ARG;
+  return cuda_status(launch_reduce(send, recv, nranks, nranks, count, in_t, op, kFoldMultiRing, kAllReduce, nrings,
+                                   resolve_scale(scale, nranks), as_stream(stream)));
+}
+
 cc_status cc_reduce_scatter(const void* const* send, void* const* recv, int nranks, size_t count, cc_dtype in_t,
                             cc_dtype out_t, cc_op op, cc_algo algo, float scale, void* stream) {
   if (!valid_ranks(nranks) || !send || !recv) return CC_ERR_INVALID_ARG;

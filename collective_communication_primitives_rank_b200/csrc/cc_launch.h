@@ -12,9 +12,10 @@ namespace cc {
 
 // Reduction family: allreduce, reduce-scatter, reduce-to-root.
 enum ReduceMode { kAllReduce = 0, kReduceScatter = 1, kReduceRoot = 2 };
-enum FoldKind { kFoldRing = 0, kFoldTree = 1, kFoldBinomial = 2, kFoldHier = 3 };
+enum FoldKind { kFoldRing = 0, kFoldTree = 1, kFoldBinomial = 2, kFoldHier = 3, kFoldMultiRing = 4 };
 
-// `root` is the root rank for kFoldBinomial and the ranks per node for kFoldHier; only the
+// `root` is the root rank for kFoldBinomial, the ranks per node for kFoldHier and the number
+// of rings for kFoldMultiRing; only the
 // elements [lo, hi) of the count are folded and written (the whole buffer by default).
 cudaError_t launch_reduce(const void* const* send, void* const* dst, int ndst, int nranks,
                           size_t count, cc_dtype in_t, cc_op op, FoldKind fold, ReduceMode mode,

@@ -166,7 +166,13 @@ __global__ void __launch_bounds__(32) copy_bulk_tile_kernel(const __grid_constan
     mbar_arrive_tx(bar, bulk);
     bulk_load(smem, P.src[k] + a, bulk, bar);
     if (!mbar_wait(bar, 0)) {
-      mbar_wait(bar, 0);  // one more bounded chance for the load to land before leaving
+      // one more bounded chance for the load to land before leaving. If it still has not,
+      // the CTA leaves with the bulk load in flight: that load may still write this CTA's
+      // shared memory after the SM has handed it to another CTA (of this or any kernel),
+      // so the outputs of this call and of whatever runs next on that SM are undefined; the
+      // status word reads CC_ERR_TIMEOUT (only a memory system that stalls a 32 KiB read for
+      // seconds gets here)
+      mbar_wait(bar, 0);
       return;
     }
   }
@@ -183,14 +189,18 @@ __global__ void __launch_bounds__(32) copy_bulk_tile_kernel(const __grid_constan
 static bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 int* async_status_word() {
+  // looked up with the device current; only a successful lookup is kept, so a failed one
+  // (for instance during a stream capture) is retried by the next call
   static int* ptr[64];
-  static std::once_flag once[64];
+  static std::mutex mu[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::call_once(once[dev], [dev] {
+  std::lock_guard<std::mutex> lock(mu[dev]);
+  if (!ptr[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_async_status) == cudaSuccess) ptr[dev] = static_cast<int*>(p);
-  });
+    else cudaGetLastError();
+  }
   return ptr[dev];
 }
 

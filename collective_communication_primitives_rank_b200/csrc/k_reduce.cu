@@ -13,6 +13,8 @@
 //   ring      chunk c folds ((x_c (+) x_{c+1}) (+) ...) (+) x_{c-1}
 //   tree      half A / half B fold over tree A / tree B, ((S_left (+) x) (+) S_right)
 //   binomial  node v folds x_v, then each child's partial in send order
+//   multi-ring  part k of K (chunk rule), chunk c inside it: the ring fold starting at rank c,
+//             walking up the ranks for even k and down for odd k (lecture 09 §5.3)
 #include <algorithm>
 #include <mutex>
 #include <vector>
@@ -241,7 +243,8 @@ __device__ __forceinline__ int chunk_of(uint64_t count, int n, uint64_t o, uint6
 }
 
 // The fold group of element o in a buffer of `count` elements: the ring chunk, the tree
-// half, or the single binomial group; returns the group and its [start, end).
+// half, the (part, chunk) pair of the multi-ring, or the single binomial group; returns the
+// group and its [start, end).
 __device__ __forceinline__ int group_of(int fold, uint64_t count, int n, uint64_t o, uint64_t& start,
                                         uint64_t& end, int per_node = 1) {
   if (fold == kFoldRing) return chunk_of(count, n, o, start, end);
@@ -254,6 +257,16 @@ __device__ __forceinline__ int group_of(int fold, uint64_t count, int n, uint64_
     start = ca + ja;
     end = ca + jb;
     return c * M + j;
+  }
+  if (fold == kFoldMultiRing) {
+    // part k of the K rings' split, then chunk c of that part's N-way split; group k * n + c
+    const int K = per_node;
+    uint64_t pa, pb, ca, cb;
+    const int k = chunk_of(count, K, o, pa, pb);
+    const int c = chunk_of(pb - pa, n, o - pa, ca, cb);
+    start = pa + ca;
+    end = pa + cb;
+    return k * n + c;
   }
   if (fold == kFoldTree) {
     const uint64_t mid = (count + 1) / 2;
@@ -319,7 +332,8 @@ __global__ void __launch_bounds__(kThreads, KIND == kLinear ? CC_RING_MIN_BLOCKS
         const int rk = P.prog.rmap[p];
         return mirror ? n - 1 - rk : rk;
       };
-      const bool shard_vec = ((P.dst_aligned >> g) & 1) && ((ga * sizeof(Out)) % 16 == 0);
+      const bool shard_vec = mode == kReduceScatter && ((P.dst_aligned >> (g & 63)) & 1) &&
+                             ((ga * sizeof(Out)) % 16 == 0);
       auto emit_unit = [&](uint64_t e, Unit<IN> u) {
         if (P.do_scale) scale_unit<IN>(u, P.scale);
         if (mode == kAllReduce) {
@@ -341,11 +355,14 @@ __global__ void __launch_bounds__(kThreads, KIND == kLinear ? CC_RING_MIN_BLOCKS
           store_elem<IN>(static_cast<Out*>(P.dst[0]) + e, v);
         }
       };
-      // linear folds: a ring chunk starts at rank g and walks up; a linear tree (g = 0 or 1
-      // for tree A / B) starts at rank 0 and walks up, or at rank n-1 and walks down; a
-      // linear binomial program starts at the root and walks up
-      const int lstart = P.fold == kFoldRing ? g : P.fold == kFoldTree ? (g == 0 ? 0 : n - 1) : P.prog.rmap[0];
-      const bool lup = P.fold != kFoldTree || g == 0;
+      // linear folds: a ring chunk starts at rank g and walks up; a multi-ring chunk (group
+      // k * n + c) starts at rank c and walks up for even k, down for odd k; a linear tree
+      // (g = 0 or 1 for tree A / B) starts at rank 0 and walks up, or at rank n-1 and walks
+      // down; a linear binomial program starts at the root and walks up
+      const int lstart = P.fold == kFoldRing ? g
+                         : P.fold == kFoldMultiRing ? g % n
+                         : P.fold == kFoldTree ? (g == 0 ? 0 : n - 1) : P.prog.rmap[0];
+      const bool lup = P.fold == kFoldMultiRing ? ((g / n) % 2 == 0) : (P.fold != kFoldTree || g == 0);
       reduce_range<IN, OP, KIND>(n, g, rank_of, P.prog, s, se, threadIdx.x, blockDim.x, P.vec != 0, src,
                                     emit_unit, emit_elem, s_stk + threadIdx.x, lstart, lup, G, hc, hj);
       s = se;
@@ -631,7 +648,8 @@ static cudaError_t run_reduce(ReduceParams& P, cudaStream_t s) {
   // buffer (N ring chunks of a few elements each) are folded by different CTAs in parallel
   const uint64_t ngroups = P.fold == kFoldRing ? (uint64_t)P.nranks
                            : P.fold == kFoldTree ? 2
-                           : P.fold == kFoldHier ? (uint64_t)P.nranks : 1;
+                           : P.fold == kFoldHier ? (uint64_t)P.nranks
+                           : P.fold == kFoldMultiRing ? (uint64_t)P.nranks * P.per_node : 1;
   const uint64_t per_group = ((P.count + ngroups - 1) / ngroups + 7) / 8 * 8;
   // units per thread and tile (measured): the linear folds (ring, linear tree, hierarchical)
   // run best with about 24 memory operations per thread and CTA (a unit costs N loads plus
@@ -709,14 +727,14 @@ cudaError_t launch_reduce(const void* const* send, void* const* dst, int ndst, i
   P.per_node = 1;
   if (fold == kFoldTree) tree_program(nranks, P.prog);
   else if (fold == kFoldBinomial) binomial_program(nranks, root, P.prog);
-  else if (fold == kFoldHier) P.per_node = root;
+  else if (fold == kFoldHier || fold == kFoldMultiRing) P.per_node = root;
   // the ring, a tree whose fold is a plain left fold (N <= 5) and a binomial program that is
   // one (N <= 3, ranks in order from the root) run the linear fold; the hierarchical fold has
   // its own nested loop; other programs run the fold machine with the smallest stack that
   // holds their pending partials (more resident CTAs for smaller stacks)
   int kind = kMachine;
-  if (fold == kFoldRing || fold == kFoldHier) {
-    kind = fold == kFoldRing ? kLinear : kHier;
+  if (fold == kFoldRing || fold == kFoldMultiRing || fold == kFoldHier) {
+    kind = fold == kFoldHier ? kHier : kLinear;
   } else if (program_is_rotation(nranks, P.prog)) {
     kind = kLinear;
   } else {

@@ -84,7 +84,10 @@ CC_API int cc_version(void);
  * calls waits on shared-memory barriers with an iteration limit). Synchronizes `stream`,
  * then returns CC_OK, or CC_ERR_TIMEOUT if a wait gave up since the last reset (the outputs
  * of that call are then incomplete); `reset` != 0 clears the status. CC_ERR_CUDA if the
- * device cannot be read. */
+ * device cannot be read. A data-movement call whose tile load timed out (twice 2 s) leaves
+ * with that load still in flight: its late write may land in shared memory the SM has
+ * since given to other work, so results computed on that device after the timeout are
+ * undefined as well; recreate the context before trusting it again. */
 CC_API cc_status cc_async_status(int reset, void* stream);
 
 /* Self-test of the device-side bounded waits: launches one thread that waits on a
@@ -139,6 +142,21 @@ CC_API cc_status cc_allreduce_stepped(const void* const* send, void* const* recv
 CC_API cc_status cc_allreduce_hierarchical(const void* const* send, void* const* recv, int nranks,
                                            int ranks_per_node, size_t count, cc_dtype in_t,
                                            cc_dtype out_t, cc_op op, float scale, void* stream);
+
+/* Multi-ring AllReduce (lecture 09 §5.3: for large cross-node messages several rings run
+ * side by side, one per NIC rail). The result is what this schedule leaves on every rank:
+ * the count elements are cut into nrings contiguous parts (chunk rule with nrings parts),
+ * and ring k runs the ring allreduce of cc_allreduce on part k (chunk rule with N parts
+ * inside the part); even-numbered rings pass chunks to rank r + 1, odd-numbered rings run the
+ * same schedule towards rank r - 1, so that with two or more rings both directions of every
+ * link carry traffic. Chunk c of part k folds ((x_c (+) x_{c+1}) (+) ...) (+) x_{c-1} for even
+ * k and ((x_c (+) x_{c-1}) (+) ...) (+) x_{c+1} for odd k; then `scale`. One fused pass (N·T
+ * in, N·T out). nrings in [1, CC_MAX_RINGS] (else CC_ERR_INVALID_ARG); 1 gives
+ * cc_allreduce's ring. Other arguments as cc_allreduce (in place allowed). */
+#define CC_MAX_RINGS 64
+CC_API cc_status cc_allreduce_multiring(const void* const* send, void* const* recv, int nranks, int nrings,
+                                        size_t count, cc_dtype in_t, cc_dtype out_t, cc_op op, float scale,
+                                        void* stream);
 
 /* ReduceScatter (lecture 09 §3.6; the from-scratch page's reduce_scatter as the first
  * half of the ring). Rank c receives, in recv[c], chunk c (chunk rule) of the ring

@@ -148,3 +148,11 @@ def test_packed_detection_for_the_host_pipeline():
     assert cc._packed(views, separate) == 0
     mixed = [[flat[0][0:30], torch.zeros(70)], [flat[1][0:30], flat[1][30:100]]]
     assert cc._packed(mixed) == 0
+
+
+def test_multiring_ring_count_is_validated(lib):
+    p = _pp(FAKE[:4])
+    for k in (0, 65, -1):
+        assert lib.cc_allreduce_multiring(p, p, 4, k, 10, cc.CC_F32, cc.CC_F32, cc.CC_SUM, 1.0, None) == \
+            cc.CC_ERR_INVALID_ARG
+    assert lib.cc_allreduce_multiring(p, p, 4, 2, 0, cc.CC_F32, cc.CC_F32, cc.CC_SUM, 1.0, None) == cc.CC_OK

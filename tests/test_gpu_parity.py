@@ -332,3 +332,63 @@ def test_scale_mean_sentinel_equals_explicit_reciprocal(n):
     for c in range(n):
         _assert_same(to_host(shards[c]), want_rs[c], f"mean reduce-scatter N={n} shard {c}")
     _assert_same(to_host(red), (want_red * np.float32(inv)).astype(np.float32), f"mean reduce N={n}")
+
+
+# ---- multi-ring allreduce: K rings side by side, odd rings reversed ---------------------------------------
+
+@pytest.mark.parametrize("n,K,count", [(2, 2, 4096 + 3), (3, 2, 1001), (4, 3, 4096), (8, 2, 8 * 4096), (8, 4, 999),
+                                       (13, 3, 2000), (16, 5, 65536 + 17), (64, 2, 64 * 40), (64, 4, 70), (8, 64, 1000),
+                                       (5, 1, 777)])
+@pytest.mark.parametrize("kind", ["spread", "i32", "bf16"])
+def test_multiring_allreduce_matches_oracle(n, K, count, kind):
+    xs = _inputs(kind, n, count, seed=60)
+    scale = 1.0 if kind == "i32" else 1.0 / n
+    want, _ = C.multiring_allreduce(xs, K, in_dtype=_IN[kind], scale=scale)
+    out = [Guarded(count, _out_dtype(kind)) for _ in range(n)]
+    cc.cc_allreduce_multiring([to_dev(x) for x in xs], [o.t for o in out], K, scale=scale)
+    torch.cuda.synchronize()
+    for r in range(n):
+        _assert_same(to_host(out[r].t), want[r], f"multi-ring {kind} N={n} K={K} rank {r}")
+        out[r].check()
+
+
+def test_multiring_in_place_misaligned_and_large_sampled():
+    n, K, count = 8, 4, 16 * 1024 * 1024 + 5
+    xs = [synth.uniform_f32(61, r, count) for r in range(n)]
+    buf = [to_dev(x) for x in xs]
+    cc.cc_allreduce_multiring(buf, buf, K, scale=0.125)
+    torch.cuda.synchronize()
+    pos = np.unique(np.concatenate([[0, count - 1], np.arange(7, count, 4093)]))
+    want, _ = C.multiring_allreduce([x[pos] for x in xs], K, scale=0.125, count=count, positions=pos)
+    idx = torch.from_numpy(pos).cuda()
+    for r in (0, 5, n - 1):
+        _assert_same(buf[r][idx].cpu().numpy(), want[r], f"multi-ring in place rank {r}")
+    small = _inputs("spread", 6, 3001, seed=62)
+    want_s, _ = C.multiring_allreduce(small, 3)
+    mis = [misaligned(x) for x in small]
+    mout = [misaligned(np.zeros_like(x)) for x in small]
+    cc.cc_allreduce_multiring(mis, mout, 3)
+    torch.cuda.synchronize()
+    for r in range(6):
+        _assert_same(to_host(mout[r]), want_s[r], f"multi-ring misaligned rank {r}")
+
+
+@pytest.mark.parametrize("n,count,kind", [(8, 8 * 1024 * 1024 + 5, "f32"), (3, 4 * 1024 * 1024 + 1, "bf16"),
+                                          (64, 64 * 65536 + 63, "i32"), (2, 6 * 1024 * 1024, "f32")])
+@pytest.mark.parametrize("algo", ["ring", "tree"])
+def test_stepped_large_messages_sampled(n, count, kind, algo):
+    """Messages whose phases run on the tile path (more units than the resident grid has
+    threads), checked on sampled positions against the oracle's full-size chunk map."""
+    xs = _inputs(kind, n, count, seed=17)
+    ws = torch.zeros(64, dtype=torch.int32, device="cuda")
+    out = [torch.empty(count, dtype=_out_dtype(kind), device="cuda") for _ in range(n)]
+    scale = 1.0 if kind == "i32" else 0.5
+    cc.cc_allreduce_stepped([to_dev(x) for x in xs], out, ws, algo=algo, scale=scale)
+    torch.cuda.synchronize()
+    assert cc.cc_async_status() == cc.CC_OK
+    pos = np.unique(np.concatenate([[0, 1, 2, 3, count - 1], np.arange(5, count, 2039)]))
+    fn = C.ring_allreduce if algo == "ring" else C.tree_allreduce
+    want, _ = fn([x[pos] for x in xs], in_dtype=_IN[kind], scale=scale, count=count, positions=pos)
+    idx = torch.from_numpy(pos).cuda()
+    for r in sorted({0, n // 2, n - 1}):
+        _assert_same(out[r][idx].cpu().numpy(), want[r], f"stepped {algo} {kind} N={n} rank {r}")
