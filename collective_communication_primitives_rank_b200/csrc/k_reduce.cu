@@ -159,11 +159,100 @@ __device__ __forceinline__ void linear_fold_units(int n, int start, bool up, uin
   }
 }
 
+// Binomial reduce programs compiled for a fixed rank count: the pre-order walk of the
+// binomial tree (relative rank v; children v + 2^k for every 2^k > v, in send order) with the
+// fold-machine code of every position, computed at compile time, so that a fully unrolled
+// fold resolves every code and keeps the pending partials in registers. The same walk and
+// codes as binomial_program() below builds at run time for any rank count.
+template <int NB> struct BinomialPlan {
+  uint8_t order[NB];
+  uint8_t code[NB];
+  int depth;
+  constexpr BinomialPlan() : order(), code(), depth(0) {
+    int stack[NB] = {};
+    int sp = 0, pos = 0;
+    stack[sp++] = 0;
+    while (sp > 0) {
+      const int v = stack[--sp];
+      order[pos++] = (uint8_t)v;
+      int k = 0;
+      if (v) while ((1 << k) <= v) ++k;
+      int ch[8] = {}, nch = 0;
+      for (; v + (1 << k) < NB; ++k) ch[nch++] = v + (1 << k);
+      for (int c = nch - 1; c >= 0; --c) stack[sp++] = ch[c];
+    }
+    int d = 0;
+    for (int p = 0; p < NB; ++p) {
+      const int v = order[p];
+      int k = 0;
+      if (v) while ((1 << k) <= v) ++k;
+      const bool leaf = !(v + (1 << k) < NB);
+      uint8_t c = 0;
+      if (!leaf) {
+        c = kPush;
+        if (++d > depth) depth = d;
+      } else {
+        int npop = 0, u = v;
+        while (u != 0) {
+          int hb = 0;
+          while ((2 << hb) <= u) ++hb;
+          const int par = u - (1 << hb);
+          int kk = 0;
+          if (par) while ((1 << kk) <= par) ++kk;
+          int last = -1;
+          for (; par + (1 << kk) < NB; ++kk) last = par + (1 << kk);
+          if (last == u) { ++npop; u = par; continue; }
+          c |= kFoldTop;
+          break;
+        }
+        c |= (uint8_t)(npop << 2);
+        d -= npop;
+      }
+      code[p] = c;
+    }
+  }
+};
+
+// NU units (or elements) at once, each folded over the NB ranks in the compiled binomial
+// order from `root`: the loads of a window of 8 positions of every unit go out before the
+// folds that consume them.
+template <int IN, int OP, int NB, int NU, typename V, typename X, typename Load, typename Widen>
+__device__ __forceinline__ void binomial_fold_ct(int root, Load ld, Widen widen, V (&cur)[NU]) {
+  constexpr BinomialPlan<NB> plan{};
+  constexpr int S = plan.depth > 0 ? plan.depth : 1;
+  FoldStack<V, S> st[NU];
+#pragma unroll
+  for (int i = 0; i < NU; ++i) st[i].depth = 0;
+#pragma unroll
+  for (int p0 = 0; p0 < NB; p0 += 8) {
+    X x[NU][8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (p0 + k < NB) {
+        int r = plan.order[p0 + k] + root;
+        if (r >= NB) r -= NB;
+#pragma unroll
+        for (int i = 0; i < NU; ++i) x[i][k] = ld(i, r);
+      }
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (p0 + k < NB)
+#pragma unroll
+        for (int i = 0; i < NU; ++i) fold_step<IN, OP>(plan.code[p0 + k], widen(x[i][k]), cur[i], st[i]);
+  }
+}
+
 // KIND: kLinear (ring order or a linear tree), kMachine (tree / binomial programs),
 // kHier (two-level), kShallow / kMid (the fold machine with 2 / 4 stack slots, for programs
 // that never hold more pending partials), kLinSmall (the linear fold of 2 ranks, four units
 // per iteration); hG / hc / hj describe the hierarchical group.
 constexpr int kLinear = 0, kMachine = 1, kHier = 2, kShallow = 3, kMid = 4, kLinSmall = 5;
+// binomial programs compiled for 4, 8, 16, 32, 64 ranks (SUM only): kBinom4 + log2(N / 4)
+constexpr int kBinom4 = 10, kBinom8 = 11, kBinom16 = 12, kBinom32 = 13, kBinom64 = 14;
+__host__ __device__ constexpr bool is_binom_ct(int kind) { return kind >= kBinom4 && kind <= kBinom64; }
+__host__ __device__ constexpr int binom_ct_ranks(int kind) { return 4 << (kind - kBinom4); }
+// units folded at once: about 16 loads in flight per thread for the small rank counts
+__host__ __device__ constexpr int binom_ct_units(int kind) { return kind == kBinom4 ? 4 : kind == kBinom8 ? 2 : 1; }
 
 template <int IN, int OP, int KIND, typename RankOf, typename Src, typename EmitU, typename EmitE>
 __device__ __forceinline__ void reduce_range(int n, int g, RankOf rank_of, const FoldProgram& prog,
@@ -180,6 +269,11 @@ __device__ __forceinline__ void reduce_range(int n, int g, RankOf rank_of, const
     auto ld = [&](int r) { return load_elem<IN>(src(r) + e); };
     if constexpr (RING) return ring_fold<IN, OP, A, A>(n, start, ld, same, up);
     else if constexpr (KIND == kHier) return hier_fold<IN, OP, A, A>(n, hG, hc, hj, ld, same);
+    else if constexpr (is_binom_ct(KIND)) {
+      A cur[1];
+      binomial_fold_ct<IN, OP, binom_ct_ranks(KIND), 1, A, A>(start, [&](int, int r) { return ld(r); }, same, cur);
+      return cur[0];
+    }
     else {
       FoldStack<A, SLOTS> st;
       return machine_fold<IN, OP, A, A, 8>(n, prog, rank_of, ld, same, st);
@@ -196,6 +290,22 @@ __device__ __forceinline__ void reduce_range(int n, int g, RankOf rank_of, const
     if constexpr (KIND == kLinSmall) {  // two ranks: four units per iteration
       for (uint64_t e0 = va + t * UE; e0 < vb; e0 += 4 * step)
         linear_fold_units<IN, OP, 2, 4>(n, start, up, e0, step, vb, src, emit_unit);
+      done = true;
+    }
+    if constexpr (is_binom_ct(KIND)) {  // compiled binomial program, NU units per iteration
+      constexpr int NU = binom_ct_units(KIND);
+      for (uint64_t e0 = va + t * UE; e0 < vb; e0 += NU * step) {
+        // a unit past vb re-reads the last whole unit and is not emitted
+        auto ld = [&](int i, int r) {
+          const uint64_t e = e0 + i * step < vb ? e0 + i * step : vb - UE;
+          return load_raw(src(r) + e);
+        };
+        Unit<IN> m[NU];
+        binomial_fold_ct<IN, OP, binom_ct_ranks(KIND), NU, Unit<IN>, uint4>(start, ld, widen, m);
+#pragma unroll
+        for (int i = 0; i < NU; ++i)
+          if (e0 + i * step < vb) emit_unit(e0 + i * step, m[i]);
+      }
       done = true;
     }
     for (uint64_t e0 = va + t * UE; !done && e0 < vb; e0 += step) {
@@ -305,6 +415,7 @@ struct ReduceParams {
 template <int IN, int OP, int KIND>
 __global__ void __launch_bounds__(kThreads, KIND == kLinear ? CC_RING_MIN_BLOCKS
                                            : KIND == kLinSmall ? CC_LINSMALL_MIN_BLOCKS
+                                           : is_binom_ct(KIND) ? (binom_ct_units(KIND) > 1 ? 2 : KIND == kBinom64 ? 3 : 4)
                                            : KIND == kHier ? 3
                                            : KIND == kShallow || KIND == kMid ? CC_SHALLOW_MIN_BLOCKS
                                                                               : CC_MACHINE_MIN_BLOCKS)
@@ -680,6 +791,13 @@ static cudaError_t dispatch_op(ReduceParams& P, cc_op op, int kind, cudaStream_t
   if (kind == kShallow) return run_reduce<IN, OPV, kShallow>(P, s);                       \
   if (kind == kMid) return run_reduce<IN, OPV, kMid>(P, s);                               \
   return run_reduce<IN, OPV, kMachine>(P, s);
+  switch (kind) {  // compiled binomial programs: SUM only (launch_reduce picks them for SUM)
+    case kBinom4: return run_reduce<IN, CC_SUM, kBinom4>(P, s);
+    case kBinom8: return run_reduce<IN, CC_SUM, kBinom8>(P, s);
+    case kBinom16: return run_reduce<IN, CC_SUM, kBinom16>(P, s);
+    case kBinom32: return run_reduce<IN, CC_SUM, kBinom32>(P, s);
+    case kBinom64: return run_reduce<IN, CC_SUM, kBinom64>(P, s);
+  }
   switch (op) {
     case CC_SUM: CC_KINDS(CC_SUM)
     case CC_MAX: CC_KINDS(CC_MAX)
@@ -746,6 +864,9 @@ cudaError_t launch_reduce(const void* const* send, void* const* dst, int ndst, i
   // N = 2 × 256 MiB: ring 5667 -> 6663 GB/s, reduce-scatter 5399 -> 6832; at N = 3..4 the
   // one-unit fold with 4 resident CTAs is faster)
   if (kind == kLinear && nranks == 2) kind = kLinSmall;
+  // binomial sums at 4, 8, 16, 32, 64 ranks run their program compiled to straight-line code
+  if (fold == kFoldBinomial && op == CC_SUM && kind != kLinear && (nranks & (nranks - 1)) == 0 && nranks >= 4)
+    kind = kBinom4 + __builtin_ctz((unsigned)nranks) - 2;
   switch (in_t) {
     case CC_F32: return dispatch_op<CC_F32>(P, op, kind, stream);
     case CC_BF16: return dispatch_op<CC_BF16>(P, op, kind, stream);

@@ -22,16 +22,17 @@
 // 16-byte units into tiles of kStepThreads x kUnits units that never cross a job; CTAs take
 // tiles in turn, and a thread issues the loads of its kUnits units before any fold or store;
 // element-wise heads and tails (ranges that do not start or end on a 16-byte boundary) are
-// done by the first tile of the job. Small phases (at most one unit per thread of the grid)
-// give every thread one slot of the flattened (job, unit) space instead, the last slot of a
-// job taking its head and tail, so a phase costs one dependent load-store round trip.
+// done by the first tile of the job. Small phases (when one slot per unit fits the resident
+// grid) give every thread up to kUnits slots of the flattened (job, unit) space per round,
+// the last slot of a job taking its head and tail, with the loads of every slot issued before
+// the first fold, so a phase costs one or two dependent load-store round trips.
 //
 // Grid. The launch is cooperative (all CTAs resident). A small phase takes as many CTAs as
-// its slots need, so a message of a few hundred units runs on one CTA, whose barrier is
-// __syncthreads(); a large one about kTilesPerCta tiles per CTA, at most the resident CTAs.
-// Between phases of a multi-CTA grid the barrier is a monotonic counter in the caller's
-// workspace; waits are bounded by time: a barrier that does not complete within 2 s records
-// CC_ERR_TIMEOUT in the device status word and every CTA leaves.
+// its slots need (kTileUnits slots per CTA), and one CTA when that is one or two, whose
+// barrier is __syncthreads(); a large one about kTilesPerCta tiles per CTA, at most the
+// resident CTAs. Between phases of a multi-CTA grid the barrier is a monotonic counter in the
+// caller's workspace; waits are bounded by time: a barrier that does not complete within 2 s
+// records CC_ERR_TIMEOUT in the device status word and every CTA leaves.
 #include <algorithm>
 #include <vector>
 
@@ -58,7 +59,7 @@ struct StepParams {
   uint64_t chunk_q, chunk_r;               // count / N, count % N
   uint64_t tiles_per_job;                  // large phases: tiles covering the longest job
   uint64_t slots_per_job;                  // small phases: unit slots per job (+1 for head and tail)
-  int small;                               // every phase is small (one slot per thread)
+  int small;                               // the small-phase kernel runs (slots rather than tiles)
   unsigned* barrier;
   int* status;  // the library's device status word
   int nranks;
@@ -93,6 +94,7 @@ __device__ __forceinline__ bool phase_barrier(unsigned* counter, int* status, un
     atomicAdd(counter, 1u);
     const unsigned target = (phase + 1) * gridDim.x;
     const uint64_t t0 = now_ns();
+    int polls = 0;
     for (;;) {
       unsigned v;
       asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
@@ -102,7 +104,7 @@ __device__ __forceinline__ bool phase_barrier(unsigned* counter, int* status, un
         s_abort = 1;
         break;
       }
-      __nanosleep(64);
+      if (++polls > 256) __nanosleep(128);  // poll back-to-back first: a phase ends within microseconds
     }
     __threadfence();
   }
@@ -218,8 +220,8 @@ __device__ __forceinline__ void job_units(const StepParams& P, const Job& j, uin
   }
 }
 
-template <int IN, int OP>
-__global__ void __launch_bounds__(kStepThreads) stepped_kernel(const __grid_constant__ StepParams P) {
+template <int IN, int OP, bool SMALL>
+__global__ void __launch_bounds__(kStepThreads, SMALL ? 1 : 3) stepped_kernel(const __grid_constant__ StepParams P) {
   using In = typename Tr<IN>::In;
   constexpr int OT = IN == CC_I32 ? CC_I32 : CC_F32;  // the buffers hold 4-byte fp32 / int32
   using V = typename Tr<OT>::Acc;
@@ -263,26 +265,71 @@ __global__ void __launch_bounds__(kStepThreads) stepped_kernel(const __grid_cons
   const uint64_t tpj = P.tiles_per_job, spj = P.slots_per_job;
   for (int ph = 0; ph < P.phases; ++ph) {
     const uint32_t njobs = (uint32_t)phase_jobs(P, ph);
-    if (P.small) {
-      // one slot per thread: unit u of job k, or (the last slot) the job's head and tail
-      for (uint64_t f = tid; f < njobs * spj; f += T) {
-        const uint32_t k = (uint32_t)f / (uint32_t)spj;
-        const uint64_t u = f - (uint64_t)k * spj;
-        const Job j = phase_job(P, ph, (int)k);
-        if (P.vec) {
+    if constexpr (SMALL) {
+      // slots f0 + i*T (i < kUnits) per round: unit u of job k, or (the job's last slot) its
+      // head and tail; every unit slot's loads are issued before the first fold
+      const uint64_t nslots = (uint64_t)njobs * spj;
+      for (uint64_t f0 = tid; f0 < nslots; f0 += T * kUnits) {
+        V* dp[kUnits];
+        const V* lp[kUnits];
+        const V* rp[kUnits];
+        int fl[kUnits];  // bit 0: a unit to fold, bit 1: copy, bit 2: scale
+        uint4 xd[kUnits], xl[kUnits], xr[kUnits];
+#pragma unroll
+        for (int i = 0; i < kUnits; ++i) {
+          fl[i] = 0;
+          dp[i] = nullptr;
+          lp[i] = rp[i] = nullptr;
+          const uint64_t f = f0 + (uint64_t)i * T;
+          if (f >= nslots) continue;
+          const uint32_t k = (uint32_t)f / (uint32_t)spj;
+          const uint64_t u = f - (uint64_t)k * spj;
+          const Job j = phase_job(P, ph, (int)k);
+          if (!P.vec) {
+            if (j.a + u < j.b) job_elem<OT, OP>(P, j, j.a + u);
+            continue;
+          }
           uint64_t va = (j.a + UE - 1) / UE * UE;
           if (va > j.b) va = j.b;
           uint64_t vb = j.b / UE * UE;
           if (vb < va) vb = va;
-          const uint64_t nu = (vb - va) / UE;
-          if (u < nu) {
-            job_units<OT, OP>(P, j, va + u * UE, 0, va + u * UE + UE, 1);
+          if (u < (vb - va) / UE) {
+            const uint64_t e = va + u * UE;
+            dp[i] = static_cast<V*>(P.buf[j.dst]) + e;
+            if (j.l >= 0) lp[i] = static_cast<const V*>(P.buf[j.l]) + e;
+            if (j.r >= 0) rp[i] = static_cast<const V*>(P.buf[j.r]) + e;
+            fl[i] = 1 | (j.copy ? 2 : 0) | (j.scale ? 4 : 0);
           } else if (u == spj - 1) {
             for (uint64_t e = j.a; e < va; ++e) job_elem<OT, OP>(P, j, e);
             for (uint64_t e = vb; e < j.b; ++e) job_elem<OT, OP>(P, j, e);
           }
-        } else if (j.a + u < j.b) {
-          job_elem<OT, OP>(P, j, j.a + u);
+        }
+#pragma unroll
+        for (int i = 0; i < kUnits; ++i) {
+          if (!(fl[i] & 1)) continue;
+          if (!(fl[i] & 2)) xd[i] = __ldcg(reinterpret_cast<const uint4*>(dp[i]));
+          if (lp[i]) xl[i] = __ldcg(reinterpret_cast<const uint4*>(lp[i]));
+          if (rp[i]) xr[i] = __ldcg(reinterpret_cast<const uint4*>(rp[i]));
+        }
+#pragma unroll
+        for (int i = 0; i < kUnits; ++i) {
+          if (!(fl[i] & 1)) continue;
+          uint4 out;
+          if (fl[i] & 2) {
+            out = xl[i];
+          } else {
+            Unit<OT> x = to_unit<OT>(xd[i]);
+            if (lp[i]) {
+              Unit<OT> y = to_unit<OT>(xl[i]);
+              op_unit<OT, OP>(y, x);
+              x = y;
+            }
+            if (rp[i]) op_unit<OT, OP>(x, to_unit<OT>(xr[i]));
+            if (fl[i] & 4) scale_unit<OT>(x, P.scale);
+            const uint32_t* w = reinterpret_cast<const uint32_t*>(x.v);
+            out = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          *reinterpret_cast<uint4*>(dp[i]) = out;
         }
       }
     } else {
@@ -377,24 +424,33 @@ static bool tree_tables(int n, StepParams& P) {
   return pos <= kMaxTreeJobs;
 }
 
-// Launch with the grid of the small-phase path (one slot per thread) when that grid fits the
-// resident CTAs, else with the large-phase path's (tiles); never more CTAs than are resident.
+template <typename K> static int resident_ctas(K kernel, int& cache) {
+  if (!cache && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&cache, kernel, kStepThreads, 0) != cudaSuccess ||
+                 cache <= 0)) {
+    cache = 0;
+    return 0;
+  }
+  return sm_count() * cache;
+}
+
+// Launch the small-phase kernel (slots) when its grid fits the resident CTAs, else the
+// large-phase kernel (tiles); never more CTAs than the occupancy the runtime reports for that
+// exact kernel (static shared memory included), since every CTA of a cooperative launch must
+// be resident at once. A small grid of one or two CTAs' worth of slots runs on one CTA.
 template <int IN, int OP>
 static cudaError_t launch_stepped(StepParams& P, uint64_t slot_ctas, uint64_t tile_ctas, cudaStream_t s) {
-  auto k = stepped_kernel<IN, OP>;
-  static int bps = 0;
-  if (!bps && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, k, kStepThreads, 0) != cudaSuccess || bps <= 0)) {
-    bps = 0;
-    return cudaErrorInvalidConfiguration;
-  }
-  // every CTA of a cooperative launch must be resident at once: never more than the
-  // occupancy the runtime reports for this kernel (static shared memory included)
-  const uint64_t resident = (uint64_t)sm_count() * (uint64_t)bps;
-  if (P.small < 0) P.small = slot_ctas <= resident ? 1 : 0;
-  const uint64_t want = P.small ? slot_ctas : tile_ctas;
-  const unsigned grid = (unsigned)std::max<uint64_t>(1, std::min<uint64_t>(want, resident));
+  auto ks = stepped_kernel<IN, OP, true>;
+  auto kl = stepped_kernel<IN, OP, false>;
+  static int bps_s = 0, bps_l = 0;
+  const int res_s = resident_ctas(ks, bps_s), res_l = resident_ctas(kl, bps_l);
+  if (!res_s || !res_l) return cudaErrorInvalidConfiguration;
+  const bool small = P.small > 0 || (P.small < 0 && slot_ctas <= (uint64_t)res_s);
+  P.small = small ? 1 : 0;
+  uint64_t want = small ? (slot_ctas <= 2 ? 1 : slot_ctas) : tile_ctas;
+  want = std::max<uint64_t>(1, std::min<uint64_t>(want, (uint64_t)(small ? res_s : res_l)));
   void* args[] = {&P};
-  return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(k), dim3(grid), dim3(kStepThreads), args, 0, s);
+  return cudaLaunchCooperativeKernel(small ? reinterpret_cast<void*>(ks) : reinterpret_cast<void*>(kl),
+                                     dim3((unsigned)want), dim3(kStepThreads), args, 0, s);
 }
 
 cudaError_t launch_stepped_allreduce(const void* const* send, void* const* recv, int nranks, size_t count,
@@ -441,9 +497,9 @@ cudaError_t launch_stepped_allreduce(const void* const* send, void* const* recv,
   for (int ph = 0; fold != kFoldRing && ph < P.phases; ++ph)
     max_jobs = std::max(max_jobs, (int)(P.phase_start[ph + 1] - P.phase_start[ph]));
   max_jobs = std::max(1, max_jobs);
-  // small: one slot per thread of a grid that fits the resident CTAs (decided at launch);
-  // the grid is sized to the slots of the busiest phase, or else to its tiles
-  const uint64_t slot_ctas = ((uint64_t)max_jobs * P.slots_per_job + kStepThreads - 1) / kStepThreads;
+  // small: the slots of the busiest phase fit the resident grid (decided at launch); the grid
+  // is sized to those slots, or else to the busiest phase's tiles
+  const uint64_t slot_ctas = ((uint64_t)max_jobs * P.slots_per_job + kTileUnits - 1) / kTileUnits;
   const uint64_t tile_ctas = ((uint64_t)max_jobs * P.tiles_per_job + kTilesPerCta - 1) / kTilesPerCta;
   P.small = -1;
   uint64_t want = slot_ctas;

@@ -189,12 +189,13 @@ def test_broadcast(n, root, count):
         out[r].check()
 
 
-# N = 2, 3: the binomial program is a left fold from the root (linear kernel); N = 4..31:
-# small-stack machines; N = 32, 64: the deep machine
-@pytest.mark.parametrize("n,root", [(1, 0), (2, 1), (3, 2), (4, 0), (8, 5), (13, 12), (32, 31), (64, 17)])
+# N = 2, 3: the binomial program is a left fold from the root (linear kernel); SUM at N = 4,
+# 8, 16, 32, 64: the program compiled to straight-line code; other N and ops: the fold machines
+@pytest.mark.parametrize("n,root", [(1, 0), (2, 1), (3, 2), (4, 0), (4, 3), (8, 5), (13, 12), (16, 9), (32, 31),
+                                    (64, 17), (64, 0)])
 @pytest.mark.parametrize("kind", ["spread", "i32", "bf16"])
-def test_reduce_to_root(n, root, kind):
-    count = 2049
+@pytest.mark.parametrize("count", [2049, 4 * 8192 + 7])
+def test_reduce_to_root(n, root, kind, count):
     xs = _inputs(kind, n, count, seed=12)
     want, _ = C.reduce(xs, root, in_dtype=_IN[kind])
     out = Guarded(count, _out_dtype(kind))
@@ -392,3 +393,25 @@ def test_stepped_large_messages_sampled(n, count, kind, algo):
     idx = torch.from_numpy(pos).cuda()
     for r in sorted({0, n // 2, n - 1}):
         _assert_same(out[r][idx].cpu().numpy(), want[r], f"stepped {algo} {kind} N={n} rank {r}")
+
+
+@pytest.mark.parametrize("n,root", [(4, 1), (8, 7), (64, 33)])
+@pytest.mark.parametrize("op", ["max", "prod"])
+def test_reduce_other_ops_take_the_fold_machine(n, root, op):
+    xs = [(1.0 + 0.01 * x).astype(np.float32) for x in _inputs("f32", n, 3001, seed=13)]
+    want, _ = C.reduce(xs, root, op=op)
+    out = torch.empty(3001, device="cuda")
+    cc.cc_reduce([to_dev(x) for x in xs], out, root, op=op)
+    torch.cuda.synchronize()
+    _assert_same(to_host(out), want, f"reduce {op} N={n} root {root}")
+
+
+def test_reduce_large_sampled():
+    n, count = 64, 4 * 1024 * 1024 + 3
+    xs = _inputs("spread", n, count, seed=14)
+    out = torch.empty(count, device="cuda")
+    cc.cc_reduce([to_dev(x) for x in xs], out, 5)
+    torch.cuda.synchronize()
+    pos = np.unique(np.concatenate([[0, 1, count - 1], np.arange(2, count, 4091)]))
+    want, _ = C.reduce([x[pos] for x in xs], 5)
+    _assert_same(out[torch.from_numpy(pos).cuda()].cpu().numpy(), want, "reduce N=64 sampled")
