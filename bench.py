@@ -71,12 +71,14 @@ def workload_desc(layers):
 
 
 def measured_peak():
+    """HBM roofline denominator: the measured copy rate (a copy kernel's read + write bytes per
+    second, not a hard ceiling: a read-heavy kernel can pass it), else the recipe's fallback."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             p = json.load(f)
-        return float(p["hbm_gbs"]), "measured"
+        return float(p["hbm_gbs"]), "measured copy rate (MEASURED_PEAKS.json hbm_gbs; not a ceiling)"
     except Exception:
-        return 6650.0, "fallback"
+        return 6650.0, "fallback copy rate (6650 GB/s, earlier measurement; not a ceiling)"
 
 
 def profile_traffic(name="bucket_allreduce_ddp.txt"):
@@ -308,6 +310,10 @@ def timed_row(torch, call, iters, nbytes, launches_per_call, *, flush=None, warm
     return row
 
 
+def _us(ms):
+    return None if ms is None else ms * 1e3
+
+
 def _flusher(torch):
     buf = torch.empty(256 * 1024 * 1024 // 4, device="cuda")  # 256 MiB write, twice the L2
     return lambda: buf.fill_(1.0)
@@ -336,30 +342,32 @@ def rows_config1(torch, cc, local, with_cpu=True):
         shards = [torch.empty(count // n, dtype=tdt, device="cuda") for _ in range(n)]
         ag = [torch.empty(count, dtype=tdt, device="cuda") for _ in range(n)]
         T = count * 4
+        calls = {}
         for algo in ("ring", "tree"):
-            ar = _prepared(cc, "cc_allreduce", cc._ptrs(send), cc._ptrs(y), n, count, dt, dt, cc.CC_SUM,
-                           cc.CC_ALGO_RING if algo == "ring" else cc.CC_ALGO_TREE, 1.0, st)
-            rows[f"allreduce_{algo}_{kind}"] = timed_row(torch, ar, 200, 2 * n * T, 1, flush=flush, local=local)
-        rs = _prepared(cc, "cc_reduce_scatter", cc._ptrs(send), cc._ptrs(shards), n, count, dt, dt, cc.CC_SUM,
-                       cc.CC_ALGO_RING, 1.0, st)
-        rows[f"reduce_scatter_{kind}"] = timed_row(torch, rs, 200, (n + 1) * T, 1, flush=flush, local=local)
-        agc = _prepared(cc, "cc_allgather", cc._ptrs(shards), cc._ptrs(ag), n, count, dt, st)
-        rows[f"allgather_{kind}"] = timed_row(torch, agc, 200, (n + 1) * T, 1, flush=flush, local=local)
+            calls[f"allreduce_{algo}_{kind}"] = (2 * n * T, lambda h, a=algo: _prepared(
+                cc, "cc_allreduce", cc._ptrs(send), cc._ptrs(y), n, count, dt, dt, cc.CC_SUM,
+                cc.CC_ALGO_RING if a == "ring" else cc.CC_ALGO_TREE, 1.0, h))
+        calls[f"reduce_scatter_{kind}"] = ((n + 1) * T, lambda h: _prepared(
+            cc, "cc_reduce_scatter", cc._ptrs(send), cc._ptrs(shards), n, count, dt, dt, cc.CC_SUM, cc.CC_ALGO_RING,
+            1.0, h))
+        calls[f"allgather_{kind}"] = ((n + 1) * T, lambda h: _prepared(
+            cc, "cc_allgather", cc._ptrs(shards), cc._ptrs(ag), n, count, dt, h))
+        for name, (nbytes, make) in calls.items():
+            rows[name] = timed_row(torch, make(st), 200, nbytes, 1, flush=flush, local=local)
+            rows[name]["device_us"] = _us(graph_time_ms(torch, make))
     for r in rows.values():
         r["us"] = r["ms"] * 1e3
     out = {"workload": "config 1: N=4 simulated ranks x 4096 elements, fp32 U[-1,1] and int32 U[-1000,1000] "
                        "(host-seeded), ring allreduce / reduce-scatter / allgather and tree allreduce; latency-bound",
-           "l2": "256 MiB flush before every timed call", "rows": rows}
+           "l2": "256 MiB flush before every timed call",
+           "timing": "us: CUDA events around each call (includes the host's launch cost); device_us: the same calls "
+                     "replayed from a CUDA graph, flush graph subtracted",
+           "rows": rows}
     if with_cpu:
         from oracle import collectives as C
-        t0 = time.perf_counter()
-        reps = 0
-        while time.perf_counter() - t0 < 2.0:
-            C.ring_allreduce(host["f32"])
-            reps += 1
-        dt = (time.perf_counter() - t0) / reps
+        dt, reps, tot = _timed_cpu(lambda: C.ring_allreduce(host["f32"]))
         out["cpu_baseline"] = {"value": 2 * n * count * 4 / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                               "sample": f"the whole config (fp32 ring allreduce), {reps} runs in {reps * dt:.1f} s"}
+                               "sample": f"the whole config (fp32 ring allreduce), {reps} runs in {tot:.1f} s"}
     return out
 
 
@@ -404,13 +412,13 @@ def rows_config3(torch, cc, gen, local, iters, with_cpu=True):
         k = 1 << 20  # sampled positions per rank, spread over every chunk of the full count
         pos = np.unique(np.linspace(0, count - 1, k).astype(np.int64))
         xs = [synth.normal_f32(SEED, r, len(pos), 1e-2, stream=3) for r in range(n)]
-        t0 = time.perf_counter()
-        sh, _ = C.ring_reduce_scatter(xs, count=count, positions=pos)
-        C.ring_allgather(sh, count=count, positions=pos)
-        dt = time.perf_counter() - t0
+        def rs_ag():
+            sh, _ = C.ring_reduce_scatter(xs, count=count, positions=pos)
+            C.ring_allgather(sh, count=count, positions=pos)
+        dt, reps, tot = _timed_cpu(rs_ag)
         out["cpu_baseline"] = {"value": 2 * n * len(pos) * 4 / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
                                "sample": f"reduce-scatter + allgather on {len(pos)} sampled positions per rank "
-                                         f"(full-size chunk map), {dt:.1f} s"}
+                                         f"(full-size chunk map), {reps} runs in {tot:.1f} s"}
     return out
 
 
@@ -463,15 +471,86 @@ def rows_config4(torch, cc, gen, local, iters, with_cpu=True):
         lg = [synth.normal_f32(SEED, r, t_s * E, stream=5).reshape(t_s, E) for r in range(n)]
         tk = [synth.to_bf16_bits(synth.normal_f32(SEED, r, t_s * hidden, stream=6)).reshape(t_s, hidden)
               for r in range(n)]
-        t0 = time.perf_counter()
-        eid = [moe.route_topk(l, topk) for l in lg]
-        d, _ = moe.dispatch(tk, eid, epr)
-        moe.combine(d, eid, epr)
-        dt = time.perf_counter() - t0
+        def rdc():
+            eid = [moe.route_topk(l, topk) for l in lg]
+            d, _ = moe.dispatch(tk, eid, epr)
+            moe.combine(d, eid, epr)
+        dt, reps, tot = _timed_cpu(rdc)
         nb = n * t_s * row + 3 * n * t_s * topk * row
         out["cpu_baseline"] = {"value": nb / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                               "sample": f"route + dispatch + combine of {t_s} tokens per rank, {dt:.1f} s"}
+                               "sample": f"route + dispatch + combine of {t_s} tokens per rank, {reps} runs in "
+                                         f"{tot:.1f} s"}
     return out
+
+
+def graph_time_ms(torch, make_call, iters=20, reps=5, flush_bytes=256 * 1024 * 1024):
+    """Device time per call, without the host's per-call launch cost: `iters` calls captured in
+    one CUDA graph on a side stream, each preceded by an L2 flush (a write of flush_bytes),
+    replayed `reps` times (median); a graph of the flushes alone is timed the same way and
+    subtracted. make_call(stream_handle) returns the call. None if the capture fails."""
+    s = torch.cuda.Stream()
+    call = make_call(s.cuda_stream)
+    buf = torch.empty(flush_bytes // 4, device="cuda") if flush_bytes else None
+    with torch.cuda.stream(s):
+        for _ in range(3):
+            call()
+    torch.cuda.synchronize()
+
+    def capture(with_call):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(iters):
+                if buf is not None:
+                    buf.fill_(1.0)
+                if with_call:
+                    call()
+        return g
+
+    def replay_ms(g):
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(s):  # the graph runs on s, between the two events
+                a.record(s)
+                g.replay()
+                b.record(s)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    try:
+        g1 = capture(True)
+        g0 = capture(False) if buf is not None else None
+    except Exception:
+        torch.cuda.synchronize()
+        return None
+    t = (replay_ms(g1) - (replay_ms(g0) if g0 is not None else 0.0)) / iters
+    del g1, g0
+    return max(t, 0.0)
+
+
+def launch_latency_s(torch, cc, st):
+    """Median CUDA-event time of a minimal cc_allreduce (N = 8 ranks x 4 elements), the
+    per-call startup cost that the alpha of the alpha-beta model stands for."""
+    x = [torch.zeros(4, device="cuda") for _ in range(8)]
+    call = _prepared(cc, "cc_allreduce", cc._ptrs(x), cc._ptrs(x), 8, 4, cc.CC_F32, cc.CC_F32, cc.CC_SUM,
+                     cc.CC_ALGO_RING, 1.0, st)
+    for _ in range(10):
+        call()
+    times = [_event_time_ms(torch, call, 1) for _ in range(200)]
+    return statistics.median(times) * 1e-3
+
+
+def _timed_cpu(fn, min_s=2.0):
+    """Seconds per run of fn(), repeated until min_s have passed (at least once)."""
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        fn()
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= min_s:
+            return dt / reps, reps, dt
 
 
 def alpha_beta_crossover(n, alpha_ring, alpha_tree, bw_ring, bw_tree):
@@ -522,26 +601,40 @@ def rows_config5(torch, cc, gen, local, with_cpu=True):
                 rows[key] = timed_row(torch, call, 10, 2 * n * size, 1, local=local, flush=flush if small else None,
                                       kernel=f"reduce_kernel<f32,sum,{algo}>")
             if n == 8:
-                sc = _prepared(cc, "cc_allreduce_stepped", cc._ptrs(x), cc._ptrs(y), n, count, cc.CC_F32, cc.CC_F32,
-                               cc.CC_SUM, a, 1.0, ws.data_ptr(), ws.numel() * 4, st)
-                r = timed_row(torch, sc, 10 if size > 1024 * 1024 else 50, 2 * n * size, 1, local=local,
+                make = (lambda h, a=a: _prepared(cc, "cc_allreduce_stepped", cc._ptrs(x), cc._ptrs(y), n, count,
+                                                 cc.CC_F32, cc.CC_F32, cc.CC_SUM, a, 1.0, ws.data_ptr(),
+                                                 ws.numel() * 4, h))
+                r = timed_row(torch, make(st), 10 if size > 1024 * 1024 else 50, 2 * n * size, 1, local=local,
                               flush=flush if small else None, kernel=f"stepped_kernel ({algo}, one launch)",
                               own_traffic_bytes=stepped_traffic(n, count, 4, algo))
                 r["own_traffic_GBps"] = r["own_traffic_bytes"] / (r["ms"] * 1e-3) / 1e9
                 r["own_traffic_frac"] = r["own_traffic_GBps"] / measured_peak()[0]
+                t = r["ms"] * 1e-3
+                if small:
+                    r["device_us"] = _us(graph_time_ms(torch, make))
+                    if r["device_us"] is not None:
+                        t = r["device_us"] * 1e-6
                 rows["stepped_" + key] = r
-                stepped[(size, algo)] = r["ms"] * 1e-3
+                stepped[(size, algo)] = t
+        if n == 8 and size >= 1024 * 1024:
+            for K in (2, 4):
+                call = _prepared(cc, "cc_allreduce_multiring", cc._ptrs(x), cc._ptrs(y), n, K, count, cc.CC_F32,
+                                 cc.CC_F32, cc.CC_SUM, 1.0, st)
+                rows[f"n{n}_{_size_name(size)}_multiring{K}"] = timed_row(
+                    torch, call, 10, 2 * n * size, 1, local=local,
+                    kernel=f"reduce_kernel<f32,sum,multi-ring K={K}>")
         del x, y
-    # launch latency of a minimal call (N = 8 ranks x 4 elements)
+    lat = launch_latency_s(torch, cc, st)
     x = [torch.zeros(4, device="cuda") for _ in range(8)]
-    call = _prepared(cc, "cc_allreduce", cc._ptrs(x), cc._ptrs(x), 8, 4, cc.CC_F32, cc.CC_F32, cc.CC_SUM,
-                     cc.CC_ALGO_RING, 1.0, st)
-    lat = timed_row(torch, call, 200, 0, 1, local=local)["ms"] * 1e-3
+    lat_dev = graph_time_ms(torch, lambda h: _prepared(cc, "cc_allreduce", cc._ptrs(x), cc._ptrs(x), 8, 4, cc.CC_F32,
+                                                       cc.CC_F32, cc.CC_SUM, cc.CC_ALGO_RING, 1.0, h))
     n, small, large = 8, 1024, 256 * 1024 * 1024
     ar, br = fit_alpha_beta(n, small, stepped[(small, "ring")], large, stepped[(large, "ring")], "ring")
     at, bt = fit_alpha_beta(n, small, stepped[(small, "tree")], large, stepped[(large, "tree")], "tree")
     model = {"n": n, "alpha_ring_us": ar * 1e6, "alpha_tree_us": at * 1e6, "B_ring_GBps": br / 1e9,
-             "B_tree_GBps": bt / 1e9, "launch_latency_us": lat * 1e6,
+             "B_tree_GBps": bt / 1e9, "launch_latency_us": lat * 1e6, "minimal_call_device_us": _us(lat_dev),
+             "alpha_from": "the stepped schedules' 1 KiB time (CUDA-graph device time) over their step counts; "
+                           "B from their 256 MiB time",
              "crossover_fitted_alpha_bytes": alpha_beta_crossover(n, ar, at, br, bt),
              "crossover_launch_alpha_bytes": alpha_beta_crossover(n, lat, lat, br, bt)}
     out = {"workload": "config 5 large points: fused ring / tree allreduce, N=8 x 256 MiB and N=64 x 64 MiB fp32 "
@@ -555,12 +648,10 @@ def rows_config5(torch, cc, gen, local, with_cpu=True):
         count = 256 * 1024 * 1024 // 4
         pos = np.unique(np.linspace(0, count - 1, 1 << 19).astype(np.int64))
         xs = [synth.uniform_f32(SEED, r, len(pos), stream=7) for r in range(8)]
-        t0 = time.perf_counter()
-        C.ring_allreduce(xs, count=count, positions=pos)
-        dt = time.perf_counter() - t0
+        dt, reps, tot = _timed_cpu(lambda: C.ring_allreduce(xs, count=count, positions=pos))
         out["cpu_baseline"] = {"value": 2 * 8 * len(pos) * 4 / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
                                "sample": f"N=8 ring allreduce on {len(pos)} sampled positions per rank of the "
-                                         f"256 MiB buffer, {dt:.1f} s"}
+                                         f"256 MiB buffer, {reps} runs in {tot:.1f} s"}
     return out
 
 
@@ -584,7 +675,7 @@ def stepped_traffic(n, count, elem, algo):
     return 2 * n * T + (2 * (n // 2) + 3 * (n - 1)) * T
 
 
-A2A_LAUNCHES = 4  # routing tables (count, tile scan, bases) + row copy per alltoallv call
+A2A_LAUNCHES = 2  # routing tables (one launch) + row copy per alltoallv call
 
 
 # ---- one rank per GPU: the DDP step as a real collective over NVLink ---------------------------------
@@ -839,15 +930,29 @@ def run_sweep(args, torch, cc, gen, local):
                     ms = _event_time_ms(torch, call, reps, flush) / reps
                     row[algo + "_us"] = ms * 1e3
                     row[algo + "_GBps"] = 2 * n * size / (ms * 1e-3) / 1e9
-                    stepped = _prepared(cc, "cc_allreduce_stepped", cc._ptrs(x), cc._ptrs(y), n, count, cc.CC_F32,
-                                        cc.CC_F32, cc.CC_SUM, a, 1.0, ws.data_ptr(), ws.numel() * 4, st)
+                    make = (lambda h, a=a: _prepared(cc, "cc_allreduce_stepped", cc._ptrs(x), cc._ptrs(y), n, count,
+                                                     cc.CC_F32, cc.CC_F32, cc.CC_SUM, a, 1.0, ws.data_ptr(),
+                                                     ws.numel() * 4, h))
+                    stepped = make(st)
                     for _ in range(2):
                         stepped()
                     sreps = max(2, reps // 4)
                     ms = _event_time_ms(torch, stepped, sreps, flush) / sreps
+                    if size <= 1024 * 1024:  # latency-bound: the device time, without the host's launch cost
+                        dev = graph_time_ms(torch, make, iters=10, reps=3)
+                        row[algo + "_stepped_event_us"] = ms * 1e3
+                        if dev is not None:
+                            ms = dev
                     row[algo + "_stepped_us"] = ms * 1e3
                     row[algo + "_stepped_GBps"] = 2 * n * size / (ms * 1e-3) / 1e9
                     row[algo + "_stepped_own_GBps"] = stepped_traffic(n, count, 4, algo) / (ms * 1e-3) / 1e9
+                for K in (2, 4):
+                    mr = _prepared(cc, "cc_allreduce_multiring", cc._ptrs(x), cc._ptrs(y), n, K, count, cc.CC_F32,
+                                   cc.CC_F32, cc.CC_SUM, 1.0, st)
+                    for _ in range(2):
+                        mr()
+                    ms = _event_time_ms(torch, mr, reps, flush) / reps
+                    row[f"multiring{K}_GBps"] = 2 * n * size / (ms * 1e-3) / 1e9
                 if n == 8:
                     bc = _prepared(cc, "cc_broadcast", x[0].data_ptr(), cc._ptrs(y), n, 0, count, cc.CC_F32, st)
                     ms = _event_time_ms(torch, bc, reps, flush) / reps
@@ -869,12 +974,7 @@ def run_sweep(args, torch, cc, gen, local):
             hier.append({"n": n, "ranks_per_node": 8, "bytes_per_rank": count * 4, "us": ms * 1e3,
                          "GBps": 2 * n * count * 4 / (ms * 1e-3) / 1e9})
             del x, y
-        x = [torch.zeros(4, device="cuda") for _ in range(8)]
-        lat_call = _prepared(cc, "cc_allreduce", cc._ptrs(x), cc._ptrs(x), 8, 4, cc.CC_F32, cc.CC_F32, cc.CC_SUM,
-                             cc.CC_ALGO_RING, 1.0, st)
-        for _ in range(5):
-            lat_call()
-        lat = _event_time_ms(torch, lat_call, 200) / 200 * 1e-3
+        lat = launch_latency_s(torch, cc, st)
     cross, cross_stepped, model = {}, {}, {}
     for n in (2, 4, 8, 16, 32, 64):
         pts = [r for r in table if r["n"] == n]
@@ -895,8 +995,8 @@ def run_sweep(args, torch, cc, gen, local):
             "warmup": args.warmup, "ms_per_step": best["ring_us"] / 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": "sweep: ring vs double-binary-tree allreduce, N in {2,4,8,16,32,64}, fp32 U[-1,1] "
-                                   "1 KiB..256 MiB per rank (powers of 4), fused and stepped; headline value = N=8, "
-                                   "256 MiB, fused ring",
+                                   "1 KiB..256 MiB per rank (powers of 4), fused and stepped, and the multi-ring "
+                                   "(K = 2, 4); headline value = N=8, 256 MiB, fused ring",
                        "l2": "L2 flushed (256 MiB write) before every timed call whose working set fits in L2"},
             "roofline": dict(roofline_fields(best["ring_GBps"], peak, kind), bound="hbm", traffic=None,
                              kernel="reduce_kernel<f32,sum,ring>"),
@@ -904,6 +1004,51 @@ def run_sweep(args, torch, cc, gen, local):
             "sweep": table, "crossover": cross, "crossover_stepped": cross_stepped, "alpha_beta_model": model,
             "launch_latency_us": lat * 1e6, "hierarchical": hier}
     print(json.dumps(line))
+    return 0
+
+
+def run_kernel(args):
+    """--workload kernel: one collective call, repeated (warm-up, then --steps timed calls), on
+    device-seeded fp32 inputs of --n ranks x --mib MiB: a small, fixed case for profilers.
+    Prints the mean CUDA-event time per call (not a bench line)."""
+    import torch
+    import collective_communication_primitives_rank_b200 as cc
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(SEED)
+    n, count = args.n, args.mib * 1024 * 1024 // 4
+    x = [torch.rand(count, device="cuda", generator=gen) * 2 - 1 for _ in range(n)]
+    y = [torch.empty_like(t) for t in x]
+    st = torch.cuda.current_stream().cuda_stream
+    ws = torch.zeros(64, dtype=torch.int32, device="cuda")
+    k = args.kernel
+    if k.startswith("stepped_"):
+        call = _prepared(cc, "cc_allreduce_stepped", cc._ptrs(x), cc._ptrs(y), n, count, cc.CC_F32, cc.CC_F32,
+                         cc.CC_SUM, cc.CC_ALGO_RING if k.endswith("ring") else cc.CC_ALGO_TREE, 1.0,
+                         ws.data_ptr(), ws.numel() * 4, st)
+    elif k.startswith("multiring"):
+        call = _prepared(cc, "cc_allreduce_multiring", cc._ptrs(x), cc._ptrs(y), n, int(k[len("multiring"):] or 2),
+                         count, cc.CC_F32, cc.CC_F32, cc.CC_SUM, 1.0, st)
+    elif k == "reduce":
+        call = _prepared(cc, "cc_reduce", cc._ptrs(x), y[0].data_ptr(), n, 0, count, cc.CC_F32, cc.CC_F32, cc.CC_SUM,
+                         1.0, st)
+    elif k == "rs":
+        shards = [torch.empty(cc.cc_chunk(count, n, c)[1], device="cuda") for c in range(n)]
+        call = _prepared(cc, "cc_reduce_scatter", cc._ptrs(x), cc._ptrs(shards), n, count, cc.CC_F32, cc.CC_F32,
+                         cc.CC_SUM, cc.CC_ALGO_RING, 1.0, st)
+    elif k == "ag":
+        shards = [x[c][:cc.cc_chunk(count, n, c)[1]] for c in range(n)]
+        call = _prepared(cc, "cc_allgather", cc._ptrs(shards), cc._ptrs(y), n, count, cc.CC_F32, st)
+    elif k in ("ring", "tree"):
+        call = _prepared(cc, "cc_allreduce", cc._ptrs(x), cc._ptrs(y), n, count, cc.CC_F32, cc.CC_F32, cc.CC_SUM,
+                         cc.CC_ALGO_RING if k == "ring" else cc.CC_ALGO_TREE, 1.0, st)
+    else:
+        raise SystemExit(f"unknown --kernel {k}")
+    for _ in range(args.warmup):
+        call()
+    ms = _event_time_ms(torch, call, max(1, args.steps)) / max(1, args.steps)
+    print(json.dumps({"kernel": k, "n": n, "mib_per_rank": args.mib, "ms_per_call": ms,
+                      "allreduce_metric_GBps": 2 * n * count * 4 / (ms * 1e-3) / 1e9}))
     return 0
 
 
@@ -918,7 +1063,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rows", action="store_true", help="headline only (configs 1, 3, 4, 5 left out)")
     ap.add_argument("--oracle-buckets", type=int, default=8)
-    ap.add_argument("--workload", default="ddp", choices=["ddp", "zero", "moe", "sweep", "peer"],
+    ap.add_argument("--kernel", default="ring", help="--workload kernel: stepped_ring, stepped_tree, "
+                    "multiring<K>, reduce, rs, ag, ring, tree")
+    ap.add_argument("--n", type=int, default=8, help="--workload kernel: simulated ranks")
+    ap.add_argument("--mib", type=int, default=32, help="--workload kernel: MiB per rank")
+    ap.add_argument("--workload", default="ddp", choices=["ddp", "zero", "moe", "sweep", "peer", "kernel"],
                     help="ddp = the headline step (plus every other config as rows at one GPU); zero, moe, sweep "
                          "= one config alone in detail; peer = the one-rank-per-GPU collective (the default at N > 1)")
     args = ap.parse_args()
@@ -927,6 +1076,8 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if world > 1 or args.workload == "peer":
         return run_multi_gpu(args)
+    if args.workload == "kernel":
+        return run_kernel(args)
     if args.workload != "ddp":
         return run_rows(args)
     return run_headline(args)

@@ -10,9 +10,11 @@
 // tiles of 256 rows, and rank_in_tile counts earlier rows of the tile with the same
 // expert (warp match + per-warp counts). All of it is integer and deterministic.
 //
-// Kernels: K1 tile counts and per-row ranks, K2 tile prefix per (s, e), K3 bases and
-// receive counts, K4 the row copy (one warp per token: the token row is read once and
-// written topk times; combine reads topk rows and writes topk rows).
+// Kernels: the routing tables in one launch (tile counts and per-row ranks in every CTA;
+// the last CTA of each source to finish builds that source's tile prefix per expert, and the
+// last of those the bases and receive counts), then the row copy (one warp per token: the
+// token row is read once and written topk times; combine reads topk rows and writes topk
+// rows). "Last to finish" is an atomic ticket on counters the call clears first.
 #include <algorithm>
 
 #include "cc_device.cuh"
@@ -25,8 +27,9 @@ constexpr int kMaxTopk = 8;
 
 struct A2AWorkspace {
   // byte offsets inside the caller's workspace; the receive counts sit first, at a
-  // fixed place, so that they can be read back without knowing the other sizes
-  size_t recv_count, tile_cnt, row_rank, totals, base, total;
+  // fixed place, so that they can be read back without knowing the other sizes; then the
+  // finish tickets (one per source and one for all)
+  size_t recv_count, done, tile_cnt, row_rank, totals, base, total;
 };
 
 static A2AWorkspace a2a_layout(int nranks, int tokens, int topk, int experts_per_rank) {
@@ -36,7 +39,8 @@ static A2AWorkspace a2a_layout(int nranks, int tokens, int topk, int experts_per
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   A2AWorkspace w;
   w.recv_count = 0;
-  w.tile_cnt = up(sizeof(int) * kMaxRanks);
+  w.done = up(sizeof(int) * kMaxRanks);
+  w.tile_cnt = w.done + up(sizeof(unsigned) * (kMaxRanks + 1));
   w.row_rank = up(w.tile_cnt + sizeof(int) * nranks * ntiles * E);
   w.totals = up(w.row_rank + sizeof(int) * nranks * rows);
   w.base = up(w.totals + sizeof(int) * nranks * E);
@@ -171,11 +175,55 @@ cudaError_t launch_route_topk(const float* const* logits, int32_t* const* ids, i
   return cudaGetLastError();
 }
 
-// ---- K1: per-tile expert counts and per-row rank within the tile -------------------------------------
+// ---- routing tables -----------------------------------------------------------------------------------
+// Every CTA counts one tile of 256 rows of one source: per expert the rows of the tile, and
+// each row's rank among the tile's rows of its expert (warp match + per-warp prefix).
 
-__global__ void __launch_bounds__(kTileRows) a2a_count_kernel(const __grid_constant__ IdPtrs I, int rows, int E,
-                                                              int* __restrict__ tile_cnt, int* __restrict__ row_rank) {
-  extern __shared__ int warp_cnt[];  // [8][E]
+constexpr int kScanSplit = 4;  // threads per expert in the per-source tile prefix
+
+// Bases and receive counts from the per-(source, expert) totals, by one CTA: the totals are
+// staged in shared memory (`sm`: nranks * E + nranks * nranks ints) with one coalesced pass.
+__device__ __forceinline__ void bases_and_counts(int nranks, int epr, const int* tot_g, int* base, int* recv_count,
+                                                 int* sm) {
+  const int E = nranks * epr;
+  int* tot = sm;
+  int* cnt = sm + nranks * E;  // rows s -> d
+  for (int i = threadIdx.x; i < nranks * E; i += blockDim.x) tot[i] = __ldcg(tot_g + i);
+  __syncthreads();
+  for (int i = threadIdx.x; i < nranks * nranks; i += blockDim.x) {
+    const int s = i / nranks, d = i % nranks;
+    int c = 0;
+    for (int l = 0; l < epr; ++l) c += tot[s * E + d * epr + l];
+    cnt[i] = c;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < nranks * E; i += blockDim.x) {
+    const int s = i / E, e = i % E, d = e / epr;
+    int off = 0;
+    for (int sp = 0; sp < s; ++sp) off += cnt[sp * nranks + d];
+    for (int l = d * epr; l < e; ++l) off += tot[s * E + l];
+    base[i] = off;
+  }
+  for (int d = threadIdx.x; d < nranks; d += blockDim.x) {
+    int c = 0;
+    for (int s = 0; s < nranks; ++s) c += cnt[s * nranks + d];
+    recv_count[d] = c;
+  }
+}
+
+constexpr int kScanSmemInts = 10240;  // a source's [tiles][experts] counts scanned in shared memory up to this
+
+__global__ void __launch_bounds__(kTileRows) a2a_tables_kernel(const __grid_constant__ IdPtrs I, int rows, int nranks,
+                                                               int epr, int* __restrict__ tile_cnt,
+                                                               int* __restrict__ row_rank, int* __restrict__ totals,
+                                                               int* __restrict__ base, int* __restrict__ recv_count,
+                                                               unsigned* __restrict__ done) {
+  extern __shared__ int warp_cnt[];  // [8][E]; reused by the last CTAs (scan, then bases)
+  __shared__ int s_last;
+  // the copy kernel (a programmatic dependent) may launch now: it waits for this grid to
+  // complete before it reads any table
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int E = nranks * epr;
   const int s = blockIdx.y, tile = blockIdx.x, ntiles = gridDim.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < 8 * E; i += blockDim.x) warp_cnt[i] = 0;
@@ -201,54 +249,75 @@ __global__ void __launch_bounds__(kTileRows) a2a_count_kernel(const __grid_const
   }
   __syncthreads();
   if (valid) row_rank[(size_t)s * rows + row] = warp_cnt[warp * E + e] + rank_w;
-}
 
-// ---- K2: exclusive prefix over tiles, per (source, expert); one warp each -----------------------------
-
-__global__ void a2a_tile_scan_kernel(int ntiles, int E, int* __restrict__ tile_cnt, int* __restrict__ totals) {
-  const int s = blockIdx.y, e = blockIdx.x, lane = threadIdx.x;
-  int carry = 0;
-  for (int t0 = 0; t0 < ntiles; t0 += 32) {
-    const int t = t0 + lane;
-    int* p = tile_cnt + ((size_t)s * ntiles + t) * E + e;
-    const int v = t < ntiles ? *p : 0;
-    int inc = v;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int o = __shfl_up_sync(0xffffffffu, inc, off);
-      if (lane >= off) inc += o;
+  // the last tile of source s to finish turns the tile counts into exclusive prefixes over
+  // tiles, per expert, and the source's totals
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(&done[1 + s], 1u) == (unsigned)ntiles - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const size_t blk = (size_t)ntiles * E;
+  int* src_cnt = tile_cnt + (size_t)s * blk;
+  if (blk <= (size_t)kScanSmemInts) {
+    // the source's counts staged in shared memory with one coalesced pass, scanned there per
+    // expert, written back as exclusive prefixes
+    for (size_t i = threadIdx.x; i < blk; i += blockDim.x) warp_cnt[i] = __ldcg(src_cnt + i);
+    __syncthreads();
+    for (int x = threadIdx.x; x < E; x += blockDim.x) {
+      int run = 0;
+      for (int t = 0; t < ntiles; ++t) {
+        const int v = warp_cnt[t * E + x];
+        warp_cnt[t * E + x] = run;
+        run += v;
+      }
+      totals[(size_t)s * E + x] = run;
     }
-    if (t < ntiles) *p = carry + inc - v;
-    carry += __shfl_sync(0xffffffffu, inc, 31);
+    __syncthreads();
+    for (size_t i = threadIdx.x; i < blk; i += blockDim.x) src_cnt[i] = warp_cnt[i];
+  } else {
+    const int q = threadIdx.x % kScanSplit;
+    const int per = (ntiles + kScanSplit - 1) / kScanSplit;
+    const int t0 = q * per, t1 = min(ntiles, t0 + per);
+    for (int e0 = 0; e0 < E; e0 += kTileRows / kScanSplit) {
+      const int x = e0 + threadIdx.x / kScanSplit;
+      const bool live = x < E;
+      int* col = src_cnt + (live ? x : 0);
+      int part = 0;
+      for (int t = t0; live && t < t1; ++t) part += __ldcg(col + (size_t)t * E);
+      // exclusive prefix of the kScanSplit partial sums (the lanes of one expert are adjacent)
+      int inc = part;
+#pragma unroll
+      for (int off = 1; off < kScanSplit; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, inc, off, kScanSplit);
+        if (q >= off) inc += o;
+      }
+      int run = inc - part;
+      for (int t = t0; live && t < t1; ++t) {
+        const int v = __ldcg(col + (size_t)t * E);
+        col[(size_t)t * E] = run;
+        run += v;
+      }
+      if (live && q == kScanSplit - 1) totals[(size_t)s * E + x] = run;
+    }
   }
-  if (lane == 0) totals[(size_t)s * E + e] = carry;
+  // the last source to finish builds the bases and the receive counts
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(&done[0], 1u) == (unsigned)nranks - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  bases_and_counts(nranks, epr, totals, base, recv_count, warp_cnt);
 }
 
-// ---- K3: bases per (source, expert) and receive counts per destination (one CTA) -------------------------
+// ---- no rows: bases and receive counts from zero totals (one CTA) ------------------------------------
 
 __global__ void __launch_bounds__(1024) a2a_base_kernel(int nranks, int epr, const int* __restrict__ tot,
                                                         int* __restrict__ base, int* __restrict__ recv_count) {
-  __shared__ int cnt[kMaxRanks * kMaxRanks];  // rows s -> d
-  const int E = nranks * epr;
-  for (int i = threadIdx.x; i < nranks * nranks; i += blockDim.x) {
-    const int s = i / nranks, d = i % nranks;
-    int c = 0;
-    for (int l = 0; l < epr; ++l) c += tot[s * E + d * epr + l];
-    cnt[i] = c;
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < nranks * E; i += blockDim.x) {
-    const int s = i / E, e = i % E, d = e / epr;
-    int off = 0;
-    for (int sp = 0; sp < s; ++sp) off += cnt[sp * nranks + d];
-    for (int l = d * epr; l < e; ++l) off += tot[s * E + l];
-    base[i] = off;
-  }
-  for (int d = threadIdx.x; d < nranks; d += blockDim.x) {
-    int c = 0;
-    for (int s = 0; s < nranks; ++s) c += cnt[s * nranks + d];
-    recv_count[d] = c;
-  }
+  __shared__ int sm[1024 + kMaxRanks * kMaxRanks];  // totals (N * E <= 1024), then rows s -> d
+  bases_and_counts(nranks, epr, tot, base, recv_count, sm);
 }
 
 // ---- K4: row copies ----------------------------------------------------------------------------------
@@ -265,11 +334,29 @@ struct A2ACopyParams {
   int tokens, topk, epr, E, ntiles, direction;
 };
 
+// The copy is launched as a programmatic dependent of the table kernel: its CTAs may start
+// while the tables are still being built, and wait (griddepcontrol.wait) for the table kernel
+// to complete before they read a position. A dispatch row does not depend on the tables, so its
+// first 16 vectors per lane are loaded before that wait.
+__device__ __forceinline__ void wait_for_tables() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __global__ void __launch_bounds__(256) a2a_copy_kernel(const __grid_constant__ A2ACopyParams P) {
   const int lane = threadIdx.x & 31;
   const int s = blockIdx.y;
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (t >= P.tokens) return;
+  // 16 loads per lane in flight before the stores that consume them (a whole 8 KiB row per
+  // warp; measured faster than 8 or 32)
+  constexpr int B = 16;
+  const uint64_t nvec = P.row_bytes / 16;
+  uint4 x[B];
+  const uint4* row = reinterpret_cast<const uint4*>(P.send[s] + (uint64_t)t * P.row_bytes);
+  if (P.direction == 0) {
+#pragma unroll
+    for (int b = 0; b < B; ++b)
+      if (lane + 32 * b < nvec) x[b] = __ldcs(row + lane + 32 * b);
+  }
+  wait_for_tables();
   const int rows = P.tokens * P.topk;
   char* ptr[kMaxTopk];
   bool ok[kMaxTopk];
@@ -284,17 +371,13 @@ __global__ void __launch_bounds__(256) a2a_copy_kernel(const __grid_constant__ A
     ok[k] = pos < P.capacity;
     ptr[k] = (P.direction == 0 ? P.recv[d] : const_cast<char*>(P.send[d])) + pos * P.row_bytes;
   }
-  // 16 loads per lane in flight before the stores that consume them (a whole 8 KiB row per
-  // warp; measured faster than 8 or 32)
-  constexpr int B = 16;
-  const uint64_t nvec = P.row_bytes / 16;
   if (P.direction == 0) {
-    const uint4* src = reinterpret_cast<const uint4*>(P.send[s] + (uint64_t)t * P.row_bytes);
     for (uint64_t v0 = lane; v0 < nvec; v0 += 32 * B) {
-      uint4 x[B];
+      if (v0 != (uint64_t)lane) {
 #pragma unroll
-      for (int b = 0; b < B; ++b)
-        if (v0 + 32 * b < nvec) x[b] = __ldcs(src + v0 + 32 * b);
+        for (int b = 0; b < B; ++b)
+          if (v0 + 32 * b < nvec) x[b] = __ldcs(row + v0 + 32 * b);
+      }
       for (int k = 0; k < P.topk; ++k) {
         if (!ok[k]) continue;
         uint4* d = reinterpret_cast<uint4*>(ptr[k]);
@@ -310,7 +393,6 @@ __global__ void __launch_bounds__(256) a2a_copy_kernel(const __grid_constant__ A
       const uint4* src = reinterpret_cast<const uint4*>(ptr[k]);
       uint4* d = reinterpret_cast<uint4*>(dst + k * P.row_bytes);
       for (uint64_t v0 = lane; v0 < nvec; v0 += 32 * B) {
-        uint4 x[B];
 #pragma unroll
         for (int b = 0; b < B; ++b)
           if (v0 + 32 * b < nvec) x[b] = __ldcs(src + v0 + 32 * b);
@@ -338,14 +420,21 @@ cudaError_t launch_alltoallv(const void* const* send, void* const* recv, int nra
   IdPtrs I{};
   for (int r = 0; r < nranks; ++r) I.ids[r] = ids[r];
   if (rows > 0) {
-    a2a_count_kernel<<<dim3(ntiles, nranks), kTileRows, sizeof(int) * 8 * E, stream>>>(I, rows, E, tile_cnt, row_rank);
-    a2a_tile_scan_kernel<<<dim3(E, nranks), 32, 0, stream>>>(ntiles, E, tile_cnt, totals);
+    // the finish tickets start at zero (stream-ordered), then one launch builds every table
+    unsigned* done = reinterpret_cast<unsigned*>(ws + w.done);
+    const cudaError_t e = cudaMemsetAsync(done, 0, sizeof(unsigned) * (kMaxRanks + 1), stream);
+    if (e != cudaSuccess) return e;
+    const size_t scan = std::min<size_t>((size_t)ntiles * E, kScanSmemInts);
+    const size_t smem = sizeof(int) * std::max<size_t>(std::max<size_t>(8 * E, nranks * E + nranks * nranks), scan);
+    a2a_tables_kernel<<<dim3(ntiles, nranks), kTileRows, smem, stream>>>(I, rows, nranks, experts_per_rank,
+                                                                         tile_cnt, row_rank, totals, base,
+                                                                         recv_count, done);
   } else {
-    // no rows: the bases read zero totals (the only write to this scratch before K3)
+    // no rows: the bases read zero totals (the only write to this scratch before them)
     const cudaError_t e = cudaMemsetAsync(totals, 0, sizeof(int) * nranks * E, stream);
     if (e != cudaSuccess) return e;
+    a2a_base_kernel<<<1, 1024, 0, stream>>>(nranks, experts_per_rank, totals, base, recv_count);
   }
-  a2a_base_kernel<<<1, 1024, 0, stream>>>(nranks, experts_per_rank, totals, base, recv_count);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess || rows == 0) return err;
   A2ACopyParams P{};
@@ -365,8 +454,18 @@ cudaError_t launch_alltoallv(const void* const* send, void* const* recv, int nra
   P.E = E;
   P.ntiles = ntiles;
   P.direction = direction;
-  a2a_copy_kernel<<<dim3((tokens + 7) / 8, nranks), 256, 0, stream>>>(P);
-  return cudaGetLastError();
+  // a programmatic dependent of the table kernel (see a2a_copy_kernel)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((tokens + 7) / 8, nranks);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, a2a_copy_kernel, P);
 }
 
 cudaError_t copy_recv_counts(const void* workspace, int nranks, int32_t* out, cudaStream_t stream) {

@@ -41,8 +41,10 @@ def _moe_case(n, tokens, hidden, epr, seed=2):
     return ids, toks
 
 
+# (4, 3000, 16, 256): 24 tiles x 1024 experts per source, more counts than the table kernel scans
+# in shared memory, so the per-source prefix runs on its global-memory path
 @pytest.mark.parametrize("n,tokens,hidden,epr", [(8, 300, 64, 8), (4, 1000, 8, 2), (3, 17, 16, 1), (1, 50, 8, 4),
-                                                 (8, 2048, 4096, 8)])
+                                                 (8, 2048, 4096, 8), (4, 3000, 16, 256)])
 def test_alltoallv_dispatch_and_combine_match_oracle(n, tokens, hidden, epr):
     ids, toks = _moe_case(n, tokens, hidden, epr)
     want, _ = moe.dispatch(toks, ids, epr)
