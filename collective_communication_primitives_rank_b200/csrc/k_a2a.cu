@@ -251,13 +251,17 @@ __global__ void __launch_bounds__(kTileRows) a2a_tables_kernel(const __grid_cons
   if (valid) row_rank[(size_t)s * rows + row] = warp_cnt[warp * E + e] + rank_w;
 
   // the last tile of source s to finish turns the tile counts into exclusive prefixes over
-  // tiles, per expert, and the source's totals
-  __threadfence();
+  // tiles, per expert, and the source's totals. Thread 0 publishes the CTA's writes (the
+  // barrier orders the other threads' writes before its fence) and takes the ticket; the last
+  // CTA's thread 0 fences again before the barrier that lets its threads read the others' counts.
   __syncthreads();
-  if (threadIdx.x == 0) s_last = atomicAdd(&done[1 + s], 1u) == (unsigned)ntiles - 1;
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(&done[1 + s], 1u) == (unsigned)ntiles - 1;
+    __threadfence();
+  }
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   const size_t blk = (size_t)ntiles * E;
   int* src_cnt = tile_cnt + (size_t)s * blk;
   if (blk <= (size_t)kScanSmemInts) {
@@ -303,12 +307,14 @@ __global__ void __launch_bounds__(kTileRows) a2a_tables_kernel(const __grid_cons
     }
   }
   // the last source to finish builds the bases and the receive counts
-  __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) s_last = atomicAdd(&done[0], 1u) == (unsigned)nranks - 1;
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(&done[0], 1u) == (unsigned)nranks - 1;
+    __threadfence();
+  }
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   bases_and_counts(nranks, epr, totals, base, recv_count, warp_cnt);
 }
 
