@@ -286,7 +286,7 @@ CC_API cc_status cc_bucket_allreduce_buckets(const void* const* grads, void* con
 /* The same fused DDP step for gradients that live in host memory: every host_grads[j] is
  * copied to dev_grads[j] (host -> device), the fused allreduce runs on the device copies,
  * and every dev_out[j] is copied back to host_out[j] (device -> host). The work is cut in
- * bucket order into slices (at most 2^20 elements per rank) grouped into stages, and the
+ * registration order into slices (at most 2^20 elements per rank) grouped into stages, and the
  * copies in, the kernels and the copies out of consecutive stages overlap on two
  * library-owned streams (created once per device) and `stream`; a slice keeps its bucket
  * offset, so the results equal cc_bucket_allreduce's. From the caller's view the call is
