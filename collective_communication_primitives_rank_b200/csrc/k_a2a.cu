@@ -265,21 +265,47 @@ __global__ void __launch_bounds__(kTileRows) a2a_tables_kernel(const __grid_cons
   const size_t blk = (size_t)ntiles * E;
   int* src_cnt = tile_cnt + (size_t)s * blk;
   if (blk <= (size_t)kScanSmemInts) {
-    // the source's counts staged in shared memory with one coalesced pass, scanned there per
-    // expert, written back as exclusive prefixes
+    // the source's counts staged in shared memory with one coalesced pass; kScanSplit threads
+    // per expert each sum a run of tiles, an exclusive prefix over the runs (shuffles), then
+    // each thread turns its run into exclusive prefixes in place. The totals are published
+    // (and the next ticket taken) before the prefixes go back to global memory: only the copy
+    // kernel reads those, after this grid has completed.
     for (size_t i = threadIdx.x; i < blk; i += blockDim.x) warp_cnt[i] = __ldcg(src_cnt + i);
     __syncthreads();
-    for (int x = threadIdx.x; x < E; x += blockDim.x) {
-      int run = 0;
-      for (int t = 0; t < ntiles; ++t) {
+    const int q = threadIdx.x % kScanSplit;
+    const int per = (ntiles + kScanSplit - 1) / kScanSplit;
+    const int t0 = q * per, t1 = min(ntiles, t0 + per);
+    for (int e0 = 0; e0 < E; e0 += kTileRows / kScanSplit) {
+      const int x = e0 + threadIdx.x / kScanSplit;
+      const bool live = x < E;
+      int part = 0;
+      for (int t = t0; live && t < t1; ++t) part += warp_cnt[t * E + x];
+      int inc = part;
+#pragma unroll
+      for (int off = 1; off < kScanSplit; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, inc, off, kScanSplit);
+        if (q >= off) inc += o;
+      }
+      int run = inc - part;
+      for (int t = t0; live && t < t1; ++t) {
         const int v = warp_cnt[t * E + x];
         warp_cnt[t * E + x] = run;
         run += v;
       }
-      totals[(size_t)s * E + x] = run;
+      if (live && q == kScanSplit - 1) totals[(size_t)s * E + x] = run;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      s_last = atomicAdd(&done[0], 1u) == (unsigned)nranks - 1;
+      __threadfence();
     }
     __syncthreads();
     for (size_t i = threadIdx.x; i < blk; i += blockDim.x) src_cnt[i] = warp_cnt[i];
+    if (!s_last) return;
+    __syncthreads();  // every thread is done with warp_cnt before the bases reuse it
+    bases_and_counts(nranks, epr, totals, base, recv_count, warp_cnt);
+    return;
   } else {
     const int q = threadIdx.x % kScanSplit;
     const int per = (ntiles + kScanSplit - 1) / kScanSplit;
