@@ -722,13 +722,24 @@ def run_multi_gpu(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
+    # CC_BENCH_BACKEND=gloo with CC_BENCH_DEVICE=0 runs every rank's process on one GPU with host
+    # barriers over gloo and without the NCCL comparator: the slice path's plumbing (layout, IPC
+    # mappings, the step, the parity check) on a machine with fewer GPUs than ranks. The ranks'
+    # kernels never wait on one another; the host barriers order them.
+    backend = os.environ.get("CC_BENCH_BACKEND", "nccl")
+    device = int(os.environ.get("CC_BENCH_DEVICE", local))
+    torch.cuda.set_device(device)
     for k, v in (("MASTER_ADDR", "127.0.0.1"), ("MASTER_PORT", "29531"), ("RANK", str(rank)),
                  ("WORLD_SIZE", str(world))):
         os.environ.setdefault(k, v)
     if not dist.is_initialized():
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", device))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    nccl = backend == "nccl"
+    mdev = "cuda" if nccl else "cpu"  # where the max over ranks is reduced
     shapes = synth.transformer_grad_shapes(layers=args.layers)
     numels = [synth.numel(s) for _, s in shapes]
     total = sum(numels)
@@ -779,9 +790,9 @@ def run_multi_gpu(args):
         b.record(stream)
         torch.cuda.synchronize()
         dist.barrier()
-        return max_over_ranks(dist, torch, a.elapsed_time(b) / steps, "cuda")
+        return max_over_ranks(dist, torch, a.elapsed_time(b) / steps, mdev)
 
-    with Clocks(local) as clk:
+    with Clocks(device) as clk:
         ms = timed(step, args.steps)
     T = total * 4
     value = aggregate_gbps(world, 2 * T, ms)
@@ -789,18 +800,20 @@ def run_multi_gpu(args):
 
     # NCCL: all_reduce of the same buckets (sum), and all_gather of 256 MiB shards as the
     # measured NVLink rate
-    x = send.clone()
+    ms_nccl, ag_busbw = None, 0.0
+    if nccl:
+        x = send.clone()
 
-    def nccl_step():
-        for start, count in ranges:
-            dist.all_reduce(x[start:start + count])
+        def nccl_step():
+            for start, count in ranges:
+                dist.all_reduce(x[start:start + count])
 
-    ms_nccl = timed(nccl_step, args.steps)
-    shard = torch.empty(64 * 1024 * 1024, device="cuda")
-    gathered = torch.empty(world * shard.numel(), device="cuda")
-    ms_ag = timed(lambda: dist.all_gather_into_tensor(gathered, shard), max(3, args.steps // 2))
-    ag_busbw = (world - 1) * shard.numel() * 4 / (ms_ag * 1e-3) / 1e9
-    del x, gathered, shard
+        ms_nccl = timed(nccl_step, args.steps)
+        shard = torch.empty(64 * 1024 * 1024, device="cuda")
+        gathered = torch.empty(world * shard.numel(), device="cuda")
+        ms_ag = timed(lambda: dist.all_gather_into_tensor(gathered, shard), max(3, args.steps // 2))
+        ag_busbw = (world - 1) * shard.numel() * 4 / (ms_ag * 1e-3) / 1e9
+        del x, gathered, shard
 
     # end to end: pinned host gradients -> device, the step, device -> pinned host
     host_out = torch.empty_like(host, pin_memory=True)
@@ -846,8 +859,9 @@ def run_multi_gpu(args):
                        "ranks": world, "bytes_per_rank": T, "buckets": len(ranges),
                        "l2": "inputs larger than L2; no flush", "parallelism": f"ranks x{world}"},
             "comm_nranks": world, "busbw": bus, "parity_rank0_vs_single_gpu": parity,
-            "nccl": {"ms_per_step": ms_nccl, "busbw": 2.0 * (world - 1) / world * T / (ms_nccl * 1e-3) / 1e9,
-                     "all_gather_busbw": ag_busbw},
+            "nccl": ({"ms_per_step": ms_nccl, "busbw": 2.0 * (world - 1) / world * T / (ms_nccl * 1e-3) / 1e9,
+                      "all_gather_busbw": ag_busbw} if nccl else None),
+            "backend": backend,
             "roofline": {"bound": "nvlink", "achieved": bus, "peak": peak, "unit": "GB/s",
                          "frac": bus / peak if peak > 0 else None,
                          "peak_kind": "NCCL all_gather bus bandwidth measured in this run", "traffic": None},

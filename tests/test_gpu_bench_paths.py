@@ -37,3 +37,22 @@ def test_one_rank_per_gpu_path_runs_and_matches_the_single_gpu_call():
     line = json.loads([l for l in r.stdout.splitlines() if l.startswith("{")][-1])
     assert line["parity_rank0_vs_single_gpu"] == "bit-exact"
     assert line["comm_nranks"] == 1 and line["value"] > 0 and line["config"]["buckets"] >= 1
+
+
+@pytest.mark.timeout(900)
+def test_two_ranks_on_one_gpu_over_gloo_match_the_single_gpu_call():
+    """Two processes (torchrun), both on this GPU, host barriers over gloo: the bucket layout,
+    the IPC mappings of the other rank's buffers, the 17-bucket step of slice calls and rank 0's
+    bit-exact comparison with the single-GPU fused call over both ranks' gradients. No kernel
+    waits on the other rank; the barriers order them."""
+    env = dict(os.environ, CC_BENCH_BACKEND="gloo", CC_BENCH_DEVICE="0")
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_port()), os.path.join(ROOT, "bench.py"),
+           "--gpus", "2", "--workload", "peer", "--layers", "1", "--steps", "2", "--warmup", "1", "--e2e-steps", "1"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=840, cwd=ROOT, env=env)
+    assert r.returncode == 0, r.stderr[-3000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1  # rank 0 alone prints
+    line = json.loads(lines[0])
+    assert line["parity_rank0_vs_single_gpu"] == "bit-exact"
+    assert line["comm_nranks"] == 2 and line["n_gpus"] == 2 and line["backend"] == "gloo"
