@@ -415,3 +415,22 @@ def test_reduce_large_sampled():
     pos = np.unique(np.concatenate([[0, 1, count - 1], np.arange(2, count, 4091)]))
     want, _ = C.reduce([x[pos] for x in xs], 5)
     _assert_same(out[torch.from_numpy(pos).cuda()].cpu().numpy(), want, "reduce N=64 sampled")
+
+
+@pytest.mark.parametrize("algo", ["ring", "tree"])
+def test_stepped_misaligned_large_takes_the_element_tiles(algo):
+    """Outputs one element off a 16-byte boundary and large enough for the large-phase kernel:
+    its element-wise tiles, compared with the oracle on sampled positions."""
+    n, count = 3, 1024 * 1024 + 7
+    xs = _inputs("spread", n, count, seed=18)
+    out = [misaligned(np.zeros(count, np.float32)) for _ in range(n)]
+    ws = torch.zeros(64, dtype=torch.int32, device="cuda")
+    cc.cc_allreduce_stepped([to_dev(x) for x in xs], out, ws, algo=algo, scale=0.25)
+    torch.cuda.synchronize()
+    assert cc.cc_async_status() == cc.CC_OK
+    pos = np.unique(np.concatenate([[0, 1, 2, count - 1], np.arange(3, count, 997)]))
+    fn = C.ring_allreduce if algo == "ring" else C.tree_allreduce
+    want, _ = fn([x[pos] for x in xs], scale=0.25, count=count, positions=pos)
+    idx = torch.from_numpy(pos).cuda()
+    for r in range(n):
+        _assert_same(out[r][idx].cpu().numpy(), want[r], f"stepped misaligned {algo} rank {r}")
