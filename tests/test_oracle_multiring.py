@@ -156,3 +156,14 @@ def test_planted_mistakes_are_caught(monkeypatch):
     out, _ = C.multiring_allreduce(xs, K)
     monkeypatch.undo()
     assert not np.array_equal(_bits(out[0]), _bits(want))
+
+
+def test_threaded_mesh_gives_the_lockstep_result():
+    """One thread per rank with receive timeouts (the from-scratch page's queue mesh) runs the
+    same multi-ring schedule to the same bits and byte counts."""
+    from oracle.mesh import LockstepMesh, ThreadedMesh
+    xs = _spread_f32(59, 6, 301)
+    a, ma = C.multiring_allreduce(xs, 3, mesh=LockstepMesh(6))
+    b, mb = C.multiring_allreduce(xs, 3, mesh=ThreadedMesh(6, recv_timeout_s=5.0))
+    assert all(np.array_equal(_bits(u), _bits(v)) for u, v in zip(a, b))
+    assert ma.sent == mb.sent and dict(ma.link_bytes) == dict(mb.link_bytes)
