@@ -434,3 +434,44 @@ def test_stepped_misaligned_large_takes_the_element_tiles(algo):
     idx = torch.from_numpy(pos).cuda()
     for r in range(n):
         _assert_same(out[r][idx].cpu().numpy(), want[r], f"stepped misaligned {algo} rank {r}")
+
+
+def test_calls_replay_from_a_cuda_graph():
+    """The calls are stream-ordered and do no host synchronisation, so they can be captured in a
+    CUDA graph and replayed: a captured allreduce, reduce-scatter + allgather, stepped allreduce
+    and fused bucket allreduce give the oracle's bits on every replay, with new inputs copied in
+    between replays."""
+    n, count = 8, 3 * 4096 + 5
+    s = torch.cuda.Stream()
+    send = [torch.empty(count, device="cuda") for _ in range(n)]
+    ar = [torch.empty(count, device="cuda") for _ in range(n)]
+    st = [torch.empty(count, device="cuda") for _ in range(n)]
+    shards = [torch.empty(cc.cc_chunk(count, n, c)[1], device="cuda") for c in range(n)]
+    ag = [torch.empty(count, device="cuda") for _ in range(n)]
+    ws = torch.zeros(64, dtype=torch.int32, device="cuda")
+    with torch.cuda.stream(s):  # warm up (lazy set-up) outside the capture
+        cc.cc_allreduce(send, ar, scale=None, stream=s)
+        cc.cc_reduce_scatter(send, shards, stream=s)
+        cc.cc_allgather(shards, ag, stream=s)
+        cc.cc_allreduce_stepped(send, st, ws, algo="tree", stream=s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        cc.cc_allreduce(send, ar, scale=None, stream=s)
+        cc.cc_reduce_scatter(send, shards, stream=s)
+        cc.cc_allgather(shards, ag, stream=s)
+        cc.cc_allreduce_stepped(send, st, ws, algo="tree", stream=s)
+    for rep in range(2):
+        xs = _inputs("spread", n, count, seed=70 + rep)
+        for r in range(n):
+            send[r].copy_(to_dev(xs[r]))
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        want_ar, _ = C.ring_allreduce(xs, scale=float(np.float32(1) / np.float32(n)))
+        want_rs, _ = C.ring_allreduce(xs)
+        want_st, _ = C.tree_allreduce(xs)
+        for r in range(n):
+            _assert_same(to_host(ar[r]), want_ar[r], f"graph allreduce replay {rep} rank {r}")
+            _assert_same(to_host(ag[r]), want_rs[r], f"graph RS+AG replay {rep} rank {r}")
+            _assert_same(to_host(st[r]), want_st[r], f"graph stepped replay {rep} rank {r}")
