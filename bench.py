@@ -258,14 +258,22 @@ def run_reference(args):
 
 # ---- the other hot-path rows: configs 1, 3, 4 and 5 ---------------------------------------------------
 
-def _event_time_ms(torch, fn, iters, flush=None):
+SPIN_CYCLES = 200_000  # about 0.1 ms of spinning at the B200's 1.97 GHz SM clock
+
+
+def _event_time_ms(torch, fn, iters, flush=None, host_launch=False):
     """Sum of per-iteration CUDA-event times of fn() on the current stream; `flush` (outside
-    the timed spans) evicts L2 between iterations when the working set would fit in it."""
+    the timed spans) evicts L2 between iterations when the working set would fit in it.
+    Each span opens on a busy GPU (behind the flush, else behind a ~0.1 ms spin kernel), so it
+    holds the device time of fn and not the host's cost of launching it; host_launch=True
+    leaves the GPU idle before each span, which counts that cost too."""
     total = 0.0
     stream = torch.cuda.current_stream()
     for _ in range(iters):
         if flush is not None:
             flush()
+        elif not host_launch:
+            torch.cuda._sleep(SPIN_CYCLES)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         fn()
@@ -294,9 +302,9 @@ def roofline_fields(achieved, peak, peak_kind):
 
 
 def timed_row(torch, call, iters, nbytes, launches_per_call, *, flush=None, warmup=3, local=0, **extra):
-    """One measured row: CUDA-event time per call (after `warmup` untimed calls), the
-    algorithmic bytes, GB/s against the measured copy rate, and the clocks sampled while the
-    timed calls ran."""
+    """One measured row: device time per call from CUDA events (after `warmup` untimed calls;
+    spans opened on a busy GPU, see _event_time_ms), the algorithmic bytes, GB/s against the
+    measured copy rate, and the clocks sampled while the timed calls ran."""
     for _ in range(warmup):
         call()
     torch.cuda.synchronize()
@@ -448,18 +456,33 @@ def rows_config4(torch, cc, gen, local, iters, with_cpu=True):
                      cap, 0, ws.data_ptr(), wsb, st)
     comb = _prepared(cc, "cc_alltoallv", cc._ptrs(recv), cc._ptrs(back), n, row, cc._ptrs(ids), tokens, topk, epr,
                      cap, 1, ws.data_ptr(), wsb, st)
+    plan = _prepared(cc, "cc_alltoallv_plan", cc._ptrs(ids), n, tokens, topk, epr, ws.data_ptr(), wsb, st)
+    disp_run = _prepared(cc, "cc_alltoallv_run", cc._ptrs(toks), cc._ptrs(recv), n, row, cc._ptrs(ids), tokens,
+                         topk, epr, cap, 0, ws.data_ptr(), wsb, st)
+    comb_run = _prepared(cc, "cc_alltoallv_run", cc._ptrs(recv), cc._ptrs(back), n, row, cc._ptrs(ids), tokens,
+                         topk, epr, cap, 1, ws.data_ptr(), wsb, st)
     b_d = n * tokens * row + rows_recv * row
     b_c = 2 * rows_recv * row
-    rows = {"route_topk": timed_row(torch, route, iters, n * tokens * E * 4 + n * tokens * topk * 4, 1, local=local),
+    b_ids = n * tokens * topk * 4
+    rows = {"route_topk": timed_row(torch, route, iters, n * tokens * E * 4 + b_ids, 1, local=local),
             "dispatch": timed_row(torch, disp, iters, b_d, A2A_LAUNCHES, local=local,
                                   kernel="alltoallv dispatch (routing tables + row copy)"),
             "combine": timed_row(torch, comb, iters, b_c, A2A_LAUNCHES, local=local,
-                                 kernel="alltoallv combine (routing tables + row copy)")}
+                                 kernel="alltoallv combine (routing tables + row copy)"),
+            # one routing plan, then the copies alone: the combine reuses the dispatch's routes
+            "plan": timed_row(torch, plan, iters, b_ids, 1, local=local,
+                              kernel="alltoallv routing tables alone (latency-bound: bytes are the ids)"),
+            "dispatch_run": timed_row(torch, disp_run, iters, b_d, 1, local=local,
+                                      kernel="alltoallv dispatch row copy over a plan"),
+            "combine_run": timed_row(torch, comb_run, iters, b_c, 1, local=local,
+                                     kernel="alltoallv combine row copy over a plan")}
     ms = sum(rows[k]["ms"] for k in ("route_topk", "dispatch", "combine"))
+    ms_plan = sum(rows[k]["ms"] for k in ("route_topk", "plan", "dispatch_run", "combine_run"))
     out = {"workload": "config 4 (MoE): N=8 simulated ranks, 8192 tokens x 4096 bf16 per rank, 64 experts (8 per "
                        "rank), top-2 routing from normal logits, dispatch then combine (device-seeded inputs)",
            "l2": "inputs larger than L2; no flush", "rows": rows, "rows_routed_total": rows_recv,
            "route_dispatch_combine": {"ms": ms, "GBps": (b_d + b_c) / (ms * 1e-3) / 1e9},
+           "route_plan_dispatch_combine": {"ms": ms_plan, "GBps": (b_d + b_c) / (ms_plan * 1e-3) / 1e9},
            "traffic_profile": profile_traffic("alltoallv_dispatch_moe.txt")}
     del logits, toks, ids, ws, recv, back
     torch.cuda.empty_cache()
@@ -537,7 +560,7 @@ def launch_latency_s(torch, cc, st):
                      cc.CC_ALGO_RING, 1.0, st)
     for _ in range(10):
         call()
-    times = [_event_time_ms(torch, call, 1) for _ in range(200)]
+    times = [_event_time_ms(torch, call, 1, host_launch=True) for _ in range(200)]
     return statistics.median(times) * 1e-3
 
 

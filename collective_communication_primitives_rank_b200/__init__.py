@@ -58,6 +58,8 @@ _SIGS = {
     "cc_alltoallv_workspace_size": (_sz, [_i, _i, _i, _i]),
     "cc_alltoallv": (_i, [_PP, _PP, _i, _sz, _PP, _i, _i, _i, _sz, _i, _vp, _sz, _vp]),
     "cc_alltoallv_recv_counts": (_i, [_vp, _i, _vp, _vp]),
+    "cc_alltoallv_plan": (_i, [_PP, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "cc_alltoallv_run": (_i, [_PP, _PP, _i, _sz, _PP, _i, _i, _i, _sz, _i, _vp, _sz, _vp]),
     "cc_alltoallv_noalloc": (_i, [_PP, _PP, _i, _sz, _PP, _i, _i, _i, _sz, _i, _vp, _vp]),
     "cc_bucket_assign": (_i, [_SZP, _i, _sz, _sz, _I32P, _I32P, _I32P]),
     "cc_bucket_flatten": (_i, [_PP, _SZP, _i, _vp, _i, _vp]),
@@ -313,12 +315,18 @@ def cc_alltoallv(send, recv, expert_ids, experts_per_rank: int, workspace, *, di
 
     Dispatch: send[s] is [tokens, hidden]; recv[d] holds up to recv_capacity_rows rows.
     Combine: send[d] is rank d's dispatch output; recv[s] is [tokens, topk, hidden]."""
+    _alltoallv(lib.cc_alltoallv, "cc_alltoallv", send, recv, expert_ids, experts_per_rank, workspace,
+               direction, row_bytes, recv_capacity_rows, stream)
+
+
+def _alltoallv(fn, name, send, recv, expert_ids, experts_per_rank, workspace, direction, row_bytes,
+               recv_capacity_rows, stream) -> None:
     torch = _torch()
-    n = _ranks(send, "cc_alltoallv")
+    n = _ranks(send, name)
     if len(recv) != n or len(expert_ids) != n:
-        raise ValueError("cc_alltoallv: one send, recv and id tensor per rank")
+        raise ValueError(f"{name}: one send, recv and id tensor per rank")
     tokens, topk = expert_ids[0].shape
-    _same(expert_ids, tokens * topk, torch.int32, "cc_alltoallv expert_ids")
+    _same(expert_ids, tokens * topk, torch.int32, f"{name} expert_ids")
     tok = send if direction == 0 else recv
     if row_bytes is None:
         row_bytes = tok[0].numel() * tok[0].element_size() // max(1, tokens * (1 if direction == 0 else topk))
@@ -328,12 +336,37 @@ def cc_alltoallv(send, recv, expert_ids, experts_per_rank: int, workspace, *, di
     need = tokens * row_bytes * (1 if direction == 0 else topk)
     for t in tok:
         if t.numel() * t.element_size() < need:
-            raise ValueError("cc_alltoallv: token buffer smaller than tokens x row_bytes (x topk for combine)")
+            raise ValueError(f"{name}: token buffer smaller than tokens x row_bytes (x topk for combine)")
     if workspace.numel() * workspace.element_size() < cc_alltoallv_workspace_size(n, tokens, topk, experts_per_rank):
-        raise ValueError("cc_alltoallv: workspace too small")
-    _check(lib.cc_alltoallv(_ptrs(send), _ptrs(recv), len(send), row_bytes, _ptrs(expert_ids), tokens, topk,
-                            experts_per_rank, recv_capacity_rows, direction, _dev_ptr(workspace),
-                            workspace.numel() * workspace.element_size(), _stream(stream)), "cc_alltoallv")
+        raise ValueError(f"{name}: workspace too small")
+    _check(fn(_ptrs(send), _ptrs(recv), len(send), row_bytes, _ptrs(expert_ids), tokens, topk, experts_per_rank,
+              recv_capacity_rows, direction, _dev_ptr(workspace), workspace.numel() * workspace.element_size(),
+              _stream(stream)), name)
+
+
+def cc_alltoallv_plan(expert_ids, experts_per_rank: int, workspace, *, stream=None) -> None:
+    """Builds in `workspace` the routing tables of expert_ids (one [tokens, topk] int32 tensor per
+    rank), for any number of cc_alltoallv_run calls, dispatch or combine, over that routing."""
+    torch = _torch()
+    n = len(expert_ids)
+    if n < 1:
+        raise ValueError("cc_alltoallv_plan: no ranks")
+    tokens, topk = expert_ids[0].shape
+    _same(expert_ids, tokens * topk, torch.int32, "cc_alltoallv_plan expert_ids")
+    if workspace.numel() * workspace.element_size() < cc_alltoallv_workspace_size(n, tokens, topk, experts_per_rank):
+        raise ValueError("cc_alltoallv_plan: workspace too small")
+    _check(lib.cc_alltoallv_plan(_ptrs(expert_ids), n, tokens, topk, experts_per_rank, _dev_ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream)),
+           "cc_alltoallv_plan")
+
+
+def cc_alltoallv_run(send, recv, expert_ids, experts_per_rank: int, workspace, *, direction: int = 0,
+                     row_bytes: Optional[int] = None, recv_capacity_rows: Optional[int] = None,
+                     stream=None) -> None:
+    """The row copy of cc_alltoallv alone, over the tables the last cc_alltoallv_plan (or
+    cc_alltoallv) left in `workspace` for these same expert_ids; arguments as cc_alltoallv."""
+    _alltoallv(lib.cc_alltoallv_run, "cc_alltoallv_run", send, recv, expert_ids, experts_per_rank, workspace,
+               direction, row_bytes, recv_capacity_rows, stream)
 
 
 def cc_alltoallv_recv_counts(workspace, nranks: int, out, *, stream=None) -> None:

@@ -466,6 +466,31 @@ cc_status cc_alltoallv(const void* const* send, void* const* recv, int nranks, s
                                       recv_capacity_rows, direction, workspace, as_stream(stream)));
 }
 
+cc_status cc_alltoallv_plan(const int32_t* const* expert_ids, int nranks, int tokens, int topk, int experts_per_rank,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  if (!a2a_shape_ok(nranks, tokens, topk, experts_per_rank) ||
+      !all_nonnull((const void* const*)expert_ids, nranks))
+    return CC_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255) ||
+      workspace_bytes < a2a_workspace_bytes(nranks, tokens, topk, experts_per_rank))
+    return CC_ERR_INVALID_ARG;
+  return cuda_status(launch_alltoallv(nullptr, nullptr, nranks, 0, expert_ids, tokens, topk, experts_per_rank, 0, 0,
+                                      workspace, as_stream(stream), kA2ATables));
+}
+
+cc_status cc_alltoallv_run(const void* const* send, void* const* recv, int nranks, size_t row_bytes,
+                           const int32_t* const* expert_ids, int tokens, int topk, int experts_per_rank,
+                           size_t recv_capacity_rows, int direction, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  if (!a2a_args_ok(send, recv, nranks, row_bytes, expert_ids, tokens, topk, experts_per_rank, direction))
+    return CC_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255) ||
+      workspace_bytes < a2a_workspace_bytes(nranks, tokens, topk, experts_per_rank))
+    return CC_ERR_INVALID_ARG;
+  return cuda_status(launch_alltoallv(send, recv, nranks, row_bytes, expert_ids, tokens, topk, experts_per_rank,
+                                      recv_capacity_rows, direction, workspace, as_stream(stream), kA2ACopy));
+}
+
 cc_status cc_alltoallv_recv_counts(const void* workspace, int nranks, int32_t* recv_rows, void* stream) {
   if (!workspace || !recv_rows || !valid_ranks(nranks)) return CC_ERR_INVALID_ARG;
   return cuda_status(copy_recv_counts(workspace, nranks, recv_rows, as_stream(stream)));

@@ -63,9 +63,12 @@ cudaError_t launch_stepped_allreduce(const void* const* send, void* const* recv,
 cudaError_t launch_route_topk(const float* const* logits, int32_t* const* ids, int nranks, int tokens,
                               int experts_total, int topk, cudaStream_t stream);
 size_t a2a_workspace_bytes(int nranks, int tokens, int topk, int experts_per_rank);
+// Which parts of an alltoallv to run: the routing tables (the plan), the row copy, or both.
+enum A2AParts { kA2ATables = 1, kA2ACopy = 2, kA2ABoth = 3 };
 cudaError_t launch_alltoallv(const void* const* send, void* const* recv, int nranks, size_t row_bytes,
                              const int32_t* const* ids, int tokens, int topk, int experts_per_rank,
-                             size_t capacity_rows, int direction, void* workspace, cudaStream_t stream);
+                             size_t capacity_rows, int direction, void* workspace, cudaStream_t stream,
+                             A2AParts parts = kA2ABoth);
 cudaError_t copy_recv_counts(const void* workspace, int nranks, int32_t* out, cudaStream_t stream);
 
 // Device properties, cached per device.

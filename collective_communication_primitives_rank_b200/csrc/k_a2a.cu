@@ -15,6 +15,7 @@
 // last of those the bases and receive counts), then the row copy (one warp per token: the
 // token row is read once and written topk times; combine reads topk rows and writes topk
 // rows). "Last to finish" is an atomic ticket on counters the call clears first.
+// cc_alltoallv_plan launches the first alone, cc_alltoallv_run the second alone.
 #include <algorithm>
 
 #include "cc_device.cuh"
@@ -181,19 +182,24 @@ cudaError_t launch_route_topk(const float* const* logits, int32_t* const* ids, i
 
 constexpr int kScanSplit = 4;  // threads per expert in the per-source tile prefix
 
-// Bases and receive counts from the per-(source, expert) totals, by one CTA: the totals are
-// staged in shared memory (`sm`: nranks * E + nranks * nranks ints) with one coalesced pass.
+// Bases and receive counts from the per-(source, expert) totals, by one CTA. `sm` holds
+// sm_ints ints: the rows s -> d (nranks^2 <= 4096 ints) first, then, when they fit, the totals
+// staged with one coalesced pass (nranks * E ints: up to 64 x 1024); otherwise the totals are
+// read from global memory.
 __device__ __forceinline__ void bases_and_counts(int nranks, int epr, const int* tot_g, int* base, int* recv_count,
-                                                 int* sm) {
+                                                 int* sm, int sm_ints) {
   const int E = nranks * epr;
-  int* tot = sm;
-  int* cnt = sm + nranks * E;  // rows s -> d
-  for (int i = threadIdx.x; i < nranks * E; i += blockDim.x) tot[i] = __ldcg(tot_g + i);
+  int* cnt = sm;  // rows s -> d
+  int* tot_s = sm + nranks * nranks;
+  const bool staged = nranks * nranks + nranks * E <= sm_ints;
+  const int* tot = staged ? tot_s : tot_g;
+  if (staged)
+    for (int i = threadIdx.x; i < nranks * E; i += blockDim.x) tot_s[i] = __ldcg(tot_g + i);
   __syncthreads();
   for (int i = threadIdx.x; i < nranks * nranks; i += blockDim.x) {
     const int s = i / nranks, d = i % nranks;
     int c = 0;
-    for (int l = 0; l < epr; ++l) c += tot[s * E + d * epr + l];
+    for (int l = 0; l < epr; ++l) c += staged ? tot[s * E + d * epr + l] : __ldcg(tot + s * E + d * epr + l);
     cnt[i] = c;
   }
   __syncthreads();
@@ -201,7 +207,7 @@ __device__ __forceinline__ void bases_and_counts(int nranks, int epr, const int*
     const int s = i / E, e = i % E, d = e / epr;
     int off = 0;
     for (int sp = 0; sp < s; ++sp) off += cnt[sp * nranks + d];
-    for (int l = d * epr; l < e; ++l) off += tot[s * E + l];
+    for (int l = d * epr; l < e; ++l) off += staged ? tot[s * E + l] : __ldcg(tot + s * E + l);
     base[i] = off;
   }
   for (int d = threadIdx.x; d < nranks; d += blockDim.x) {
@@ -211,13 +217,17 @@ __device__ __forceinline__ void bases_and_counts(int nranks, int epr, const int*
   }
 }
 
+// Dynamic shared memory of the table kernel, in ints (with its static words, within the 48 KiB
+// a launch gets without opting in): a tile's [8][E] warp counts, the source's [tiles][E] counts
+// when they fit kScanSmemInts, and the bases' rows s -> d with the totals when they fit.
+constexpr int kTablesSmemInts = 12000;
 constexpr int kScanSmemInts = 10240;  // a source's [tiles][experts] counts scanned in shared memory up to this
 
 __global__ void __launch_bounds__(kTileRows) a2a_tables_kernel(const __grid_constant__ IdPtrs I, int rows, int nranks,
                                                                int epr, int* __restrict__ tile_cnt,
                                                                int* __restrict__ row_rank, int* __restrict__ totals,
                                                                int* __restrict__ base, int* __restrict__ recv_count,
-                                                               unsigned* __restrict__ done) {
+                                                               unsigned* __restrict__ done, int sm_ints) {
   extern __shared__ int warp_cnt[];  // [8][E]; reused by the last CTAs (scan, then bases)
   __shared__ int s_last;
   // the copy kernel (a programmatic dependent) may launch now: it waits for this grid to
@@ -304,7 +314,7 @@ __global__ void __launch_bounds__(kTileRows) a2a_tables_kernel(const __grid_cons
     for (size_t i = threadIdx.x; i < blk; i += blockDim.x) src_cnt[i] = warp_cnt[i];
     if (!s_last) return;
     __syncthreads();  // every thread is done with warp_cnt before the bases reuse it
-    bases_and_counts(nranks, epr, totals, base, recv_count, warp_cnt);
+    bases_and_counts(nranks, epr, totals, base, recv_count, warp_cnt, sm_ints);
     return;
   } else {
     const int q = threadIdx.x % kScanSplit;
@@ -341,54 +351,54 @@ __global__ void __launch_bounds__(kTileRows) a2a_tables_kernel(const __grid_cons
   }
   __syncthreads();
   if (!s_last) return;
-  bases_and_counts(nranks, epr, totals, base, recv_count, warp_cnt);
+  bases_and_counts(nranks, epr, totals, base, recv_count, warp_cnt, sm_ints);
 }
 
 // ---- no rows: bases and receive counts from zero totals (one CTA) ------------------------------------
 
+constexpr int kBaseSmemInts = 8192;
+
 __global__ void __launch_bounds__(1024) a2a_base_kernel(int nranks, int epr, const int* __restrict__ tot,
                                                         int* __restrict__ base, int* __restrict__ recv_count) {
-  __shared__ int sm[1024 + kMaxRanks * kMaxRanks];  // totals (N * E <= 1024), then rows s -> d
-  bases_and_counts(nranks, epr, tot, base, recv_count, sm);
+  __shared__ int sm[kBaseSmemInts];
+  bases_and_counts(nranks, epr, tot, base, recv_count, sm, kBaseSmemInts);
 }
 
-// ---- K4: row copies ----------------------------------------------------------------------------------
+// ---- row copies ---------------------------------------------------------------------------------------
 
 struct A2ACopyParams {
   const char* send[kMaxRanks];
   char* recv[kMaxRanks];
   const int32_t* ids[kMaxRanks];
-  const int* tile_off;   // [N][ntiles][E]
-  const int* row_rank;   // [N][rows]
+  const int* tile_off;   // [N][ntiles][E] exclusive prefixes over tiles
+  const int* row_rank;   // [N][rows] rank in the row's tile
   const int* base;       // [N][E]
   uint64_t row_bytes;
   uint64_t capacity;
   int tokens, topk, epr, E, ntiles, direction;
 };
 
-// The copy is launched as a programmatic dependent of the table kernel: its CTAs may start
-// while the tables are still being built, and wait (griddepcontrol.wait) for the table kernel
-// to complete before they read a position. A dispatch row does not depend on the tables, so its
-// first 16 vectors per lane are loaded before that wait.
-__device__ __forceinline__ void wait_for_tables() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+constexpr int kCopyVecs = 16;  // 16-byte loads per lane in flight before the stores that consume
+                               // them (a whole 8 KiB row per warp; measured faster than 8 or 32)
 
-__global__ void __launch_bounds__(256) a2a_copy_kernel(const __grid_constant__ A2ACopyParams P) {
-  const int lane = threadIdx.x & 31;
-  const int s = blockIdx.y;
-  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (t >= P.tokens) return;
-  // 16 loads per lane in flight before the stores that consume them (a whole 8 KiB row per
-  // warp; measured faster than 8 or 32)
-  constexpr int B = 16;
+// The first kCopyVecs vectors per lane of a dispatch row (the token row of source s).
+__device__ __forceinline__ void load_token_head(const A2ACopyParams& P, int s, int t, int lane, uint4 (&x)[kCopyVecs]) {
   const uint64_t nvec = P.row_bytes / 16;
-  uint4 x[B];
   const uint4* row = reinterpret_cast<const uint4*>(P.send[s] + (uint64_t)t * P.row_bytes);
-  if (P.direction == 0) {
 #pragma unroll
-    for (int b = 0; b < B; ++b)
-      if (lane + 32 * b < nvec) x[b] = __ldcs(row + lane + 32 * b);
-  }
-  wait_for_tables();
+  for (int b = 0; b < kCopyVecs; ++b)
+    if (lane + 32 * b < nvec) x[b] = __ldcs(row + lane + 32 * b);
+}
+
+// One token of source s, by one warp: dispatch writes its row to each selected expert's
+// position; combine reads the rows back from those positions into slots [t][k]. `base` is
+// [N][E] in global or shared memory; the tile prefixes and ranks are read through L2 (another
+// SM may have written them in the same launch). With `head` the dispatch row's first vectors
+// are already in x.
+__device__ __forceinline__ void copy_token(const A2ACopyParams& P, const int* base, int s, int t, int lane,
+                                           uint4 (&x)[kCopyVecs], bool head) {
+  constexpr int B = kCopyVecs;
+  const uint64_t nvec = P.row_bytes / 16;
   const int rows = P.tokens * P.topk;
   char* ptr[kMaxTopk];
   bool ok[kMaxTopk];
@@ -397,15 +407,16 @@ __global__ void __launch_bounds__(256) a2a_copy_kernel(const __grid_constant__ A
     const int e = P.ids[s][i];
     if (e < 0 || e >= P.E) { ok[k] = false; ptr[k] = nullptr; continue; }
     const int d = e / P.epr;
-    const uint64_t pos = (uint64_t)P.base[s * P.E + e] +
-                         P.tile_off[((size_t)s * P.ntiles + i / kTileRows) * P.E + e] +
-                         P.row_rank[(size_t)s * rows + i];
+    const uint64_t pos = (uint64_t)base[s * P.E + e] +
+                         __ldcg(P.tile_off + ((size_t)s * P.ntiles + i / kTileRows) * P.E + e) +
+                         __ldcg(P.row_rank + (size_t)s * rows + i);
     ok[k] = pos < P.capacity;
     ptr[k] = (P.direction == 0 ? P.recv[d] : const_cast<char*>(P.send[d])) + pos * P.row_bytes;
   }
   if (P.direction == 0) {
+    const uint4* row = reinterpret_cast<const uint4*>(P.send[s] + (uint64_t)t * P.row_bytes);
     for (uint64_t v0 = lane; v0 < nvec; v0 += 32 * B) {
-      if (v0 != (uint64_t)lane) {
+      if (v0 != (uint64_t)lane || !head) {
 #pragma unroll
         for (int b = 0; b < B; ++b)
           if (v0 + 32 * b < nvec) x[b] = __ldcs(row + v0 + 32 * b);
@@ -436,9 +447,51 @@ __global__ void __launch_bounds__(256) a2a_copy_kernel(const __grid_constant__ A
   }
 }
 
+// The copy alone, one warp per token. After a table kernel it is launched as that kernel's
+// programmatic dependent: its CTAs may start while the tables are still being built, and wait
+// (griddepcontrol.wait) for the table kernel to complete before they read a position. A
+// dispatch row does not depend on the tables, so its first vectors are loaded before that wait.
+// Launched on its own (a run over an earlier plan) it follows plain stream order, where the
+// wait returns at once.
+__global__ void __launch_bounds__(256) a2a_copy_kernel(const __grid_constant__ A2ACopyParams P) {
+  const int lane = threadIdx.x & 31;
+  const int s = blockIdx.y;
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= P.tokens) return;
+  uint4 x[kCopyVecs];
+  if (P.direction == 0) load_token_head(P, s, t, lane, x);
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  copy_token(P, P.base, s, t, lane, x, P.direction == 0);
+}
+
+static A2ACopyParams copy_params(const void* const* send, void* const* recv, int nranks, size_t row_bytes,
+                                 const int32_t* const* ids, int tokens, int topk, int experts_per_rank,
+                                 size_t capacity_rows, int direction, const int* tile_off, const int* row_rank,
+                                 const int* base) {
+  A2ACopyParams P{};
+  for (int r = 0; r < nranks; ++r) {
+    P.send[r] = static_cast<const char*>(send[r]);
+    P.recv[r] = static_cast<char*>(recv[r]);
+    P.ids[r] = ids[r];
+  }
+  P.tile_off = tile_off;
+  P.row_rank = row_rank;
+  P.base = base;
+  P.row_bytes = row_bytes;
+  P.capacity = capacity_rows;
+  P.tokens = tokens;
+  P.topk = topk;
+  P.epr = experts_per_rank;
+  P.E = nranks * experts_per_rank;
+  P.ntiles = (tokens * topk + kTileRows - 1) / kTileRows;
+  P.direction = direction;
+  return P;
+}
+
 cudaError_t launch_alltoallv(const void* const* send, void* const* recv, int nranks, size_t row_bytes,
                              const int32_t* const* ids, int tokens, int topk, int experts_per_rank,
-                             size_t capacity_rows, int direction, void* workspace, cudaStream_t stream) {
+                             size_t capacity_rows, int direction, void* workspace, cudaStream_t stream,
+                             A2AParts parts) {
   const int E = nranks * experts_per_rank;
   const int rows = tokens * topk;
   const int ntiles = (rows + kTileRows - 1) / kTileRows;
@@ -449,44 +502,35 @@ cudaError_t launch_alltoallv(const void* const* send, void* const* recv, int nra
   int* totals = reinterpret_cast<int*>(ws + w.totals);
   int* base = reinterpret_cast<int*>(ws + w.base);
   int* recv_count = reinterpret_cast<int*>(ws + w.recv_count);
+  unsigned* done = reinterpret_cast<unsigned*>(ws + w.done);
   IdPtrs I{};
   for (int r = 0; r < nranks; ++r) I.ids[r] = ids[r];
-  if (rows > 0) {
-    // the finish tickets start at zero (stream-ordered), then one launch builds every table
-    unsigned* done = reinterpret_cast<unsigned*>(ws + w.done);
-    const cudaError_t e = cudaMemsetAsync(done, 0, sizeof(unsigned) * (kMaxRanks + 1), stream);
-    if (e != cudaSuccess) return e;
-    const size_t scan = std::min<size_t>((size_t)ntiles * E, kScanSmemInts);
-    const size_t smem = sizeof(int) * std::max<size_t>(std::max<size_t>(8 * E, nranks * E + nranks * nranks), scan);
-    a2a_tables_kernel<<<dim3(ntiles, nranks), kTileRows, smem, stream>>>(I, rows, nranks, experts_per_rank,
-                                                                         tile_cnt, row_rank, totals, base,
-                                                                         recv_count, done);
-  } else {
-    // no rows: the bases read zero totals (the only write to this scratch before them)
-    const cudaError_t e = cudaMemsetAsync(totals, 0, sizeof(int) * nranks * E, stream);
-    if (e != cudaSuccess) return e;
-    a2a_base_kernel<<<1, 1024, 0, stream>>>(nranks, experts_per_rank, totals, base, recv_count);
+  if (parts & kA2ATables) {
+    if (rows > 0) {
+      // the finish tickets start at zero (stream-ordered), then one launch builds every table
+      const cudaError_t e = cudaMemsetAsync(done, 0, sizeof(unsigned) * (kMaxRanks + 1), stream);
+      if (e != cudaSuccess) return e;
+      const int scan = (int)std::min<size_t>((size_t)ntiles * E, kScanSmemInts);
+      const int bases = std::min(nranks * nranks + nranks * E, kTablesSmemInts);
+      const int sm_ints = std::max(std::max(8 * E, nranks * nranks), std::max(scan, bases));
+      a2a_tables_kernel<<<dim3(ntiles, nranks), kTileRows, sizeof(int) * sm_ints, stream>>>(
+          I, rows, nranks, experts_per_rank, tile_cnt, row_rank, totals, base, recv_count, done, sm_ints);
+    } else {
+      // no rows: the bases read zero totals (the only write to this scratch before them)
+      const cudaError_t e = cudaMemsetAsync(totals, 0, sizeof(int) * nranks * E, stream);
+      if (e != cudaSuccess) return e;
+      a2a_base_kernel<<<1, 1024, 0, stream>>>(nranks, experts_per_rank, totals, base, recv_count);
+    }
+    const cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
   }
-  cudaError_t err = cudaGetLastError();
-  if (err != cudaSuccess || rows == 0) return err;
-  A2ACopyParams P{};
-  for (int r = 0; r < nranks; ++r) {
-    P.send[r] = static_cast<const char*>(send[r]);
-    P.recv[r] = static_cast<char*>(recv[r]);
-    P.ids[r] = ids[r];
-  }
-  P.tile_off = tile_cnt;
-  P.row_rank = row_rank;
-  P.base = base;
-  P.row_bytes = row_bytes;
-  P.capacity = capacity_rows;
-  P.tokens = tokens;
-  P.topk = topk;
-  P.epr = experts_per_rank;
-  P.E = E;
-  P.ntiles = ntiles;
-  P.direction = direction;
-  // a programmatic dependent of the table kernel (see a2a_copy_kernel)
+  // the copy; with parts == kA2ACopy it reads the tables an earlier plan left in the workspace
+  if (!(parts & kA2ACopy) || rows == 0) return cudaSuccess;
+  const A2ACopyParams P = copy_params(send, recv, nranks, row_bytes, ids, tokens, topk, experts_per_rank,
+                                      capacity_rows, direction, tile_cnt, row_rank, base);
+  // a programmatic dependent of the table kernel launched just before it (see a2a_copy_kernel).
+  // A copy on its own follows plain stream order: the kernel before it may be the one that
+  // writes the rows this copy reads ahead of its griddepcontrol.wait.
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((tokens + 7) / 8, nranks);
   cfg.blockDim = dim3(256);
@@ -496,7 +540,7 @@ cudaError_t launch_alltoallv(const void* const* send, void* const* recv, int nra
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = (parts & kA2ATables) ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, a2a_copy_kernel, P);
 }
 

@@ -211,12 +211,33 @@ CC_API size_t cc_alltoallv_workspace_size(int nranks, int tokens, int topk, int 
  *   cc_alltoallv_recv_counts tells the true counts).
  * Combine: send[d] is rank d's [rows, row_bytes] buffer in dispatch order; recv[s] is
  *   [tokens, topk, row_bytes] and receives each row back at slot [t][k].
+ * An expert id outside [0, N * experts_per_rank) routes its row nowhere: dispatch sends it
+ *   to no rank and combine leaves slot [t][k] of recv[s] as it was (so does a row that the
+ *   capacity dropped).
  * Both directions rebuild the routing table from expert_ids in `workspace`.
  * row_bytes must be a positive multiple of 16. */
 CC_API cc_status cc_alltoallv(const void* const* send, void* const* recv, int nranks, size_t row_bytes,
                        const int32_t* const* expert_ids, int tokens, int topk, int experts_per_rank,
                        size_t recv_capacity_rows, int direction, void* workspace,
                        size_t workspace_bytes, void* stream);
+
+/* The two halves of cc_alltoallv, for a routing that serves more than one call (lecture 09
+ * §6.4: the second AllToAll sends the experts' outputs back along the routes of the first, so
+ * a dispatch and its combine share one routing).
+ * cc_alltoallv_plan builds in `workspace` the routing tables cc_alltoallv builds at every call
+ * (per-source tile counts and prefixes, per-row ranks, bases, receive counts) from expert_ids;
+ * cc_alltoallv_run does only the row copy of cc_alltoallv, in either direction, reading the
+ * tables that the last plan (or the last cc_alltoallv) left in `workspace`. A run gives exactly
+ * cc_alltoallv's result as long as expert_ids, tokens, topk, experts_per_rank and nranks are
+ * those of that plan and nothing else wrote the workspace in between; after expert_ids change,
+ * plan again. Arguments, layouts, workspace rules and errors as cc_alltoallv (plan takes no
+ * row buffers). cc_alltoallv_recv_counts reads the counts of the last plan. */
+CC_API cc_status cc_alltoallv_plan(const int32_t* const* expert_ids, int nranks, int tokens, int topk,
+                                   int experts_per_rank, void* workspace, size_t workspace_bytes, void* stream);
+CC_API cc_status cc_alltoallv_run(const void* const* send, void* const* recv, int nranks, size_t row_bytes,
+                                  const int32_t* const* expert_ids, int tokens, int topk, int experts_per_rank,
+                                  size_t recv_capacity_rows, int direction, void* workspace,
+                                  size_t workspace_bytes, void* stream);
 
 /* Copies the per-destination received row counts of the last cc_alltoallv that used
  * `workspace` into recv_rows[0..nranks) (host or device memory), stream-ordered. */

@@ -125,6 +125,14 @@ def test_other_entry_points_validate(lib):
     assert lib.cc_alltoallv(p4, p4, 4, 64, p4, 10, 2, 2, 100, 0, FAKE[0], 16, 16, None) == cc.CC_ERR_INVALID_ARG
     assert lib.cc_alltoallv(p4, p4, 4, 64, p4, 10, 2, 2, 100, 2, FAKE[0], ws, ws, None) == cc.CC_ERR_INVALID_ARG
     assert lib.cc_alltoallv_workspace_size(65, 10, 2, 2) == 0
+    # the plan / run halves check what cc_alltoallv checks
+    assert lib.cc_alltoallv_plan(p4, 4, 10, 9, 2, FAKE[0], ws, None) == cc.CC_ERR_INVALID_ARG      # topk > 8
+    assert lib.cc_alltoallv_plan(None, 4, 10, 2, 2, FAKE[0], ws, None) == cc.CC_ERR_INVALID_ARG    # no ids
+    assert lib.cc_alltoallv_plan(p4, 4, 10, 2, 2, FAKE[0] + 8, ws, None) == cc.CC_ERR_INVALID_ARG  # misaligned
+    assert lib.cc_alltoallv_plan(p4, 4, 10, 2, 2, FAKE[0], 16, None) == cc.CC_ERR_INVALID_ARG      # too small
+    assert lib.cc_alltoallv_run(p4, p4, 4, 60, p4, 10, 2, 2, 100, 0, FAKE[0], ws, None) == cc.CC_ERR_INVALID_ARG
+    assert lib.cc_alltoallv_run(p4, p4, 4, 64, p4, 10, 2, 2, 100, 2, FAKE[0], ws, None) == cc.CC_ERR_INVALID_ARG
+    assert lib.cc_alltoallv_run(p4, p4, 4, 64, p4, 10, 2, 2, 100, 0, FAKE[0], 16, None) == cc.CC_ERR_INVALID_ARG
     sizes = (ctypes.c_size_t * 2)(10, 10)
     assert lib.cc_bucket_allreduce(p4, p4, 2, 2, sizes, 0, 0, 0.5, None) == cc.CC_ERR_INVALID_ARG  # cap 0
     assert lib.cc_bucket_allreduce(p4, p4, 2, 0, sizes, 100, 0, 0.5, None) == cc.CC_OK  # nothing to do

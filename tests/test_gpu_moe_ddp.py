@@ -43,8 +43,11 @@ def _moe_case(n, tokens, hidden, epr, seed=2):
 
 # (4, 3000, 16, 256): 24 tiles x 1024 experts per source, more counts than the table kernel scans
 # in shared memory, so the per-source prefix runs on its global-memory path
+# (16, 300, 16, 64): 16 x 1024 totals, more than one CTA stages, so cc_alltoallv takes the
+# separate table and copy launches instead of the single cooperative one
 @pytest.mark.parametrize("n,tokens,hidden,epr", [(8, 300, 64, 8), (4, 1000, 8, 2), (3, 17, 16, 1), (1, 50, 8, 4),
-                                                 (8, 2048, 4096, 8), (4, 3000, 16, 256)])
+                                                 (8, 2048, 4096, 8), (4, 3000, 16, 256), (2, 20000, 8, 4),
+                                                 (5, 16384, 16, 6), (16, 300, 16, 64)])
 def test_alltoallv_dispatch_and_combine_match_oracle(n, tokens, hidden, epr):
     ids, toks = _moe_case(n, tokens, hidden, epr)
     want, _ = moe.dispatch(toks, ids, epr)
@@ -68,6 +71,115 @@ def test_alltoallv_dispatch_and_combine_match_oracle(n, tokens, hidden, epr):
     for s in range(n):
         assert np.array_equal(to_host(back[s].t), combined[s]), f"combine rank {s}"
         back[s].check()
+
+
+@pytest.mark.parametrize("n,tokens,hidden,epr", [(8, 300, 64, 8), (3, 17, 16, 1), (4, 3000, 16, 256),
+                                                 (16, 300, 16, 64)])
+def test_alltoallv_plan_then_runs_match_oracle(n, tokens, hidden, epr):
+    """One plan serves a dispatch and its combine, twice over; after the ids change, a new plan
+    gives the new routing (the second routing is a different seed, same shape)."""
+    ws = torch.empty(cc.cc_alltoallv_workspace_size(n, tokens, 2, epr) // 4 + 64, dtype=torch.int32, device="cuda")
+    for seed in (3, 11):
+        ids, toks = _moe_case(n, tokens, hidden, epr, seed=seed)
+        want, _ = moe.dispatch(toks, ids, epr)
+        combined, _ = moe.combine(want, ids, epr)
+        cap = max(w.shape[0] for w in want) + 5
+        d_ids = [to_dev(i) for i in ids]
+        d_tok = [to_dev(t) for t in toks]
+        cc.cc_alltoallv_plan(d_ids, epr, ws)
+        counts = torch.zeros(n, dtype=torch.int32, device="cuda")
+        cc.cc_alltoallv_recv_counts(ws, n, counts)
+        for _ in range(2):
+            recv = [Guarded(cap * hidden, torch.bfloat16, shape=(cap, hidden)) for _ in range(n)]
+            back = [Guarded(tokens * 2 * hidden, torch.bfloat16, shape=(tokens, 2, hidden)) for _ in range(n)]
+            cc.cc_alltoallv_run(d_tok, [g.t for g in recv], d_ids, epr, ws, direction=0)
+            cc.cc_alltoallv_run([g.t for g in recv], [g.t for g in back], d_ids, epr, ws, direction=1)
+            torch.cuda.synchronize()
+            assert to_host(counts).tolist() == [w.shape[0] for w in want]
+            for d in range(n):
+                assert np.array_equal(to_host(recv[d].t)[:want[d].shape[0]], want[d]), f"dispatch rank {d}"
+                recv[d].check()
+            for s in range(n):
+                assert np.array_equal(to_host(back[s].t), combined[s]), f"combine rank {s}"
+                back[s].check()
+
+
+@pytest.mark.parametrize("n,epr", [(4, 2), (8, 32), (16, 64), (64, 16)])
+def test_alltoallv_without_tokens_reports_zero_rows(n, epr):
+    """tokens = 0 at every size of the N x E totals (up to 64 ranks x 1024 experts): nothing
+    is copied and the receive counts are zeros, whatever an earlier plan left in the workspace."""
+    ids, _ = _moe_case(n, 40, 8, epr, seed=6)
+    ws = torch.empty(cc.cc_alltoallv_workspace_size(n, 40, 2, epr) // 4 + 64, dtype=torch.int32, device="cuda")
+    cc.cc_alltoallv_plan([to_dev(i) for i in ids], epr, ws)
+    ids1 = [torch.zeros(1, 2, dtype=torch.int32, device="cuda") for _ in range(n)]  # tokens = 0 below
+    tok = [torch.zeros(1, 16, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+    out = [torch.full((4, 16), 3.0, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+    st = cc.lib.cc_alltoallv(cc._ptrs(tok), cc._ptrs(out), n, 32, cc._ptrs(ids1), 0, 2, epr, 4, 0, ws.data_ptr(),
+                             ws.numel() * 4, torch.cuda.current_stream().cuda_stream)
+    assert st == cc.CC_OK
+    counts = torch.full((n,), -1, dtype=torch.int32, device="cuda")
+    cc.cc_alltoallv_recv_counts(ws, n, counts)
+    torch.cuda.synchronize()
+    assert counts.tolist() == [0] * n
+    assert all(bool((o == 3.0).all()) for o in out)
+
+
+def test_alltoallv_run_reads_rows_written_just_before_it():
+    """A run launched right after the kernel that writes its send rows sees those rows: the
+    rows are rewritten on the device between plan and run, with no host sync in between."""
+    n, tokens, hidden, epr = 4, 4096, 2048, 4
+    ids, toks = _moe_case(n, tokens, hidden, epr, seed=5)
+    want, _ = moe.dispatch(toks, ids, epr)
+    cap = max(w.shape[0] for w in want)
+    d_ids = [to_dev(i) for i in ids]
+    d_tok = [to_dev(t) for t in toks]
+    ws = torch.empty(cc.cc_alltoallv_workspace_size(n, tokens, 2, epr) // 4 + 64, dtype=torch.int32, device="cuda")
+    recv = [torch.empty(cap, hidden, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+    stale = [torch.zeros_like(t) for t in d_tok]
+    cc.cc_alltoallv_plan(d_ids, epr, ws)
+    for s in range(n):
+        stale[s].copy_(d_tok[s])          # device writes of the send rows, stream-ordered before the run
+    cc.cc_alltoallv_run(stale, recv, d_ids, epr, ws, direction=0)
+    torch.cuda.synchronize()
+    for d in range(n):
+        assert np.array_equal(to_host(recv[d])[:want[d].shape[0]], want[d]), f"dispatch rank {d}"
+
+
+@pytest.mark.parametrize("n,tokens,epr", [(4, 700, 3), (2, 20000, 4), (4, 3000, 256), (16, 300, 64)])
+def test_alltoallv_out_of_range_ids_route_nowhere(n, tokens, epr):
+    """Ids below 0 or at / past N * experts_per_rank are sent to no rank (the oracle's send
+    lists hold no such row); combine leaves their slots as they were."""
+    hidden = 8
+    ids, toks = _moe_case(n, tokens, hidden, epr, seed=13)
+    E = n * epr
+    rng = np.random.default_rng(4)
+    for r in range(n):
+        flat = ids[r].reshape(-1).copy()
+        pick = rng.choice(flat.size, size=flat.size // 7, replace=False)
+        flat[pick] = rng.choice(np.array([-1, -5, E, E + 3, 2 ** 31 - 1], dtype=np.int32), size=pick.size)
+        ids[r] = flat.reshape(ids[r].shape)
+    want, _ = moe.dispatch(toks, ids, epr)
+    combined, _ = moe.combine(want, ids, epr)
+    cap = max(w.shape[0] for w in want) + 2
+    d_ids = [to_dev(i) for i in ids]
+    recv = [Guarded(cap * hidden, torch.bfloat16, shape=(cap, hidden)) for _ in range(n)]
+    ws = torch.empty(cc.cc_alltoallv_workspace_size(n, tokens, 2, epr) // 4 + 64, dtype=torch.int32, device="cuda")
+    cc.cc_alltoallv([to_dev(t) for t in toks], [g.t for g in recv], d_ids, epr, ws, direction=0)
+    counts = torch.zeros(n, dtype=torch.int32, device="cuda")
+    cc.cc_alltoallv_recv_counts(ws, n, counts)
+    back = [torch.full((tokens, 2, hidden), 7.0, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+    cc.cc_alltoallv([g.t for g in recv], back, d_ids, epr, ws, direction=1)
+    torch.cuda.synchronize()
+    assert to_host(counts).tolist() == [w.shape[0] for w in want]
+    seven = to_host(torch.full((1,), 7.0, dtype=torch.bfloat16))[0]
+    for d in range(n):
+        assert np.array_equal(to_host(recv[d].t)[:want[d].shape[0]], want[d]), f"dispatch rank {d}"
+        recv[d].check()
+    for s in range(n):
+        got = to_host(back[s])
+        bad = (ids[s] < 0) | (ids[s] >= E)
+        assert np.array_equal(got[~bad], combined[s][~bad]), f"combine rank {s}"
+        assert (got[bad] == seven).all(), f"combine rank {s}: an unrouted slot was written"
 
 
 def test_alltoallv_capacity_drops_overflow_rows_only():
