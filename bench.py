@@ -368,7 +368,7 @@ def rows_config1(torch, cc, local, with_cpu=True):
     out = {"workload": "config 1: N=4 simulated ranks x 4096 elements, fp32 U[-1,1] and int32 U[-1000,1000] "
                        "(host-seeded), ring allreduce / reduce-scatter / allgather and tree allreduce; latency-bound",
            "l2": "256 MiB flush before every timed call",
-           "timing": "us: CUDA events around each call (includes the host's launch cost); device_us: the same calls "
+           "timing": "us: CUDA events around each call, opened behind the L2 flush; device_us: the same calls "
                      "replayed from a CUDA graph, flush graph subtracted",
            "rows": rows}
     if with_cpu:
