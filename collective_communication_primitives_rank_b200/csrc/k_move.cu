@@ -6,11 +6,15 @@
 // a CTA finds its tile's entry by binary search in the tile prefix table.
 //
 // copy_bulk_tile_kernel (every entry 16-byte aligned): the tensor memory accelerator moves
-// the data. One CTA per 32 KiB tile; its one working thread issues a cp.async.bulk load of
-// the tile into shared memory (completion on an mbarrier), then one cp.async.bulk store of
-// the same shared-memory tile per destination, so a tile costs the SM a handful of
-// instructions however many replicas it has, and several CTAs per SM keep loads in flight.
-// (Measured against a persistent 4-stage pipeline per SM: 98–100% vs 88% of the copy rate.)
+// the data. One CTA per tile; its one working thread issues a cp.async.bulk load of the
+// tile into shared memory (completion on an mbarrier), then one cp.async.bulk store of the
+// same shared-memory tile per destination, so a tile costs the SM a handful of instructions
+// however many replicas it has, and several CTAs per SM keep loads in flight. (Measured
+// against a persistent 4-stage pipeline per SM: 98–100% vs 88% of the copy rate.) Tiles are
+// 2 KiB (32 CTAs per SM) for a launch that reads less than 1 GiB and 32 KiB above: measured on
+// allgather N = 8..64 × 16–512 MiB, broadcast and scatter, 2 KiB tiles took the write-heavy
+// fan-out from 5.3–6.5 to 6.2–6.8 TB/s, while the 1.2 GB shards of an N = 8 allgather ran 2%
+// slower with them than with 32 KiB tiles; 1 KiB tiles halved a one-destination copy.
 // The wait is bounded: one that gives up records CC_ERR_TIMEOUT in the device status word.
 //
 // copy_kernel (any alignment): 128-bit streaming loads/stores per thread where an entry is
@@ -28,6 +32,7 @@ constexpr int kCopyMaxEntries = 128;
 constexpr uint64_t kCopyTile = 64 * 1024;  // bytes
 
 struct CopyParams {
+  uint32_t bulk_tile;  // bytes per CTA of copy_bulk_tile_kernel
   int nentries;
   int fanout;
   int ndst;
@@ -85,7 +90,9 @@ __global__ void __launch_bounds__(kCopyThreads) copy_kernel(const __grid_constan
 
 __device__ int g_async_status;  // CC_OK, or CC_ERR_TIMEOUT after a bounded wait gave up
 
-constexpr uint32_t kBulkTile = 32 * 1024;  // bytes; a multiple of 16
+constexpr uint32_t kBulkTileSmall = 2 * 1024;   // bytes; multiples of 16
+constexpr uint32_t kBulkTileLarge = 32 * 1024;
+constexpr uint64_t kBulkLargeLaunch = 1ull << 30;  // source bytes from which a launch takes large tiles
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // a wait gives up after 2 s (no load takes that long)
 constexpr long kWaitPolls = 1l << 30;             // and after this many polls, whatever the clock says
 
@@ -147,7 +154,8 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 // keep loads in flight; the hardware hands out tiles as CTAs finish.
 __global__ void __launch_bounds__(32) copy_bulk_tile_kernel(const __grid_constant__ CopyParams P) {
   extern __shared__ __align__(128) unsigned char smem[];
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kBulkTile);
+  const uint32_t tile_bytes = P.bulk_tile;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + tile_bytes);
   if (threadIdx.x != 0) return;
   const uint32_t tile = blockIdx.x;
   if (tile >= P.tile_prefix[P.nentries]) return;
@@ -157,8 +165,8 @@ __global__ void __launch_bounds__(32) copy_bulk_tile_kernel(const __grid_constan
     if (P.tile_prefix[mid] <= tile) lo = mid; else hi = mid - 1;
   }
   const int k = lo;
-  const uint64_t a = (uint64_t)(tile - P.tile_prefix[k]) * kBulkTile;
-  const uint32_t bytes = (uint32_t)min((uint64_t)kBulkTile, P.nbytes[k] - a);
+  const uint64_t a = (uint64_t)(tile - P.tile_prefix[k]) * tile_bytes;
+  const uint32_t bytes = (uint32_t)min((uint64_t)tile_bytes, P.nbytes[k] - a);
   const uint32_t bulk = bytes & ~15u;
   if (bulk) {
     mbar_init(bar);
@@ -170,7 +178,7 @@ __global__ void __launch_bounds__(32) copy_bulk_tile_kernel(const __grid_constan
       // the CTA leaves with the bulk load in flight: that load may still write this CTA's
       // shared memory after the SM has handed it to another CTA (of this or any kernel),
       // so the outputs of this call and of whatever runs next on that SM are undefined; the
-      // status word reads CC_ERR_TIMEOUT (only a memory system that stalls a 32 KiB read for
+      // status word reads CC_ERR_TIMEOUT (only a memory system that stalls a 2 KiB read for
       // seconds gets here)
       mbar_wait(bar, 0);
       return;
@@ -225,7 +233,7 @@ cudaError_t launch_copy(const CopyEntry* entries, int nentries, void* const* dst
   static int bps = 0;
   if (!bps && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, copy_kernel, kCopyThreads, 0) != cudaSuccess || bps <= 0))
     bps = 4;
-  static const size_t bulk_smem = (size_t)kBulkTile + 16;
+  static const size_t bulk_smem = (size_t)kBulkTileLarge + 16;
   static const cudaError_t bulk_attr =
       cudaFuncSetAttribute(copy_bulk_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bulk_smem);
   bool bases_aligned = true;
@@ -261,14 +269,17 @@ cudaError_t launch_copy(const CopyEntry* entries, int nentries, void* const* dst
     bool all_vec = true;
     for (int k = 0; k < m; ++k) all_vec = all_vec && ((P.vec_mask[k >> 6] >> (k & 63)) & 1);
     if (all_vec && !plain && bulk_attr == cudaSuccess) {
-      // retile for the bulk kernel: kBulkTile-byte tiles, one CTA each
+      // retile for the bulk kernel, one CTA per tile
+      uint64_t total = 0;
+      for (int k = 0; k < m; ++k) total += P.nbytes[k];
+      P.bulk_tile = total >= kBulkLargeLaunch ? kBulkTileLarge : kBulkTileSmall;
       uint32_t bt = 0;
       for (int k = 0; k < m; ++k) {
         P.tile_prefix[k] = bt;
-        bt += (uint32_t)((P.nbytes[k] + kBulkTile - 1) / kBulkTile);
+        bt += (uint32_t)((P.nbytes[k] + P.bulk_tile - 1) / P.bulk_tile);
       }
       P.tile_prefix[m] = bt;
-      copy_bulk_tile_kernel<<<bt, 32, bulk_smem, stream>>>(P);
+      copy_bulk_tile_kernel<<<bt, 32, (size_t)P.bulk_tile + 16, stream>>>(P);
     } else {
       const uint32_t grid = std::min<uint32_t>(tiles, (uint32_t)(sm_count() * bps));
       copy_kernel<<<grid, kCopyThreads, 0, stream>>>(P);
