@@ -1193,13 +1193,20 @@ def run_headline(args):
                                 "sample": f"first {args.oracle_buckets} of 17 buckets ({elems} fp32 per rank, "
                                           f"{N_SIM} ranks), {dt:.1f} s single-threaded"}
     if not args.no_rows:
-        del w, plan, host_plan, host_out, h_in, h_out
+        it = max(3, args.steps // 2)
+        # the same step with the double binary tree's fold order (config 2, the other algorithm)
+        tree_plan = cc.BucketAllreducePlan(w["dev_in"], w["dev_out"], cap_bytes=CAP, algo="tree")
+        tree_row = timed_row(torch, lambda: tree_plan.run(cuda_stream), it, bytes_step, launches_per_step, local=local,
+                             kernel="bucket_allreduce_kernel<tree> (compiled 8-rank double binary tree)")
+        config2 = {"workload": workload_desc(args.layers) + "; double-binary-tree fold order",
+                   "l2": "inputs larger than L2; no flush", "rows": {"bucket_allreduce_tree": tree_row}}
+        del w, plan, tree_plan, host_plan, host_out, h_in, h_out
         torch.cuda.empty_cache()
         gen = torch.Generator(device="cuda")
         gen.manual_seed(SEED)
         cpu = not args.no_cpu_baseline
-        it = max(3, args.steps // 2)
-        line["rows"] = {"config1": rows_config1(torch, cc, local, cpu),
+        line["rows"] = {"config2": config2,
+                        "config1": rows_config1(torch, cc, local, cpu),
                         "config3": rows_config3(torch, cc, gen, local, it, cpu),
                         "config4": rows_config4(torch, cc, gen, local, it, cpu),
                         "config5": rows_config5(torch, cc, gen, local, cpu)}

@@ -242,6 +242,81 @@ __device__ __forceinline__ void binomial_fold_ct(int root, Load ld, Widen widen,
   }
 }
 
+// Double-binary-tree programs compiled for a fixed rank count: tree A in the in-order
+// labelling (position p = rank p, node q = p + 1: a node of height h > 0 has the left child
+// q - 2^(h-1) and as right child the first of q + 2^(j-1), j = h..1, that exists), with the
+// fold-machine code of every position and the same leaf merge as tree_program() below; tree B
+// is the mirror (position p = rank N-1-p). Computed at compile time, so that a fully unrolled
+// fold resolves every code and keeps the pending partials in registers.
+template <int NT> struct TreePlan {
+  uint8_t code[NT];
+  int depth;
+  constexpr TreePlan() : code(), depth(0) {
+    int left[NT + 2] = {}, right[NT + 2] = {}, parent[NT + 2] = {};
+    bool is_right[NT + 2] = {};
+    for (int q = 1; q <= NT; ++q) {
+      int h = 0;
+      while (!((q >> h) & 1)) ++h;
+      if (h == 0) continue;
+      const int lq = q - (1 << (h - 1));
+      left[q] = lq;
+      parent[lq] = q;
+      for (int j = h; j >= 1; --j) {
+        const int rq = q + (1 << (j - 1));
+        if (rq <= NT) {
+          right[q] = rq;
+          parent[rq] = q;
+          is_right[rq] = true;
+          break;
+        }
+      }
+    }
+    for (int p = 0; p < NT; ++p) {
+      const int q = p + 1;
+      uint8_t c = left[q] ? kFoldCur : 0;
+      if (right[q]) {
+        c |= kPush;
+      } else {
+        int npop = 0, u = q;
+        while (parent[u] && is_right[u]) { ++npop; u = parent[u]; }
+        c |= (uint8_t)(npop << 2);
+      }
+      code[p] = c;
+    }
+    for (int p = 0; p + 1 < NT; ++p) {
+      const int q = p + 1;
+      if (right[q] == q + 1 && (code[p] & kPush) && npop_of(code[p + 1]) > 0) {
+        code[p] &= (uint8_t)~kPush;
+        const int np = npop_of(code[p + 1]) - 1;
+        code[p + 1] = (uint8_t)((code[p + 1] & ~(7 << 2)) | kFoldCur | (np << 2));
+      }
+    }
+    int d = 0;
+    for (int p = 0; p < NT; ++p) {
+      if (code[p] & kPush)
+        if (++d > depth) depth = d;
+      d -= npop_of(code[p]);
+    }
+  }
+};
+
+// One unit (or element) folded over the NT ranks in the compiled tree order, every load
+// issued before the first fold; `mirror` selects tree B.
+template <int IN, int OP, int NT, typename V, typename X, typename Load, typename Widen>
+__device__ __forceinline__ V tree_fold_ct(bool mirror, Load ld, Widen widen) {
+  constexpr TreePlan<NT> plan{};
+  constexpr int S = plan.depth > 0 ? plan.depth : 1;
+  FoldStack<V, S> st;
+  st.depth = 0;
+  X x[NT];
+#pragma unroll
+  for (int p = 0; p < NT; ++p) x[p] = ld(mirror ? NT - 1 - p : p);
+  V cur;
+#pragma unroll
+  for (int p = 0; p < NT; ++p) fold_step<IN, OP>(plan.code[p], widen(x[p]), cur, st);
+  return cur;
+}
+
 // KIND: kLinear (ring order or a linear tree), kMachine (tree / binomial programs),
 // kHier (two-level), kShallow / kMid (the fold machine with 2 / 4 stack slots, for programs
 // that never hold more pending partials), kLinSmall (the linear fold of 2 ranks, four units
@@ -253,6 +328,10 @@ __host__ __device__ constexpr bool is_binom_ct(int kind) { return kind >= kBinom
 __host__ __device__ constexpr int binom_ct_ranks(int kind) { return 4 << (kind - kBinom4); }
 // units folded at once: about 16 loads in flight per thread for the small rank counts
 __host__ __device__ constexpr int binom_ct_units(int kind) { return kind == kBinom4 ? 4 : kind == kBinom8 ? 2 : 1; }
+// double-binary-tree programs compiled for 8 and 16 ranks (the bucket allreduce)
+constexpr int kTree8 = 20, kTree16 = 21;
+__host__ __device__ constexpr bool is_tree_ct(int kind) { return kind == kTree8 || kind == kTree16; }
+__host__ __device__ constexpr int tree_ct_ranks(int kind) { return kind == kTree8 ? 8 : 16; }
 
 template <int IN, int OP, int KIND, typename RankOf, typename Src, typename EmitU, typename EmitE>
 __device__ __forceinline__ void reduce_range(int n, int g, RankOf rank_of, const FoldProgram& prog,
@@ -274,6 +353,7 @@ __device__ __forceinline__ void reduce_range(int n, int g, RankOf rank_of, const
       binomial_fold_ct<IN, OP, binom_ct_ranks(KIND), 1, A, A>(start, [&](int, int r) { return ld(r); }, same, cur);
       return cur[0];
     }
+    else if constexpr (is_tree_ct(KIND)) return tree_fold_ct<IN, OP, tree_ct_ranks(KIND), A, A>(start == 1, ld, same);
     else {
       FoldStack<A, SLOTS> st;
       return machine_fold<IN, OP, A, A, 8>(n, prog, rank_of, ld, same, st);
@@ -313,6 +393,7 @@ __device__ __forceinline__ void reduce_range(int n, int g, RankOf rank_of, const
       Unit<IN> m;
       if constexpr (RING) m = ring_fold<IN, OP, Unit<IN>, uint4>(n, start, ld, widen, up);
       else if constexpr (KIND == kHier) m = hier_fold<IN, OP, Unit<IN>, uint4>(n, hG, hc, hj, ld, widen);
+      else if constexpr (is_tree_ct(KIND)) m = tree_fold_ct<IN, OP, tree_ct_ranks(KIND), Unit<IN>, uint4>(start == 1, ld, widen);
       else {
         SmemStack<IN> st{stk, (int)T};
         m = machine_fold<IN, OP, Unit<IN>, uint4, 8>(n, prog, rank_of, ld, widen, st);
@@ -528,16 +609,19 @@ using BucketParamsSmall = BucketParamsT<8, 64>;
 static_assert(sizeof(BucketParams) <= 32000, "kernel parameter block too large");
 static_assert(sizeof(BucketParamsSmall) <= 4096, "small parameter block must stay under 4 KB");
 
-template <bool RING, typename PT>
-__global__ void __launch_bounds__(kThreads, RING ? CC_BUCKET_MIN_BLOCKS : CC_BUCKET_TREE_MIN_BLOCKS)
+// KIND: kLinear (ring), kTree8 / kTree16 (the compiled double binary tree of 8 / 16 ranks),
+// kMachine (the tree of any other rank count, on the fold machine).
+template <int KIND, typename PT>
+__global__ void __launch_bounds__(kThreads, KIND == kMachine ? CC_BUCKET_TREE_MIN_BLOCKS : CC_BUCKET_MIN_BLOCKS)
     bucket_allreduce_kernel(const __grid_constant__ PT P) {
   constexpr int IN = CC_F32, OP = CC_SUM;
+  constexpr bool RING = KIND == kLinear;
   // the tile's per-rank pointers, staged once per tile: the fold reads them for every
   // 16-byte unit, and the parameter table is too large to stay in the constant cache
   __shared__ const float* s_in[kMaxRanks];
   __shared__ float* s_out[kMaxRanks];
   __shared__ int s_tensor;
-  __shared__ uint4 s_stk[RING ? 1 : kStackSlots * kThreads];  // the tree's pending partials
+  __shared__ uint4 s_stk[KIND == kMachine ? kStackSlots * kThreads : 1];  // the machine's pending partials
   const int n = P.nranks, nt = P.ntensors;
   const uint32_t ntiles = P.tile_prefix[nt];
   for (uint32_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
@@ -587,9 +671,8 @@ __global__ void __launch_bounds__(kThreads, RING ? CC_BUCKET_MIN_BLOCKS : CC_BUC
         const int rk = P.prog.rmap[p];
         return mirror ? n - 1 - rk : rk;
       };
-      reduce_range<IN, OP, RING ? kLinear : kMachine>(n, g, rank_of, P.prog, s, se, threadIdx.x, blockDim.x,
-                                                         P.vec != 0, src, emit_unit, emit_elem, s_stk + threadIdx.x,
-                                                         g, true);
+      reduce_range<IN, OP, KIND>(n, g, rank_of, P.prog, s, se, threadIdx.x, blockDim.x, P.vec != 0, src, emit_unit,
+                                 emit_elem, s_stk + threadIdx.x, g, true);
       s = se;
     }
     __syncthreads();  // every thread is done with s_in / s_out before the next tile restages them
@@ -912,11 +995,18 @@ static cudaError_t launch_bucket_with(PT& P, const void* const* grads, void* con
   if (fold == kFoldTree) tree_program(nranks, P.prog);
   if (tiles == 0) return cudaSuccess;
   const bool ring = fold == kFoldRing;
-  auto k = ring ? bucket_allreduce_kernel<true, PT> : bucket_allreduce_kernel<false, PT>;
-  static const int bps_ring = blocks_per_sm(bucket_allreduce_kernel<true, PT>);
-  static const int bps_tree = blocks_per_sm(bucket_allreduce_kernel<false, PT>);
-  const uint32_t grid =
-      std::min<uint32_t>(tiles, (uint32_t)(CC_BUCKET_OVERSUB * sm_count() * (ring ? bps_ring : bps_tree)));
+  // the ring; the tree compiled for 8 or 16 ranks; the fold machine for any other tree
+  const int kind = ring ? kLinear : nranks == 8 ? kTree8 : nranks == 16 ? kTree16 : kMachine;
+  auto k = kind == kLinear ? bucket_allreduce_kernel<kLinear, PT>
+           : kind == kTree8 ? bucket_allreduce_kernel<kTree8, PT>
+           : kind == kTree16 ? bucket_allreduce_kernel<kTree16, PT>
+                             : bucket_allreduce_kernel<kMachine, PT>;
+  static const int bps[4] = {blocks_per_sm(bucket_allreduce_kernel<kLinear, PT>),
+                             blocks_per_sm(bucket_allreduce_kernel<kTree8, PT>),
+                             blocks_per_sm(bucket_allreduce_kernel<kTree16, PT>),
+                             blocks_per_sm(bucket_allreduce_kernel<kMachine, PT>)};
+  const int b = bps[kind == kLinear ? 0 : kind == kTree8 ? 1 : kind == kTree16 ? 2 : 3];
+  const uint32_t grid = std::min<uint32_t>(tiles, (uint32_t)(CC_BUCKET_OVERSUB * sm_count() * b));
   k<<<grid, kThreads, 0, stream>>>(P);
   return cudaGetLastError();
 }

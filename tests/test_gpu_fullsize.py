@@ -40,7 +40,8 @@ def _gather(dev, pos):
     return dev[torch.from_numpy(pos).cuda()].cpu().numpy()
 
 
-def test_config2_ddp_full_size_sampled():
+@pytest.mark.parametrize("algo", ["ring", "tree"])
+def test_config2_ddp_full_size_sampled(algo):
     n, cap = 8, 25 * 1024 * 1024
     shapes = synth.transformer_grad_shapes()
     numels = [synth.numel(s) for _, s in shapes]
@@ -51,7 +52,7 @@ def test_config2_ddp_full_size_sampled():
     dev_out = [torch.empty_like(d) for d in dev_in]
     views = lambda flat: [flat[offs[i]:offs[i + 1]].view(shapes[i][1]) for i in range(len(numels))]
     plan = cc.BucketAllreducePlan([views(d) for d in dev_in], [views(d) for d in dev_out], cap_bytes=cap,
-                                  scale=1.0 / n)
+                                  scale=1.0 / n, algo=algo)
     plan.run()
     torch.cuda.synchronize()
     for r in range(1, n):
@@ -61,12 +62,14 @@ def test_config2_ddp_full_size_sampled():
     assert len(buckets) == 17
     for members in buckets:
         bcount = sum(numels[i] for i in members)
-        bpos = _positions(bcount, L.chunk_bounds(bcount, n), rng, extra=300)
+        bounds = L.chunk_bounds(bcount, n) if algo == "ring" else [(0, (bcount + 1) // 2), ((bcount + 1) // 2, bcount)]
+        bpos = _positions(bcount, bounds, rng, extra=300)
         # bucket position -> flat offset of the per-rank buffer
         starts = np.cumsum([0] + [numels[i] for i in members])
         k = np.searchsorted(starts, bpos, side="right") - 1
         flat = offs[np.array(members)[k]] + (bpos - starts[k])
-        want, _ = C.ring_allreduce([h[flat] for h in host], scale=1.0 / n, count=bcount, positions=bpos)
+        fn = C.ring_allreduce if algo == "ring" else C.tree_allreduce
+        want, _ = fn([h[flat] for h in host], scale=1.0 / n, count=bcount, positions=bpos)
         got = _gather(dev_out[3], flat)
         assert np.array_equal(bits(got), bits(want[3])), f"bucket {members[:3]}..."
 
