@@ -590,6 +590,23 @@ def alpha_beta_crossover(n, alpha_ring, alpha_tree, bw_ring, bw_tree):
     return lat / per_byte
 
 
+def crossover_reading(n, alpha_ring, alpha_tree, bw_ring, bw_tree):
+    """The model's answer in words: the crossover size, or which schedule is faster at every
+    size (and why) when there is none."""
+    import math
+    m = alpha_beta_crossover(n, alpha_ring, alpha_tree, bw_ring, bw_tree)
+    if m is not None:
+        return f"ring faster above {m / 1e6:.3g} MB per rank, tree below"
+    steps_tree = 2 * math.ceil(math.log2(n)) if n > 1 else 0
+    ring_lat = 2 * (n - 1) * alpha_ring > steps_tree * alpha_tree
+    ring_byte = 2.0 * (n - 1) / n / bw_ring > 2.0 / bw_tree
+    if ring_lat and ring_byte:
+        return "no crossover: the tree is faster at every size (smaller latency and per-byte terms)"
+    if not ring_lat and not ring_byte:
+        return "no crossover: the ring is at least as fast at every size (latency and per-byte terms no larger)"
+    return "no crossover"
+
+
 def fit_alpha_beta(n, small_bytes, t_small, large_bytes, t_large, algo):
     """alpha from the smallest message (its time over the schedule's step count) and the
     bandwidth B from the largest (M over the model's bandwidth term), per algorithm."""
@@ -659,7 +676,9 @@ def rows_config5(torch, cc, gen, local, with_cpu=True):
              "alpha_from": "the stepped schedules' 1 KiB time (CUDA-graph device time) over their step counts; "
                            "B from their 256 MiB time",
              "crossover_fitted_alpha_bytes": alpha_beta_crossover(n, ar, at, br, bt),
-             "crossover_launch_alpha_bytes": alpha_beta_crossover(n, lat, lat, br, bt)}
+             "crossover_fitted_alpha": crossover_reading(n, ar, at, br, bt),
+             "crossover_launch_alpha_bytes": alpha_beta_crossover(n, lat, lat, br, bt),
+             "crossover_launch_alpha": crossover_reading(n, lat, lat, br, bt)}
     out = {"workload": "config 5 large points: fused ring / tree allreduce, N=8 x 256 MiB and N=64 x 64 MiB fp32 "
                        "U[-1,1] (device-seeded); stepped ring / tree at N=8 x 1 KiB and 256 MiB",
            "l2": "256 MiB flush before each timed call whose working set fits in L2; the large points exceed it",

@@ -137,3 +137,25 @@ def test_multi_gpu_bucket_layout_agrees_across_ranks_and_tiles_the_buffer():
             assert offs[members[0]] == start and sum(numels[i] for i in members) == count
         for (start, _), p in zip(ranges, ptrs):
             assert p == [b + 4 * start for b in bases]
+
+
+def test_alpha_beta_model_against_closed_forms():
+    """The lecture's alpha-beta model (lecture 09 §7.3: ring 2(N-1) alpha + 2(N-1)/N M / B, tree
+    2 log2(N) alpha + 2 M / B): with one alpha and one B the ring's extra latency
+    2(N-1-log2 N) alpha is paid back by its smaller per-byte term at
+    M* = 2(N-1-log2 N) alpha / (2/B - 2(N-1)/(N B)) = (N-1-log2 N) N alpha B."""
+    sys.path.insert(0, ROOT)
+    import bench
+    a, B = 2e-6, 100e9
+    for n in (4, 8, 16, 64):
+        import math
+        want = (n - 1 - math.log2(n)) * n * a * B
+        got = bench.alpha_beta_crossover(n, a, a, B, B)
+        assert abs(got - want) <= 1e-9 * want, (n, got, want)
+        assert bench.crossover_reading(n, a, a, B, B).startswith("ring faster above")
+    # the fitted stepped numbers of one GPU: the tree wins both terms, so no crossover
+    assert bench.alpha_beta_crossover(8, 1.78e-6, 2.71e-6, 200e9, 254e9) is None
+    assert "tree is faster at every size" in bench.crossover_reading(8, 1.78e-6, 2.71e-6, 200e9, 254e9)
+    # N = 2: the same steps, so the ring's smaller per-byte term never loses
+    assert bench.alpha_beta_crossover(2, a, a, B, B) is None
+    assert "ring is at least as fast" in bench.crossover_reading(2, a, a, B, B)
