@@ -392,9 +392,8 @@ __device__ __forceinline__ void load_token_head(const A2ACopyParams& P, int s, i
 
 // One token of source s, by one warp: dispatch writes its row to each selected expert's
 // position; combine reads the rows back from those positions into slots [t][k]. `base` is
-// [N][E] in global or shared memory; the tile prefixes and ranks are read through L2 (another
-// SM may have written them in the same launch). With `head` the dispatch row's first vectors
-// are already in x.
+// [N][E]; the table entries are read once each, through L2. With `head` the dispatch row's
+// first vectors are already in x.
 __device__ __forceinline__ void copy_token(const A2ACopyParams& P, const int* base, int s, int t, int lane,
                                            uint4 (&x)[kCopyVecs], bool head) {
   constexpr int B = kCopyVecs;
