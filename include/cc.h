@@ -239,8 +239,9 @@ CC_API cc_status cc_alltoallv_run(const void* const* send, void* const* recv, in
                                   size_t recv_capacity_rows, int direction, void* workspace,
                                   size_t workspace_bytes, void* stream);
 
-/* Copies the per-destination received row counts of the last cc_alltoallv that used
- * `workspace` into recv_rows[0..nranks) (host or device memory), stream-ordered. */
+/* Copies the per-destination received row counts of the last cc_alltoallv or
+ * cc_alltoallv_plan that used `workspace` into recv_rows[0..nranks) (host or device memory),
+ * stream-ordered. */
 CC_API cc_status cc_alltoallv_recv_counts(const void* workspace, int nranks, int32_t* recv_rows,
                                    void* stream);
 
