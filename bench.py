@@ -64,10 +64,11 @@ def aggregate_gbps(world, bytes_per_step, ms_per_step):
     return world * bytes_per_step / (ms_per_step * 1e-3) / 1e9
 
 
-def workload_desc(layers):
+def workload_desc(layers, algo="ring"):
+    fold = "ring" if algo == "ring" else "double-binary-tree"
     return (f"ddp_bucket_allreduce: N={N_SIM} simulated ranks on one GPU, fp32 gradients of a "
             f"{layers}-layer d=768 ffn=3072 vocab=32000 transformer, 25 MiB buckets in reverse "
-            f"registration order, ring allreduce with scale 1/{N_SIM}, fused flatten/unflatten")
+            f"registration order, {fold} allreduce with scale 1/{N_SIM}, fused flatten/unflatten")
 
 
 def measured_peak():
@@ -79,6 +80,9 @@ def measured_peak():
         return float(p["hbm_gbs"]), "measured copy rate (MEASURED_PEAKS.json hbm_gbs; not a ceiling)"
     except Exception:
         return 6650.0, "fallback copy rate (6650 GB/s, earlier measurement; not a ceiling)"
+
+
+DDP_PROFILES = {"ring": "bucket_allreduce_ddp.txt", "tree": "bucket_allreduce_ddp_tree.txt"}
 
 
 def profile_traffic(name="bucket_allreduce_ddp.txt"):
@@ -1115,6 +1119,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--layers", type=int, default=12, help="model depth (12 = the workload; smaller for profiling)")
+    ap.add_argument("--algo", default="ring", choices=["ring", "tree"],
+                    help="ddp: the fold order of the headline step (ring, the default, or the double binary tree)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rows", action="store_true", help="headline only (configs 1, 3, 4, 5 left out)")
@@ -1151,7 +1157,8 @@ def run_headline(args):
     w = build_workload(torch, args.layers, SEED, pinned_inputs=True)
     bytes_step = 2 * N_SIM * w["total"] * 4
     stream = torch.cuda.current_stream()
-    plan = cc.BucketAllreducePlan(w["dev_in"], w["dev_out"], cap_bytes=CAP)  # scale: the library's mean
+    # scale: the library's mean; algo: the ring (the headline) unless --algo tree
+    plan = cc.BucketAllreducePlan(w["dev_in"], w["dev_out"], cap_bytes=CAP, algo=args.algo)
     cuda_stream = stream.cuda_stream
 
     def step():
@@ -1178,7 +1185,7 @@ def run_headline(args):
     host_out = [torch.empty(w["total"], dtype=torch.float32, pin_memory=True) for _ in range(N_SIM)]
     h_in = [w["views"](h) for h in w["host"]]
     h_out = [w["views"](h) for h in host_out]
-    host_plan = cc.BucketAllreduceHostPlan(h_in, h_out, w["dev_in"], w["dev_out"], cap_bytes=CAP)
+    host_plan = cc.BucketAllreduceHostPlan(h_in, h_out, w["dev_in"], w["dev_out"], cap_bytes=CAP, algo=args.algo)
     host_plan.run(cuda_stream)
     torch.cuda.synchronize()
     s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -1197,12 +1204,12 @@ def run_headline(args):
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "pct_of_8TBps": 100.0 * value / NOMINAL_HBM_GBS,
         "elems_per_s": N_SIM * w["total"] / (ms_step * 1e-3),
-        "config": {"workload": workload_desc(args.layers), "sim_ranks": N_SIM, "tensors": len(w["numels"]),
+        "config": {"workload": workload_desc(args.layers, args.algo), "sim_ranks": N_SIM, "tensors": len(w["numels"]),
                    "elems_per_rank": w["total"], "bytes_per_step": bytes_step, "buckets": 17 if args.layers == 12 else None,
                    "l2": "inputs (3.5 GB) larger than L2 (126 MB); no flush", "parallelism": "replicas x1"},
         "roofline": dict(roofline_fields(achieved, peak, peak_kind), bound="hbm",
-                         traffic=profile_traffic() if args.layers == 12 else None,
-                         kernel="bucket_allreduce_kernel<ring>"),
+                         traffic=profile_traffic(DDP_PROFILES[args.algo]) if args.layers == 12 else None,
+                         kernel=f"bucket_allreduce_kernel<{args.algo}>"),
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": N_SIM * w["total"] * 4,
                 "d2h_bytes_per_step": N_SIM * w["total"] * 4},
         "gpu_launches": launches_per_step * args.steps,
@@ -1219,7 +1226,7 @@ def run_headline(args):
         tree_plan = cc.BucketAllreducePlan(w["dev_in"], w["dev_out"], cap_bytes=CAP, algo="tree")
         tree_row = timed_row(torch, lambda: tree_plan.run(cuda_stream), it, bytes_step, launches_per_step, local=local,
                              kernel="bucket_allreduce_kernel<tree> (compiled 8-rank double binary tree)")
-        config2 = {"workload": workload_desc(args.layers) + "; double-binary-tree fold order",
+        config2 = {"workload": workload_desc(args.layers, "tree"),
                    "l2": "inputs larger than L2; no flush", "rows": {"bucket_allreduce_tree": tree_row}}
         del w, plan, tree_plan, host_plan, host_out, h_in, h_out
         torch.cuda.empty_cache()
