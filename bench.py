@@ -87,14 +87,18 @@ DDP_PROFILES = {"ring": "bucket_allreduce_ddp.txt", "tree": "bucket_allreduce_dd
 
 def profile_traffic(name="bucket_allreduce_ddp.txt"):
     """DRAM bytes per launch of a line's dominant kernel from a committed ncu summary in
-    profiles/, or None when the kernel's source file changed since the counters were taken
-    (the summary records the file and its SHA-256)."""
+    profiles/, or None when a source file of the kernel changed since the counters were taken
+    (the summary records the files, comma-separated, and their SHA-256s in the same order)."""
     try:
         text = open(os.path.join(ROOT, "profiles", name)).read()
         lines = dict(l.split(":", 1) for l in text.splitlines() if ":" in l and not l.startswith(" "))
-        src = os.path.join(ROOT, lines.get("kernel_source", os.path.relpath(KERNEL_SRC, ROOT)).strip())
-        if lines.get("kernel_source_sha256", "").strip() != hashlib.sha256(open(src, "rb").read()).hexdigest():
+        srcs = [x.strip() for x in lines.get("kernel_source", os.path.relpath(KERNEL_SRC, ROOT)).split(",")]
+        shas = [x.strip() for x in lines.get("kernel_source_sha256", "").split(",")]
+        if len(srcs) != len(shas):
             return None
+        for src, sha in zip(srcs, shas):
+            if sha != hashlib.sha256(open(os.path.join(ROOT, src), "rb").read()).hexdigest():
+                return None
         return int(float(lines["dram_bytes_per_launch_full_workload"].strip()))
     except Exception:
         return None

@@ -86,6 +86,17 @@ def test_profile_traffic_goes_null_when_the_kernel_source_changes(tmp_path):
     src.write_text("kernel v2\n")
     assert b.profile_traffic("p.txt") is None
     assert b.profile_traffic("missing.txt") is None
+    # a kernel spread over two files: both must be unchanged
+    hdr = tmp_path / "k.cuh"
+    hdr.write_text("folds v1\n")
+    sha1 = hashlib.sha256(b"kernel v2\n").hexdigest()
+    sha2 = hashlib.sha256(b"folds v1\n").hexdigest()
+    (tmp_path / "profiles" / "q.txt").write_text(
+        f"kernel_source: k.cu, k.cuh\nkernel_source_sha256: {sha1}, {sha2}\n"
+        "dram_bytes_per_launch_full_workload: 99\n")
+    assert b.profile_traffic("q.txt") == 99
+    hdr.write_text("folds v2\n")
+    assert b.profile_traffic("q.txt") is None
 
 
 def _layout_worker(rank, world, port, q):

@@ -191,7 +191,8 @@ def test_broadcast(n, root, count):
 
 # N = 2, 3: the binomial program is a left fold from the root (linear kernel); SUM at N = 4,
 # 8, 16, 32, 64: the program compiled to straight-line code; other N and ops: the fold machines
-@pytest.mark.parametrize("n,root", [(1, 0), (2, 1), (3, 2), (4, 0), (4, 3), (8, 5), (13, 12), (16, 9), (32, 31),
+@pytest.mark.parametrize("n,root", [(1, 0), (2, 1), (3, 2), (4, 0), (4, 3), (5, 3), (6, 0), (7, 6), (8, 5), (9, 4),
+                                    (10, 9), (11, 1), (12, 7), (13, 12), (14, 2), (15, 8), (16, 9), (17, 3), (32, 31),
                                     (64, 17), (64, 0)])
 @pytest.mark.parametrize("kind", ["spread", "i32", "bf16"])
 @pytest.mark.parametrize("count", [2049, 4 * 8192 + 7])
