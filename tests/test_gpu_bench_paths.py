@@ -56,3 +56,29 @@ def test_two_ranks_on_one_gpu_over_gloo_match_the_single_gpu_call():
     line = json.loads(lines[0])
     assert line["parity_rank0_vs_single_gpu"] == "bit-exact"
     assert line["comm_nranks"] == 2 and line["n_gpus"] == 2 and line["backend"] == "gloo"
+
+
+@pytest.mark.timeout(600)
+@pytest.mark.parametrize("algo", ["ring", "tree"])
+def test_default_line_carries_every_contract_key(algo):
+    """The one-GPU headline line (1-layer model, no rows): the keys the bench contract names,
+    with a roofline against the copy rate, the end-to-end number through host buffers, the
+    clock record and the count of the library's launches."""
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--layers", "1", "--steps", "3", "--warmup", "3",
+           "--e2e-steps", "1", "--no-rows", "--no-cpu-baseline", "--algo", algo]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=540, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-3000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+              "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
+        assert k in line, k
+    assert line["n_gpus"] == 1 and line["steps"] == 3 and line["value"] > 0 and line["higher_is_better"] is True
+    assert line["gpu_launches"] == 3 and line["config"]["workload"]
+    roof = line["roofline"]
+    assert roof["bound"] == "hbm" and roof["unit"] == "GB/s" and roof["peak"] > 0
+    assert abs(roof["frac"] - roof["achieved"] / roof["peak"]) < 1e-9 and algo in roof["kernel"]
+    e2e = line["e2e"]
+    assert e2e["value"] > 0 and e2e["h2d_bytes_per_step"] == e2e["d2h_bytes_per_step"] > 0
+    assert line["clocks"]["samples"] >= 1 and "reasons" in line["clocks"]
