@@ -65,12 +65,14 @@ struct RouteParams {
   int tokens, experts, topk;
 };
 
-// Eight lanes per token. Lane g of a token's group scans the 4-expert chunks g, g+8, ... in
+// Four lanes per token. Lane g of a token's group scans the 4-expert chunks g, g+4, ... in
 // expert order with a running, descending top-k list in registers (a later expert enters
-// only with a strictly larger value, so equal values keep the lower id first); the eight
-// lists are then merged pairwise with shuffles (three butterfly steps), ordering by larger
-// value, then lower id. All lanes end with the token's top-k; lane 0 writes it.
-constexpr int kRouteLanes = 8;
+// only with a strictly larger value, so equal values keep the lower id first); the four
+// lists are then merged pairwise with shuffles (two butterfly steps), ordering by larger
+// value, then lower id. All lanes end with the token's top-k; lane 0 writes it. (Measured on
+// 8 x 8192 tokens x 64 experts: 8 lanes 11.3-12.1 us, 4 lanes 9.7 us, 2 lanes 10.2 us.)
+constexpr int kRouteLanes = 4;
+constexpr int kRoutePre = 4;  // chunks per lane loaded before the first insert
 
 __device__ __forceinline__ bool route_better(float a, int ia, float b, int ib) {
   return ib < 0 || (ia >= 0 && (a > b || (a == b && ia < ib)));
@@ -105,12 +107,24 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const __grid_constant__
     const float* row = P.logits[s] + (size_t)t * P.experts;
     const bool vec = (P.experts % 4 == 0) && ((reinterpret_cast<uintptr_t>(P.logits[s]) & 15) == 0);
     if (vec) {
-      for (int e = 4 * g; e < P.experts; e += 4 * kRouteLanes) {
-        const float4 v = __ldcs(reinterpret_cast<const float4*>(row + e));
-        insert(v.x, e);
-        insert(v.y, e + 1);
-        insert(v.z, e + 2);
-        insert(v.w, e + 3);
+      // kRoutePre chunks per lane loaded before the first insert (one DRAM round trip for up to
+      // 4 * 8 * kRoutePre experts), then inserted in the same expert order as one at a time
+      for (int e0 = 4 * g; e0 < P.experts; e0 += 4 * kRouteLanes * kRoutePre) {
+        float4 v[kRoutePre];
+#pragma unroll
+        for (int q = 0; q < kRoutePre; ++q) {
+          const int e = e0 + 4 * kRouteLanes * q;
+          if (e < P.experts) v[q] = __ldcs(reinterpret_cast<const float4*>(row + e));
+        }
+#pragma unroll
+        for (int q = 0; q < kRoutePre; ++q) {
+          const int e = e0 + 4 * kRouteLanes * q;
+          if (e >= P.experts) break;
+          insert(v[q].x, e);
+          insert(v[q].y, e + 1);
+          insert(v[q].z, e + 2);
+          insert(v[q].w, e + 3);
+        }
       }
     } else {
       for (int e = g; e < P.experts; e += kRouteLanes) insert(__ldcs(row + e), e);
