@@ -821,9 +821,13 @@ def run_multi_gpu(args):
             if stt != cc.CC_OK:
                 raise RuntimeError(f"cc_allreduce_slice: status {stt}")
 
-    def step():
-        stream.synchronize()
-        dist.barrier()
+    def step(before=False):
+        # every rank's slices of a step are done on every GPU once the barrier after it has
+        # passed, so back-to-back steps need no barrier before (the inputs did not change);
+        # a step whose inputs were just rewritten (the end-to-end copy in) takes one
+        if before:
+            stream.synchronize()
+            dist.barrier()
         launch_slices()
         stream.synchronize()
         dist.barrier()
@@ -870,7 +874,7 @@ def run_multi_gpu(args):
 
     def e2e_step():
         send.copy_(host, non_blocking=True)
-        step()
+        step(before=True)
         host_out.copy_(recv, non_blocking=True)
 
     ems = timed(e2e_step, args.e2e_steps)
