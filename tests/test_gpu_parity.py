@@ -173,7 +173,8 @@ def test_allgather_misaligned_shards_and_bf16_width():
 
 # ---- broadcast, reduce, scatter, gather ------------------------------------------------------------------
 
-@pytest.mark.parametrize("n,root,count", [(1, 0, 10), (4, 0, 4099), (7, 3, 100_000), (64, 63, 333)])
+@pytest.mark.parametrize("n,root,count", [(1, 0, 10), (4, 0, 4099), (7, 3, 100_000), (64, 63, 333),
+                                          (64, 5, 64 * 1024 + 3), (16, 0, 3 * 512 + 1)])
 def test_broadcast(n, root, count):
     x = synth.uniform_f32(5, 0, count)
     want, _ = C.broadcast(x, n, root)
@@ -206,7 +207,8 @@ def test_reduce_to_root(n, root, kind, count):
     out.check()
 
 
-@pytest.mark.parametrize("n,count", [(4, 4), (4, 4099), (9, 100_001), (64, 70)])
+@pytest.mark.parametrize("n,count", [(4, 4), (4, 4099), (9, 100_001), (64, 70), (16, 16 * 2048 + 15),
+                                     (3, 3 * 4096 * 7)])
 def test_scatter_and_gather(n, count):
     x = synth.int32_uniform(6, 0, count, -5, 5)
     parts, _ = C.scatter(x, n, root=n - 1)
@@ -220,6 +222,27 @@ def test_scatter_and_gather(n, count):
         out[r].check()
     _assert_same(to_host(back.t), x)
     back.check()
+
+
+@pytest.mark.parametrize("n,shard", [(64, 4096), (64, 4096 + 13), (16, 512 * 7 + 1), (32, 511)])
+@pytest.mark.parametrize("kind", ["f32", "bf16"])
+def test_wide_allgather_spans_many_bulk_tiles(n, shard, kind):
+    """Fan-out to many ranks with shards of several 2 KiB bulk tiles and a ragged last tile
+    (every tile stored to all N outputs), bit for bit against the oracle's ring allgather."""
+    count = n * shard
+    shards = []
+    for c in range(n):
+        _, ln = cc.cc_chunk(count, n, c)
+        x = synth.uniform_f32(8, c, ln)
+        shards.append(synth.to_bf16_bits(x) if kind == "bf16" else x)
+    want, _ = C.ring_allgather(shards)
+    dt = torch.bfloat16 if kind == "bf16" else torch.float32
+    out = [Guarded(count, dt) for _ in range(n)]
+    cc.cc_allgather([to_dev(x) for x in shards], [g.t for g in out])
+    torch.cuda.synchronize()
+    for r in (0, n // 2, n - 1):
+        _assert_same(to_host(out[r].t), want[r], f"allgather N={n} rank {r}")
+        out[r].check()
 
 
 # ---- failure detection on the device: a bounded wait that runs out reports, never hangs ----------
