@@ -17,8 +17,11 @@
 // slower with them than with 32 KiB tiles; 1 KiB tiles halved a one-destination copy.
 // The wait is bounded: one that gives up records CC_ERR_TIMEOUT in the device status word.
 //
-// copy_kernel (any alignment): 128-bit streaming loads/stores per thread where an entry is
-// 16-byte aligned, element by element otherwise.
+// copy_kernel (any alignment, and every copy that touches peer memory): 128-bit streaming
+// loads/stores, four in flight per thread, where source and destinations share their offset
+// from a 16-byte boundary; element copies, eight in flight per thread, for the rest
+// (measured on an allgather N = 8 × 256 MiB whose shards sit one element off: 1.25 TB/s one
+// element at a time, 4.79 TB/s with eight in flight).
 #include <algorithm>
 #include <mutex>
 
@@ -39,7 +42,8 @@ struct CopyParams {
   int skip;
   uint32_t esize;
   uint32_t tile_prefix[kCopyMaxEntries + 1];
-  uint64_t vec_mask[kCopyMaxEntries / 64];
+  uint64_t vec_mask[kCopyMaxEntries / 64];   // every address of the entry 16-byte aligned
+  uint64_t coal_mask[kCopyMaxEntries / 64];  // source and destinations equal modulo 16 bytes
   const char* src[kCopyMaxEntries];
   char* dst[kCopyMaxEntries];
   uint64_t nbytes[kCopyMaxEntries];
@@ -52,6 +56,38 @@ __device__ __forceinline__ void copy_elem(char* d, const char* s, uint32_t esize
   else __stcs(reinterpret_cast<unsigned short*>(d), __ldcs(reinterpret_cast<const unsigned short*>(s)));
 }
 
+// Element-wise part of a tile, kCopyElems elements per thread in flight before their stores;
+// the 128-bit part keeps kCopyVecs loads per thread in flight.
+constexpr int kCopyElems = 8;
+constexpr int kCopyVecs = 4;
+
+template <typename E>
+__device__ __forceinline__ void copy_elems(const CopyParams& P, int k, const char* src, uint64_t lo, uint64_t hi) {
+  constexpr uint64_t ES = sizeof(E);
+  for (uint64_t o0 = lo + threadIdx.x * ES; o0 < hi; o0 += (uint64_t)kCopyThreads * ES * kCopyElems) {
+    E v[kCopyElems];
+#pragma unroll
+    for (int q = 0; q < kCopyElems; ++q) {
+      const uint64_t o = o0 + (uint64_t)q * kCopyThreads * ES;
+      if (o < hi) v[q] = __ldcs(reinterpret_cast<const E*>(src + o));
+    }
+#pragma unroll
+    for (int q = 0; q < kCopyElems; ++q) {
+      const uint64_t o = o0 + (uint64_t)q * kCopyThreads * ES;
+      if (o >= hi) continue;
+      if (P.fanout) {
+        for (int r = 0; r < P.ndst; ++r)
+          if (r != P.skip) __stcs(reinterpret_cast<E*>(P.dst_base[r] + P.dst_off[k] + o), v[q]);
+      } else {
+        __stcs(reinterpret_cast<E*>(P.dst[k] + o), v[q]);
+      }
+    }
+  }
+}
+
+// One tile of an entry: 128-bit loads and stores over the part where the source and every
+// destination sit on 16-byte boundaries (the whole tile when all are aligned; after a head of
+// under 16 bytes when they are equally misaligned), element copies for the rest.
 __global__ void __launch_bounds__(kCopyThreads) copy_kernel(const __grid_constant__ CopyParams P) {
   const uint32_t ntiles = P.tile_prefix[P.nentries];
   for (uint32_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
@@ -65,23 +101,38 @@ __global__ void __launch_bounds__(kCopyThreads) copy_kernel(const __grid_constan
     const uint64_t a = (uint64_t)(tile - P.tile_prefix[k]) * kCopyTile;
     const uint64_t b = min(a + kCopyTile, P.nbytes[k]);
     const bool vec = (P.vec_mask[k >> 6] >> (k & 63)) & 1;
-    const uint64_t vb = vec ? a + (b - a) / 16 * 16 : a;
-    for (uint64_t o = a + threadIdx.x * 16ull; o < vb; o += kCopyThreads * 16ull) {
-      const uint4 v = __ldcs(reinterpret_cast<const uint4*>(src + o));
-      if (P.fanout) {
-        for (int r = 0; r < P.ndst; ++r)
-          if (r != P.skip) __stcs(reinterpret_cast<uint4*>(P.dst_base[r] + P.dst_off[k] + o), v);
-      } else {
-        __stcs(reinterpret_cast<uint4*>(P.dst[k] + o), v);
+    const bool coal = (P.coal_mask[k >> 6] >> (k & 63)) & 1;
+    uint64_t va = a, vb = a;
+    if (vec || coal) {
+      const uint64_t head = (16 - ((reinterpret_cast<uintptr_t>(src) + a) & 15)) & 15;
+      va = min(b, a + head);
+      vb = va + (b - va) / 16 * 16;
+    }
+    for (uint64_t o0 = va + threadIdx.x * 16ull; o0 < vb; o0 += kCopyThreads * 16ull * kCopyVecs) {
+      uint4 v[kCopyVecs];
+#pragma unroll
+      for (int q = 0; q < kCopyVecs; ++q) {
+        const uint64_t o = o0 + (uint64_t)q * kCopyThreads * 16;
+        if (o < vb) v[q] = __ldcs(reinterpret_cast<const uint4*>(src + o));
+      }
+#pragma unroll
+      for (int q = 0; q < kCopyVecs; ++q) {
+        const uint64_t o = o0 + (uint64_t)q * kCopyThreads * 16;
+        if (o >= vb) continue;
+        if (P.fanout) {
+          for (int r = 0; r < P.ndst; ++r)
+            if (r != P.skip) __stcs(reinterpret_cast<uint4*>(P.dst_base[r] + P.dst_off[k] + o), v[q]);
+        } else {
+          __stcs(reinterpret_cast<uint4*>(P.dst[k] + o), v[q]);
+        }
       }
     }
-    for (uint64_t o = vb + threadIdx.x * (uint64_t)P.esize; o < b; o += (uint64_t)kCopyThreads * P.esize) {
-      if (P.fanout) {
-        for (int r = 0; r < P.ndst; ++r)
-          if (r != P.skip) copy_elem(P.dst_base[r] + P.dst_off[k] + o, src + o, P.esize);
-      } else {
-        copy_elem(P.dst[k] + o, src + o, P.esize);
-      }
+    if (P.esize == 4) {
+      copy_elems<unsigned>(P, k, src, a, va);
+      copy_elems<unsigned>(P, k, src, vb, b);
+    } else {
+      copy_elems<unsigned short>(P, k, src, a, va);
+      copy_elems<unsigned short>(P, k, src, vb, b);
     }
   }
 }
@@ -166,13 +217,18 @@ __global__ void __launch_bounds__(32) copy_bulk_tile_kernel(const __grid_constan
   }
   const int k = lo;
   const uint64_t a = (uint64_t)(tile - P.tile_prefix[k]) * tile_bytes;
-  const uint32_t bytes = (uint32_t)min((uint64_t)tile_bytes, P.nbytes[k] - a);
-  const uint32_t bulk = bytes & ~15u;
+  const uint64_t nb = P.nbytes[k];
+  // An entry whose source sits h0 bytes before a 16-byte boundary (its destinations the same):
+  // tile t moves [a + h0, a + h0 + tile) in bulk, clipped to the entry; the entry's first h0
+  // bytes (tile 0) and a last partial 16 bytes go element by element. h0 = 0 when aligned.
+  const uint64_t h0 = (16 - (reinterpret_cast<uintptr_t>(P.src[k]) & 15)) & 15;
+  const uint64_t lo = min(nb, a + h0), hi = min(nb, a + tile_bytes + h0);
+  const uint32_t bulk = (uint32_t)((hi - lo) & ~15ull);
   if (bulk) {
     mbar_init(bar);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     mbar_arrive_tx(bar, bulk);
-    bulk_load(smem, P.src[k] + a, bulk, bar);
+    bulk_load(smem, P.src[k] + lo, bulk, bar);
     if (!mbar_wait(bar, 0)) {
       // one more bounded chance for the load to land before leaving. If it still has not,
       // the CTA leaves with the bulk load in flight: that load may still write this CTA's
@@ -186,9 +242,11 @@ __global__ void __launch_bounds__(32) copy_bulk_tile_kernel(const __grid_constan
   }
   for (int r = 0; r < (P.fanout ? P.ndst : 1); ++r) {
     if (P.fanout && r == P.skip) continue;
-    char* d = P.fanout ? P.dst_base[r] + P.dst_off[k] + a : P.dst[k] + a;
-    if (bulk) bulk_store(d, smem, bulk);
-    for (uint32_t o = bulk; o < bytes; o += P.esize) copy_elem(d + o, P.src[k] + a + o, P.esize);
+    char* d = P.fanout ? P.dst_base[r] + P.dst_off[k] : P.dst[k];
+    if (bulk) bulk_store(d + lo, smem, bulk);
+    if (a == 0)
+      for (uint64_t o = 0; o < min(h0, nb); o += P.esize) copy_elem(d + o, P.src[k] + o, P.esize);
+    for (uint64_t o = lo + bulk; o < hi; o += P.esize) copy_elem(d + o, P.src[k] + o, P.esize);
   }
   bulk_commit();
   bulk_wait_all();
@@ -259,6 +317,16 @@ cudaError_t launch_copy(const CopyEntry* entries, int nentries, void* const* dst
       P.dst_off[m] = e.dst_off * elem_bytes;
       const bool v = al16(P.src[m]) && (fanout ? bases_aligned && (P.dst_off[m] % 16 == 0) : al16(P.dst[m]));
       if (v) P.vec_mask[m >> 6] |= 1ull << (m & 63);
+      // equally misaligned source and destinations: 128-bit copies after a short head
+      bool c = true;
+      const uintptr_t sa = reinterpret_cast<uintptr_t>(P.src[m]) & 15;
+      if (fanout) {
+        for (int r = 0; r < ndst; ++r)
+          if (r != skip) c = c && ((reinterpret_cast<uintptr_t>(P.dst_base[r]) + P.dst_off[m]) & 15) == sa;
+      } else {
+        c = (reinterpret_cast<uintptr_t>(P.dst[m]) & 15) == sa;
+      }
+      if (c) P.coal_mask[m >> 6] |= 1ull << (m & 63);
       P.tile_prefix[m] = tiles;
       tiles += (uint32_t)((nb + kCopyTile - 1) / kCopyTile);
       ++m;
@@ -266,9 +334,10 @@ cudaError_t launch_copy(const CopyEntry* entries, int nentries, void* const* dst
     P.nentries = m;
     P.tile_prefix[m] = tiles;
     if (tiles == 0) continue;
-    bool all_vec = true;
-    for (int k = 0; k < m; ++k) all_vec = all_vec && ((P.vec_mask[k >> 6] >> (k & 63)) & 1);
-    if (all_vec && !plain && bulk_attr == cudaSuccess) {
+    // the bulk kernel when every entry's source and destinations are equally aligned
+    bool all_coal = true;
+    for (int k = 0; k < m; ++k) all_coal = all_coal && ((P.coal_mask[k >> 6] >> (k & 63)) & 1);
+    if (all_coal && !plain && bulk_attr == cudaSuccess) {
       // retile for the bulk kernel, one CTA per tile
       uint64_t total = 0;
       for (int k = 0; k < m; ++k) total += P.nbytes[k];

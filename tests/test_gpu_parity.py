@@ -245,6 +245,41 @@ def test_wide_allgather_spans_many_bulk_tiles(n, shard, kind):
         out[r].check()
 
 
+def _off(a: np.ndarray, elems: int):
+    """A CUDA tensor holding `a`, `elems` elements past a 16-byte boundary."""
+    full = to_dev(np.concatenate([np.zeros(elems, a.dtype), a]))
+    return full[elems:]
+
+
+@pytest.mark.parametrize("kind", ["f32", "bf16"])
+@pytest.mark.parametrize("shift_src,shift_dst", [(1, 1), (3, 3), (1, 2), (2, 0)])
+def test_misaligned_copies_equal_or_unequal_offsets(kind, shift_src, shift_dst):
+    """Allgather, scatter and gather with sources and destinations off 16-byte boundaries:
+    equally misaligned (128-bit copies after a short head) or not (element copies), large enough
+    for several 64 KiB tiles, bit for bit against the oracle."""
+    n, count = 4, 4 * 70_001
+    dt = torch.bfloat16 if kind == "bf16" else torch.float32
+    def data(seed, r, ln):
+        x = synth.uniform_f32(seed, r, ln)
+        return synth.to_bf16_bits(x) if kind == "bf16" else x
+    shards = [data(21, c, cc.cc_chunk(count, n, c)[1]) for c in range(n)]
+    want, _ = C.ring_allgather(shards)
+    zeros = np.zeros(count, np.uint16 if kind == "bf16" else np.float32)
+    outs = [_off(zeros, shift_dst) for _ in range(n)]
+    cc.cc_allgather([_off(x, shift_src) for x in shards], outs)
+    x = data(22, 0, count)
+    parts, _ = C.scatter(x, n, root=1)
+    sc = [_off(np.zeros(p.size, zeros.dtype), shift_dst) for p in parts]
+    cc.cc_scatter(_off(x, shift_src), sc, 1)
+    back = _off(np.zeros(count, zeros.dtype), shift_src)
+    cc.cc_gather(sc, back, 1)
+    torch.cuda.synchronize()
+    for r in range(n):
+        _assert_same(to_host(outs[r]), want[r], f"allgather rank {r}")
+        _assert_same(to_host(sc[r]), parts[r], f"scatter rank {r}")
+    _assert_same(to_host(back), x, "gather")
+
+
 # ---- failure detection on the device: a bounded wait that runs out reports, never hangs ----------
 
 def test_bounded_wait_timeout_is_reported_and_the_context_survives():
