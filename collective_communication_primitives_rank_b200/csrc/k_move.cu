@@ -222,13 +222,13 @@ __global__ void __launch_bounds__(32) copy_bulk_tile_kernel(const __grid_constan
   // tile t moves [a + h0, a + h0 + tile) in bulk, clipped to the entry; the entry's first h0
   // bytes (tile 0) and a last partial 16 bytes go element by element. h0 = 0 when aligned.
   const uint64_t h0 = (16 - (reinterpret_cast<uintptr_t>(P.src[k]) & 15)) & 15;
-  const uint64_t lo = min(nb, a + h0), hi = min(nb, a + tile_bytes + h0);
-  const uint32_t bulk = (uint32_t)((hi - lo) & ~15ull);
+  const uint64_t blo = min(nb, a + h0), bhi = min(nb, a + tile_bytes + h0);
+  const uint32_t bulk = (uint32_t)((bhi - blo) & ~15ull);
   if (bulk) {
     mbar_init(bar);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     mbar_arrive_tx(bar, bulk);
-    bulk_load(smem, P.src[k] + lo, bulk, bar);
+    bulk_load(smem, P.src[k] + blo, bulk, bar);
     if (!mbar_wait(bar, 0)) {
       // one more bounded chance for the load to land before leaving. If it still has not,
       // the CTA leaves with the bulk load in flight: that load may still write this CTA's
@@ -243,10 +243,10 @@ __global__ void __launch_bounds__(32) copy_bulk_tile_kernel(const __grid_constan
   for (int r = 0; r < (P.fanout ? P.ndst : 1); ++r) {
     if (P.fanout && r == P.skip) continue;
     char* d = P.fanout ? P.dst_base[r] + P.dst_off[k] : P.dst[k];
-    if (bulk) bulk_store(d + lo, smem, bulk);
+    if (bulk) bulk_store(d + blo, smem, bulk);
     if (a == 0)
       for (uint64_t o = 0; o < min(h0, nb); o += P.esize) copy_elem(d + o, P.src[k] + o, P.esize);
-    for (uint64_t o = lo + bulk; o < hi; o += P.esize) copy_elem(d + o, P.src[k] + o, P.esize);
+    for (uint64_t o = blo + bulk; o < bhi; o += P.esize) copy_elem(d + o, P.src[k] + o, P.esize);
   }
   bulk_commit();
   bulk_wait_all();

@@ -338,17 +338,23 @@ cudaError_t launch_reduce(const void* const* send, void* const* dst, int ndst, i
   P.fold = fold;
   P.scale = scale;
   P.do_scale = (in_t != CC_I32) && scale != 1.0f;
-  bool vec = true;
+  // 16-byte units when every source sits at the same offset from a 16-byte boundary, a whole
+  // number of elements, and so does every allreduce / root output (for equal element sizes;
+  // a bf16 -> fp32 fold needs aligned buffers); reduce-scatter shards are checked one by one in
+  // the kernel. The units then start `shift` elements past each boundary.
+  const size_t es_in = in_t == CC_BF16 ? 2 : 4;
+  const uintptr_t m0 = reinterpret_cast<uintptr_t>(send[0]) & 15;
+  bool vec = m0 % es_in == 0 && (m0 == 0 || es_in == 4);
   for (int r = 0; r < nranks; ++r) {
     P.src[r] = send[r];
-    vec = vec && aligned16(send[r]);
+    vec = vec && (reinterpret_cast<uintptr_t>(send[r]) & 15) == m0;
   }
   for (int r = 0; r < ndst; ++r) {
     P.dst[r] = dst[r];
-    if (aligned16(dst[r])) P.dst_aligned |= (1ull << r);
-    else if (mode != kReduceScatter) vec = false;
+    if (mode != kReduceScatter) vec = vec && (reinterpret_cast<uintptr_t>(dst[r]) & 15) == m0;
   }
   P.vec = vec;
+  P.shift = vec ? m0 / es_in : 0;
   P.per_node = 1;
   if (fold == kFoldTree) tree_program(nranks, P.prog);
   else if (fold == kFoldBinomial) binomial_program(nranks, root, P.prog);

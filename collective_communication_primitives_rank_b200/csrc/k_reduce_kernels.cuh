@@ -335,7 +335,8 @@ template <int IN, int OP, int KIND, typename RankOf, typename Src, typename Emit
 __device__ __forceinline__ void reduce_range(int n, int g, RankOf rank_of, const FoldProgram& prog,
                                              uint64_t a, uint64_t b, uint64_t t, uint64_t T, bool vec,
                                              Src src, EmitU emit_unit, EmitE emit_elem, uint4* stk,
-                                             int start = 0, bool up = true, int hG = 1, int hc = 0, int hj = 0) {
+                                             int start = 0, bool up = true, int hG = 1, int hc = 0, int hj = 0,
+                                             uint64_t shift = 0) {
   constexpr bool RING = KIND == kLinear || KIND == kLinSmall;
   constexpr int SLOTS = KIND == kShallow ? 2 : KIND == kMid ? 4 : kStackSlots;
   using A = typename Tr<IN>::Acc;
@@ -358,9 +359,12 @@ __device__ __forceinline__ void reduce_range(int n, int g, RankOf rank_of, const
     }
   };
   if (vec) {
-    uint64_t va = (a + UE - 1) / UE * UE;
+    // 16-byte units start where (e + shift) is a multiple of UE: every buffer sits `shift`
+    // elements past a 16-byte boundary (0 when aligned)
+    uint64_t va = a + (UE - (a + shift) % UE) % UE;
     if (va > b) va = b;
-    uint64_t vb = b / UE * UE;
+    const uint64_t vbs = (b + shift) / UE * UE;  // the last unit boundary, in shifted coordinates
+    uint64_t vb = vbs >= shift ? vbs - shift : 0;
     if (vb < va) vb = va;
     const uint64_t step = T * UE;
     auto widen = [](const uint4& x) { return to_unit<IN>(x); };
@@ -478,7 +482,7 @@ struct ReduceParams {
   uint64_t count;
   uint64_t lo, hi;       // the elements this launch folds: [lo, hi) of the count
   uint64_t tile;         // elements per tile (a multiple of 8)
-  uint64_t dst_aligned;  // bit r: dst[r] is 16-byte aligned
+  uint64_t shift;        // elements every source (and allreduce / root output) sits past a 16-byte boundary
   int nranks;
   int per_node;  // ranks per node (hierarchical fold)
   int mode;
@@ -522,8 +526,11 @@ __global__ void __launch_bounds__(kThreads, KIND == kLinear ? CC_RING_MIN_BLOCKS
         const int rk = P.prog.rmap[p];
         return mirror ? n - 1 - rk : rk;
       };
-      const bool shard_vec = mode == kReduceScatter && ((P.dst_aligned >> (g & 63)) & 1) &&
-                             ((ga * sizeof(Out)) % 16 == 0);
+      // a shard takes whole-unit stores when its element under the group's first unit is aligned
+      constexpr uint64_t UEk = Tr<IN>::UE;
+      const uint64_t first_unit = ga + (UEk - (ga + P.shift) % UEk) % UEk;
+      const bool shard_vec = mode == kReduceScatter &&
+                             ((reinterpret_cast<uintptr_t>(static_cast<Out*>(P.dst[g]) + (first_unit - ga)) & 15) == 0);
       auto emit_unit = [&](uint64_t e, Unit<IN> u) {
         if (P.do_scale) scale_unit<IN>(u, P.scale);
         if (mode == kAllReduce) {
@@ -554,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, KIND == kLinear ? CC_RING_MIN_BLOCKS
                          : P.fold == kFoldTree ? (g == 0 ? 0 : n - 1) : P.prog.rmap[0];
       const bool lup = P.fold == kFoldMultiRing ? ((g / n) % 2 == 0) : (P.fold != kFoldTree || g == 0);
       reduce_range<IN, OP, KIND>(n, g, rank_of, P.prog, s, se, threadIdx.x, blockDim.x, P.vec != 0, src,
-                                    emit_unit, emit_elem, s_stk + threadIdx.x, lstart, lup, G, hc, hj);
+                                    emit_unit, emit_elem, s_stk + threadIdx.x, lstart, lup, G, hc, hj, P.shift);
       s = se;
     }
   }

@@ -128,6 +128,42 @@ def test_allreduce_in_place_and_misaligned():
         _assert_same(to_host(mout[r]), want[r], "misaligned")
 
 
+def _shifted(a: np.ndarray, elems: int):
+    """A CUDA tensor holding `a`, `elems` elements past a 16-byte boundary."""
+    return to_dev(np.concatenate([np.zeros(elems, a.dtype), a]))[elems:]
+
+
+@pytest.mark.parametrize("algo", ["ring", "tree"])
+@pytest.mark.parametrize("kind", ["spread", "i32", "bf16"])
+@pytest.mark.parametrize("ss,sd", [(1, 1), (3, 3), (2, 2), (1, 0), (0, 3), (2, 1)])
+def test_allreduce_reduce_scatter_and_reduce_with_shifted_buffers(algo, kind, ss, sd):
+    """Sources `ss` and outputs `sd` elements past a 16-byte boundary: equal shifts take the
+    16-byte units after an element-wise head (fp32 and int32; bf16 inputs with fp32 outputs
+    keep the element path), unequal shifts the element path; every result bit for bit against
+    the oracle, over several tiles and a ragged tail."""
+    n, count = 8, 8 * 12_289 + 5
+    xs = _inputs(kind, n, count, seed=31)
+    scale = 1.0 if kind == "i32" else 0.125
+    fn = C.ring_allreduce if algo == "ring" else C.tree_allreduce
+    want, _ = fn(xs, in_dtype=_IN[kind], scale=scale)
+    od = np.int32 if kind == "i32" else np.float32
+    srcs = [_shifted(x, ss) for x in xs]
+    outs = [_shifted(np.zeros(count, od), sd) for _ in range(n)]
+    cc.cc_allreduce(srcs, outs, algo=algo, scale=scale)
+    rs_want, _ = C.ring_reduce_scatter(xs, in_dtype=_IN[kind], scale=scale)
+    shards = [_shifted(np.zeros(cc.cc_chunk(count, n, c)[1], od), sd) for c in range(n)]
+    cc.cc_reduce_scatter(srcs, shards, scale=scale)
+    red_want, _ = C.reduce(xs, 5, in_dtype=_IN[kind])
+    root = _shifted(np.zeros(count, od), sd)
+    cc.cc_reduce(srcs, root, 5)
+    torch.cuda.synchronize()
+    for r in (0, 3, n - 1):
+        _assert_same(to_host(outs[r]), want[r], f"allreduce {algo} {kind} ({ss},{sd}) rank {r}")
+    for c in range(n):
+        _assert_same(to_host(shards[c]), rs_want[c], f"reduce-scatter {kind} ({ss},{sd}) shard {c}")
+    _assert_same(to_host(root), red_want, f"reduce {kind} ({ss},{sd})")
+
+
 def test_allreduce_empty_is_a_no_op():
     t = [torch.empty(0, device="cuda") for _ in range(4)]
     cc.cc_allreduce(t, t)
