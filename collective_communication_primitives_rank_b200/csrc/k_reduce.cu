@@ -377,8 +377,11 @@ cudaError_t launch_reduce(const void* const* send, void* const* dst, int ndst, i
   // N = 2 × 256 MiB: ring 5667 -> 6663 GB/s, reduce-scatter 5399 -> 6832; at N = 3..4 the
   // one-unit fold with 4 resident CTAs is faster)
   if (kind == kLinear && nranks == 2) kind = kLinSmall;
-  // binomial sums at 4, 8, 16, 32, 64 ranks, and at every other rank count from 5 to 15 (their
-  // own translation unit), run their program compiled to straight-line code
+  // tree sums at 8 and 16 ranks run the tree compiled to straight-line code (as the bucket
+  // kernel does); binomial sums at 4, 8, 16, 32, 64 ranks, and at every other rank count from
+  // 5 to 15, their program compiled likewise (k_reduce_binom.cu holds the ones not here)
+  if (fold == kFoldTree && op == CC_SUM && kind != kLinear && (nranks == 8 || nranks == 16))
+    return run_reduce_tree_ct(P, in_t, nranks == 8 ? kTree8 : kTree16, stream);
   if (fold == kFoldBinomial && op == CC_SUM && kind != kLinear && nranks >= 4) {
     if ((nranks & (nranks - 1)) == 0) kind = kBinom4 + __builtin_ctz((unsigned)nranks) - 2;
     else if (nranks >= kBinomNLo && nranks <= kBinomNHi) return run_reduce_binom_np2(P, in_t, kBinomN0 + nranks, stream);

@@ -1,6 +1,7 @@
 // Binomial reduce-to-root programs (lecture 09 §3.4) compiled to straight-line code for the
 // rank counts from 5 to 15 that are not powers of two (SUM only; the powers of two are in
-// k_reduce.cu). Each is the same pre-order walk and fold-machine codes as the run-time program
+// k_reduce.cu), and the double-binary-tree allreduce programs (lecture 09 §5.2) of 8 and 16
+// ranks (SUM; TreePlan, the same program as tree_program in k_reduce.cu). Each is the same pre-order walk and fold-machine codes as the run-time program
 // of any rank count (binomial_program in k_reduce.cu), built at compile time by BinomialPlan,
 // so the result is bit for bit the fold machine's. A translation unit of its own: the build
 // compiles it beside k_reduce.cu.
@@ -30,6 +31,21 @@ cudaError_t run_reduce_binom_np2(ReduceParams& P, cc_dtype in_t, int kind, cudaS
     case CC_F32: return run_binom_np2<CC_F32>(P, kind, s);
     case CC_BF16: return run_binom_np2<CC_BF16>(P, kind, s);
     case CC_I32: return run_binom_np2<CC_I32>(P, kind, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <int IN>
+static cudaError_t run_tree_ct(ReduceParams& P, int kind, cudaStream_t s) {
+  return kind == kTree8 ? run_reduce<IN, CC_SUM, kTree8>(P, s) : run_reduce<IN, CC_SUM, kTree16>(P, s);
+}
+
+cudaError_t run_reduce_tree_ct(ReduceParams& P, cc_dtype in_t, int kind, cudaStream_t s) {
+  if (kind != kTree8 && kind != kTree16) return cudaErrorInvalidValue;
+  switch (in_t) {
+    case CC_F32: return run_tree_ct<CC_F32>(P, kind, s);
+    case CC_BF16: return run_tree_ct<CC_BF16>(P, kind, s);
+    case CC_I32: return run_tree_ct<CC_I32>(P, kind, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -352,7 +352,7 @@ __device__ __forceinline__ void reduce_range(int n, int g, RankOf rank_of, const
       binomial_fold_ct<IN, OP, binom_ct_ranks(KIND), 1, A, A>(start, [&](int, int r) { return ld(r); }, same, cur);
       return cur[0];
     }
-    else if constexpr (is_tree_ct(KIND)) return tree_fold_ct<IN, OP, tree_ct_ranks(KIND), A, A>(start == 1, ld, same);
+    else if constexpr (is_tree_ct(KIND)) return tree_fold_ct<IN, OP, tree_ct_ranks(KIND), A, A>(start != 0, ld, same);
     else {
       FoldStack<A, SLOTS> st;
       return machine_fold<IN, OP, A, A, 8>(n, prog, rank_of, ld, same, st);
@@ -395,7 +395,7 @@ __device__ __forceinline__ void reduce_range(int n, int g, RankOf rank_of, const
       Unit<IN> m;
       if constexpr (RING) m = ring_fold<IN, OP, Unit<IN>, uint4>(n, start, ld, widen, up);
       else if constexpr (KIND == kHier) m = hier_fold<IN, OP, Unit<IN>, uint4>(n, hG, hc, hj, ld, widen);
-      else if constexpr (is_tree_ct(KIND)) m = tree_fold_ct<IN, OP, tree_ct_ranks(KIND), Unit<IN>, uint4>(start == 1, ld, widen);
+      else if constexpr (is_tree_ct(KIND)) m = tree_fold_ct<IN, OP, tree_ct_ranks(KIND), Unit<IN>, uint4>(start != 0, ld, widen);
       else {
         SmemStack<IN> st{stk, (int)T};
         m = machine_fold<IN, OP, Unit<IN>, uint4, 8>(n, prog, rank_of, ld, widen, st);
@@ -610,5 +610,8 @@ static cudaError_t run_reduce(ReduceParams& P, cudaStream_t s) {
 // The binomial SUM programs compiled for 5..7 and 9..15 ranks (k_reduce_binom.cu); `kind` is
 // kBinomN0 + N.
 cudaError_t run_reduce_binom_np2(ReduceParams& P, cc_dtype in_t, int kind, cudaStream_t s);
+// The double-binary-tree SUM programs compiled for 8 and 16 ranks (k_reduce_binom.cu); `kind`
+// is kTree8 or kTree16.
+cudaError_t run_reduce_tree_ct(ReduceParams& P, cc_dtype in_t, int kind, cudaStream_t s);
 
 }  // namespace cc
