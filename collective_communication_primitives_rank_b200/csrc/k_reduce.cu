@@ -289,6 +289,20 @@ int sm_count() {
   return cached[dev];
 }
 
+// Sums over sources at one offset into outputs at another: element stores on the sources' units.
+template <int IN>
+static cudaError_t dispatch_scalar_out(ReduceParams& P, int kind, cudaStream_t s) {
+  switch (kind) {
+    case kLinear: return run_reduce<IN, CC_SUM, kLinear, true>(P, s);
+    case kLinSmall: return run_reduce<IN, CC_SUM, kLinSmall, true>(P, s);
+    case kHier: return run_reduce<IN, CC_SUM, kHier, true>(P, s);
+    case kShallow: return run_reduce<IN, CC_SUM, kShallow, true>(P, s);
+    case kMid: return run_reduce<IN, CC_SUM, kMid, true>(P, s);
+    case kMachine: return run_reduce<IN, CC_SUM, kMachine, true>(P, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
 template <int IN>
 static cudaError_t dispatch_op(ReduceParams& P, cc_op op, int kind, cudaStream_t s) {
 #define CC_KINDS(OPV)                                                                         \
@@ -339,20 +353,25 @@ cudaError_t launch_reduce(const void* const* send, void* const* dst, int ndst, i
   P.scale = scale;
   P.do_scale = (in_t != CC_I32) && scale != 1.0f;
   // 16-byte units when every source sits at the same offset from a 16-byte boundary, a whole
-  // number of elements, and so does every allreduce / root output (for equal element sizes;
-  // a bf16 -> fp32 fold needs aligned buffers); reduce-scatter shards are checked one by one in
-  // the kernel. The units then start `shift` elements past each boundary.
+  // number of elements (bf16 sources: aligned). The units then start `shift` elements past each
+  // boundary. Allreduce / root outputs at that same offset (for equal element sizes; fp32
+  // outputs of bf16 sources: aligned) take 16-byte stores; reduce-scatter shards are checked one
+  // by one in the kernel. fp32 / int32 sums into outputs at another offset keep the units and
+  // store element by element; other folds over such buffers take the element path.
   const size_t es_in = in_t == CC_BF16 ? 2 : 4;
   const uintptr_t m0 = reinterpret_cast<uintptr_t>(send[0]) & 15;
-  bool vec = m0 % es_in == 0 && (m0 == 0 || es_in == 4);
+  bool src_vec = m0 % es_in == 0 && (m0 == 0 || es_in == 4);
+  bool dst_vec = true;
   for (int r = 0; r < nranks; ++r) {
     P.src[r] = send[r];
-    vec = vec && (reinterpret_cast<uintptr_t>(send[r]) & 15) == m0;
+    src_vec = src_vec && (reinterpret_cast<uintptr_t>(send[r]) & 15) == m0;
   }
   for (int r = 0; r < ndst; ++r) {
     P.dst[r] = dst[r];
-    if (mode != kReduceScatter) vec = vec && (reinterpret_cast<uintptr_t>(dst[r]) & 15) == m0;
+    if (mode != kReduceScatter) dst_vec = dst_vec && (reinterpret_cast<uintptr_t>(dst[r]) & 15) == m0;
   }
+  const bool scalar_out = src_vec && !dst_vec && op == CC_SUM && es_in == 4;
+  const bool vec = src_vec && (dst_vec || scalar_out);
   P.vec = vec;
   P.shift = vec ? m0 / es_in : 0;
   P.per_node = 1;
@@ -377,6 +396,17 @@ cudaError_t launch_reduce(const void* const* send, void* const* dst, int ndst, i
   // N = 2 × 256 MiB: ring 5667 -> 6663 GB/s, reduce-scatter 5399 -> 6832; at N = 3..4 the
   // one-unit fold with 4 resident CTAs is faster)
   if (kind == kLinear && nranks == 2) kind = kLinSmall;
+  // element stores: the runtime folds and the trees compiled for 8 and 16 ranks (binomial
+  // programs run on the fold machine)
+  if (scalar_out) {
+    if (fold == kFoldTree && kind != kLinear && (nranks == 8 || nranks == 16))
+      return run_reduce_tree_ct(P, in_t, nranks == 8 ? kTree8 : kTree16, stream, true);
+    switch (in_t) {
+      case CC_F32: return dispatch_scalar_out<CC_F32>(P, kind, stream);
+      case CC_I32: return dispatch_scalar_out<CC_I32>(P, kind, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   // tree sums at 8 and 16 ranks run the tree compiled to straight-line code (as the bucket
   // kernel does); binomial sums at 4, 8, 16, 32, 64 ranks, and at every other rank count from
   // 5 to 15, their program compiled likewise (k_reduce_binom.cu holds the ones not here)

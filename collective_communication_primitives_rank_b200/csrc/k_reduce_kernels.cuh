@@ -487,7 +487,8 @@ struct ReduceParams {
   int per_node;  // ranks per node (hierarchical fold)
   int mode;
   int fold;
-  int vec;  // every source (and every allreduce / root destination) is 16-byte aligned
+  int vec;  // every source sits `shift` elements past a 16-byte boundary (and so does every
+            // allreduce / root output, unless the kernel stores element by element)
   float scale;
   int do_scale;
 };
@@ -495,7 +496,10 @@ struct ReduceParams {
 // Each CTA folds contiguous tiles (normally exactly one: the grid is sized to the tile
 // count); a tile is split where it crosses a fold group (ring chunk or tree half) and each
 // piece is folded by the whole CTA.
-template <int IN, int OP, int KIND>
+// SS: the units follow the sources and the allreduce / root outputs, which sit at another
+// offset from a 16-byte boundary, take four element stores per unit (fp32 / int32), as
+// reduce-scatter shards that the units meet off a boundary always do.
+template <int IN, int OP, int KIND, bool SS = false>
 __global__ void __launch_bounds__(kThreads, KIND == kLinear ? CC_RING_MIN_BLOCKS
                                            : KIND == kLinSmall ? CC_LINSMALL_MIN_BLOCKS
                                            : is_binom_ct(KIND) ? (binom_ct_units(KIND) > 1 ? 2 : KIND == kBinom64 ? 3 : 4)
@@ -534,10 +538,15 @@ __global__ void __launch_bounds__(kThreads, KIND == kLinear ? CC_RING_MIN_BLOCKS
       auto emit_unit = [&](uint64_t e, Unit<IN> u) {
         if (P.do_scale) scale_unit<IN>(u, P.scale);
         if (mode == kAllReduce) {
-          for (int r = 0; r < n; ++r) store_unit<IN>(static_cast<Out*>(P.dst[r]) + e, u);
+          for (int r = 0; r < n; ++r) {
+            if constexpr (SS) store_unit_scalar<IN>(static_cast<Out*>(P.dst[r]) + e, u);
+            else store_unit<IN>(static_cast<Out*>(P.dst[r]) + e, u);
+          }
         } else if (mode == kReduceScatter) {
           Out* d = static_cast<Out*>(P.dst[g]) + (e - ga);
           if (shard_vec) store_unit<IN>(d, u); else store_unit_scalar<IN>(d, u);
+        } else if constexpr (SS) {
+          store_unit_scalar<IN>(static_cast<Out*>(P.dst[0]) + e, u);
         } else {
           store_unit<IN>(static_cast<Out*>(P.dst[0]) + e, u);
         }
@@ -574,9 +583,9 @@ static int blocks_per_sm(K kernel) {
   return b;
 }
 
-template <int IN, int OP, int KIND>
+template <int IN, int OP, int KIND, bool SS = false>
 static cudaError_t run_reduce(ReduceParams& P, cudaStream_t s) {
-  auto k = reduce_kernel<IN, OP, KIND>;
+  auto k = reduce_kernel<IN, OP, KIND, SS>;
   static const int bps = blocks_per_sm(k);
   constexpr uint64_t UE = Tr<IN>::UE;
   const uint64_t resident = (uint64_t)sm_count() * bps;
@@ -611,7 +620,7 @@ static cudaError_t run_reduce(ReduceParams& P, cudaStream_t s) {
 // kBinomN0 + N.
 cudaError_t run_reduce_binom_np2(ReduceParams& P, cc_dtype in_t, int kind, cudaStream_t s);
 // The double-binary-tree SUM programs compiled for 8 and 16 ranks (k_reduce_binom.cu); `kind`
-// is kTree8 or kTree16.
-cudaError_t run_reduce_tree_ct(ReduceParams& P, cc_dtype in_t, int kind, cudaStream_t s);
+// is kTree8 or kTree16; `scalar_out`: outputs stored element by element (fp32 / int32).
+cudaError_t run_reduce_tree_ct(ReduceParams& P, cc_dtype in_t, int kind, cudaStream_t s, bool scalar_out = false);
 
 }  // namespace cc

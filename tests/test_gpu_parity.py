@@ -139,8 +139,9 @@ def _shifted(a: np.ndarray, elems: int):
 def test_allreduce_reduce_scatter_and_reduce_with_shifted_buffers(algo, kind, ss, sd):
     """Sources `ss` and outputs `sd` elements past a 16-byte boundary: equal shifts take the
     16-byte units after an element-wise head (fp32 and int32; bf16 inputs with fp32 outputs
-    keep the element path), unequal shifts the element path; every result bit for bit against
-    the oracle, over several tiles and a ragged tail."""
+    keep the element path), unequal shifts the sources' units with element stores (sums), or
+    the element path; every result bit for bit against the oracle, over several tiles and a
+    ragged tail."""
     n, count = 8, 8 * 12_289 + 5
     xs = _inputs(kind, n, count, seed=31)
     scale = 1.0 if kind == "i32" else 0.125
@@ -162,6 +163,63 @@ def test_allreduce_reduce_scatter_and_reduce_with_shifted_buffers(algo, kind, ss
     for c in range(n):
         _assert_same(to_host(shards[c]), rs_want[c], f"reduce-scatter {kind} ({ss},{sd}) shard {c}")
     _assert_same(to_host(root), red_want, f"reduce {kind} ({ss},{sd})")
+
+
+@pytest.mark.parametrize("n", [2, 5, 8, 16])
+@pytest.mark.parametrize("kind", ["spread", "i32", "bf16"])
+@pytest.mark.parametrize("offs,sd", [("mixed", 0), ("mixed", 2), ("one", 0), ("zero", 3), ("one", 2)])
+def test_sums_with_sources_and_outputs_at_different_offsets(n, kind, offs, sd):
+    """Sources at one offset from a 16-byte boundary and outputs at another take the sources'
+    16-byte units with element stores (sums); sources at different offsets ("mixed": rank r
+    r mod 4 elements past a boundary) take the element path. Ring, double binary tree,
+    multi-ring and hierarchical allreduce, reduce-scatter (each shard at its own offset) and
+    reduce to a root, bit for bit against the oracle over several tiles and a ragged tail, no
+    write outside an output; a MAX over the same buffers (element path) as well."""
+    count = n * 6_007 + 3
+    xs = _inputs(kind, n, count, seed=33)
+    scale = 1.0 if kind == "i32" else 0.125
+    ss = [r % 4 if offs == "mixed" else 1 if offs == "one" else 0 for r in range(n)]
+    srcs = [_shifted(x, s) for x, s in zip(xs, ss)]
+    od = _out_dtype(kind)
+
+    def outs():
+        return [Guarded(count, od, misalign=sd) for _ in range(n)]
+
+    cases = [("ring", lambda o: cc.cc_allreduce(srcs, o, algo="ring", scale=scale),
+              C.ring_allreduce(xs, in_dtype=_IN[kind], scale=scale)[0]),
+             ("tree", lambda o: cc.cc_allreduce(srcs, o, algo="tree", scale=scale),
+              C.tree_allreduce(xs, in_dtype=_IN[kind], scale=scale)[0]),
+             ("multiring", lambda o: cc.cc_allreduce_multiring(srcs, o, 2, scale=scale),
+              C.multiring_allreduce(xs, 2, in_dtype=_IN[kind], scale=scale)[0])]
+    if n % 4 == 0:
+        cases.append(("hierarchical", lambda o: cc.cc_allreduce_hierarchical(srcs, o, 4, scale=scale),
+                      C.hierarchical_allreduce(xs, 4, in_dtype=_IN[kind], scale=scale)[0]))
+    for name, call, want in cases:
+        out = outs()
+        call([g.t for g in out])
+        torch.cuda.synchronize()
+        for r in range(n):
+            _assert_same(to_host(out[r].t), want[r], f"{name} {kind} {offs}/{sd} N={n} rank {r}")
+            out[r].check()
+    rs_want, _ = C.ring_reduce_scatter(xs, in_dtype=_IN[kind], scale=scale)
+    shards = [Guarded(cc.cc_chunk(count, n, c)[1], od, misalign=(sd + c) % 4) for c in range(n)]
+    cc.cc_reduce_scatter(srcs, [g.t for g in shards], scale=scale)
+    root = n // 2
+    red_want, _ = C.reduce(xs, root, in_dtype=_IN[kind])
+    red = Guarded(count, od, misalign=sd)
+    cc.cc_reduce(srcs, red.t, root)
+    mx_want, _ = C.ring_allreduce(xs, op="max", in_dtype=_IN[kind])
+    mx = outs()
+    cc.cc_allreduce(srcs, [g.t for g in mx], op="max")
+    torch.cuda.synchronize()
+    for c in range(n):
+        _assert_same(to_host(shards[c].t), rs_want[c], f"reduce-scatter {kind} {offs}/{sd} N={n} shard {c}")
+        shards[c].check()
+    _assert_same(to_host(red.t), red_want, f"reduce {kind} {offs}/{sd} N={n}")
+    red.check()
+    for r in range(n):
+        _assert_same(to_host(mx[r].t), mx_want[r], f"max {kind} {offs}/{sd} N={n} rank {r}")
+        mx[r].check()
 
 
 def test_allreduce_empty_is_a_no_op():
