@@ -346,11 +346,12 @@ def _off(a: np.ndarray, elems: int):
 
 
 @pytest.mark.parametrize("kind", ["f32", "bf16"])
-@pytest.mark.parametrize("shift_src,shift_dst", [(1, 1), (3, 3), (1, 2), (2, 0)])
+@pytest.mark.parametrize("shift_src,shift_dst", [(1, 1), (3, 3), (1, 2), (2, 0), (0, 1), (0, 3), (3, 1)])
 def test_misaligned_copies_equal_or_unequal_offsets(kind, shift_src, shift_dst):
     """Allgather, scatter and gather with sources and destinations off 16-byte boundaries:
-    equally misaligned (128-bit copies after a short head) or not (element copies), large enough
-    for several 64 KiB tiles, bit for bit against the oracle."""
+    equally misaligned (128-bit copies after a short head) or not (128-bit stores on the
+    destinations' boundaries, each 16 bytes loaded element by element), large enough for several
+    64 KiB tiles, bit for bit against the oracle."""
     n, count = 4, 4 * 70_001
     dt = torch.bfloat16 if kind == "bf16" else torch.float32
     def data(seed, r, ln):
@@ -372,6 +373,45 @@ def test_misaligned_copies_equal_or_unequal_offsets(kind, shift_src, shift_dst):
         _assert_same(to_host(outs[r]), want[r], f"allgather rank {r}")
         _assert_same(to_host(sc[r]), parts[r], f"scatter rank {r}")
     _assert_same(to_host(back), x, "gather")
+
+
+@pytest.mark.parametrize("kind", ["f32", "bf16"])
+def test_copies_with_destinations_at_different_offsets(kind):
+    """Allgather into outputs at different offsets from each other (rank r: r mod 4 elements
+    past a 16-byte boundary: element copies) and from the shards, and broadcast / flatten /
+    unflatten of odd-sized tensors whose places in the flat buffer fall at every offset
+    (destination-aligned 128-bit stores per entry); guard bands around every output."""
+    n, count = 5, 5 * 40_003 + 2
+    dt = torch.bfloat16 if kind == "bf16" else torch.float32
+
+    def data(seed, r, ln):
+        x = synth.uniform_f32(seed, r, ln)
+        return synth.to_bf16_bits(x) if kind == "bf16" else x
+    shards = [data(23, c, cc.cc_chunk(count, n, c)[1]) for c in range(n)]
+    want, _ = C.ring_allgather(shards)
+    outs = [Guarded(count, dt, misalign=r % 4) for r in range(n)]
+    cc.cc_allgather([_off(x, 1) for x in shards], [g.t for g in outs])
+    x = data(24, 0, count)
+    bwant, _ = C.broadcast(x, n, 2)
+    bout = [Guarded(count, dt, misalign=3) for _ in range(n)]
+    cc.cc_broadcast(_off(x, 2), [g.t for g in bout], 2)
+    sizes = [70_001 + 13 * i for i in range(9)]
+    ts = [data(25, i, m) for i, m in enumerate(sizes)]
+    flat = Guarded(sum(sizes), dt, misalign=1)
+    cc.cc_bucket_flatten([_off(t, i % 4) for i, t in enumerate(ts)], flat.t)
+    back = [Guarded(m, dt, misalign=(i + 2) % 4) for i, m in enumerate(sizes)]
+    cc.cc_bucket_unflatten(flat.t, [g.t for g in back])
+    torch.cuda.synchronize()
+    for r in range(n):
+        _assert_same(to_host(outs[r].t), want[r], f"allgather rank {r}")
+        outs[r].check()
+        _assert_same(to_host(bout[r].t), bwant[r], f"broadcast rank {r}")
+        bout[r].check()
+    _assert_same(to_host(flat.t), np.concatenate(ts), "flatten")
+    flat.check()
+    for i in range(len(sizes)):
+        _assert_same(to_host(back[i].t), ts[i], f"unflatten {i}")
+        back[i].check()
 
 
 # ---- failure detection on the device: a bounded wait that runs out reports, never hangs ----------
