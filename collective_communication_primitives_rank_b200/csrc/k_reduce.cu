@@ -374,6 +374,7 @@ cudaError_t launch_reduce(const void* const* send, void* const* dst, int ndst, i
   const bool vec = src_vec && (dst_vec || scalar_out);
   P.vec = vec;
   P.shift = vec ? m0 / es_in : 0;
+  P.lshift = vec ? (reinterpret_cast<uintptr_t>(send[0]) & 127) / es_in : 0;
   P.per_node = 1;
   if (fold == kFoldTree) tree_program(nranks, P.prog);
   else if (fold == kFoldBinomial) binomial_program(nranks, root, P.prog);

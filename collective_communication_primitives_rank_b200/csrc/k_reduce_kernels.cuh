@@ -482,6 +482,8 @@ struct ReduceParams {
   uint64_t count;
   uint64_t lo, hi;       // the elements this launch folds: [lo, hi) of the count
   uint64_t tile;         // elements per tile (a multiple of 8)
+  uint64_t skew;         // tile k >= 1 starts at lo + k * tile - skew (the first tile is that much shorter)
+  uint64_t lshift;       // elements the first source sits past a 128-byte line (16-byte units only)
   uint64_t shift;        // elements every source (and allreduce / root output) sits past a 16-byte boundary
   int nranks;
   int per_node;  // ranks per node (hierarchical fold)
@@ -515,10 +517,11 @@ __global__ void __launch_bounds__(kThreads, KIND == kLinear ? CC_RING_MIN_BLOCKS
   using A = typename Tr<IN>::Acc;
   const int n = P.nranks;
   const int mode = P.mode;
-  const uint64_t ntiles = (P.hi - P.lo + P.tile - 1) / P.tile;
+  const uint64_t ntiles = (P.hi - P.lo + P.skew + P.tile - 1) / P.tile;
   auto src = [&](int r) { return static_cast<const In*>(P.src[r]); };
   for (uint64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    const uint64_t ea = P.lo + tile * P.tile, eb = min(ea + P.tile, P.hi);
+    const uint64_t ea = tile == 0 ? P.lo : P.lo + tile * P.tile - P.skew;
+    const uint64_t eb = min(P.lo + (tile + 1) * P.tile - P.skew, P.hi);
     uint64_t s = ea;
     while (s < eb) {
       uint64_t ga, gb;
@@ -610,7 +613,12 @@ static cudaError_t run_reduce(ReduceParams& P, cudaStream_t s) {
   const uint64_t units = (P.hi - P.lo + UE - 1) / UE;
   const uint64_t upt = std::max<uint64_t>(1, std::min<uint64_t>(target, units / (resident * kThreads)));
   P.tile = std::max<uint64_t>(8, std::min<uint64_t>(upt * kThreads * UE, per_group));
-  const uint64_t ntiles = (P.hi - P.lo + P.tile - 1) / P.tile;
+  // tiles after the first start on a 128-byte line of the first source (and of the others
+  // that share its offset modulo 128 bytes), so that each warp's 512 bytes per buffer fill four
+  // whole lines when the buffers sit off a line; aligned buffers keep skew 0
+  constexpr uint64_t L = 128 / sizeof(typename Tr<IN>::In);
+  P.skew = (P.vec && P.tile % L == 0) ? (P.lo + P.lshift) % L : 0;
+  const uint64_t ntiles = (P.hi - P.lo + P.skew + P.tile - 1) / P.tile;
   const uint64_t grid = std::max<uint64_t>(1, std::min<uint64_t>(ntiles, CC_REDUCE_OVERSUB * resident));
   k<<<(unsigned)grid, kThreads, 0, s>>>(P);
   return cudaGetLastError();
