@@ -7,7 +7,7 @@ import pytest
 import synth
 from oracle import collectives as C
 
-from .helpers import bits, misaligned, to_dev, to_host
+from .helpers import Guarded, bits, misaligned, to_dev, to_host
 
 pytestmark = pytest.mark.gpu
 
@@ -107,3 +107,57 @@ def test_reduce_scatter_reduce_allgather_random_shapes(seed):
         torch.cuda.synchronize()
         for r in range(n):
             assert np.array_equal(bits(to_host(full[r])), bits(want_ar[r])), f"AG(RS) {kind} {op} N={n}"
+
+
+def _at(x: np.ndarray, elems: int):
+    """A CUDA tensor holding `x`, `elems` elements past a 16-byte boundary."""
+    return to_dev(np.concatenate([np.zeros(elems, x.dtype), x]))[elems:]
+
+
+@pytest.mark.parametrize("seed", range(40, 64))
+def test_random_offsets_for_sources_and_outputs(seed):
+    """Sources at one common or at per-rank random offsets from a 16-byte boundary, outputs at
+    another (the element-store, realigned-copy and element paths, and line-skewed tiles over
+    several hundred tiles), guard bands around every output: allreduce (ring, tree), reduce-
+    scatter, reduce and allgather, bit for bit against the oracle."""
+    n, count, kind, op, _, s = _case(seed)
+    rng = np.random.default_rng(seed + 1000)
+    if seed % 3 == 0:  # hundreds of tiles
+        count = int(rng.integers(1 << 20, 3 << 20)) if n <= 16 else int(rng.integers(1 << 16, 1 << 18))
+    xs = _inputs(kind, n, count, s, op)
+    ind = {"f32": "f32", "i32": "i32", "bf16": "bf16"}[kind]
+    common = bool(rng.integers(0, 2))
+    so = [int(rng.integers(0, 4))] * n if common else [int(x) for x in rng.integers(0, 4, n)]
+    do = int(rng.integers(0, 4))
+    send = [_at(x, o) for x, o in zip(xs, so)]
+    od = torch.int32 if kind == "i32" else torch.float32
+    scale = 1.0 if kind == "i32" or op != "sum" else 0.5
+    for algo, fn in (("ring", C.ring_allreduce), ("tree", C.tree_allreduce)):
+        want, _ = fn(xs, op=op, in_dtype=ind, scale=scale)
+        out = [Guarded(count, od, misalign=do) for _ in range(n)]
+        cc.cc_allreduce(send, [g.t for g in out], op=op, algo=algo, scale=scale)
+        torch.cuda.synchronize()
+        for r in range(n):
+            assert np.array_equal(bits(to_host(out[r].t)), bits(want[r])), f"{algo} {kind} {op} N={n} {so}/{do}"
+            out[r].check()
+    want, _ = C.ring_reduce_scatter(xs, op=op, in_dtype=ind)
+    shards = [Guarded(cc.cc_chunk(count, n, c)[1], od, misalign=(do + c) % 4) for c in range(n)]
+    cc.cc_reduce_scatter(send, [g.t for g in shards], op=op)
+    root = s % n
+    want_red, _ = C.reduce(xs, root, op=op, in_dtype=ind)
+    red = Guarded(count, od, misalign=do)
+    cc.cc_reduce(send, red.t, root, op=op)
+    torch.cuda.synchronize()
+    for c in range(n):
+        assert np.array_equal(bits(to_host(shards[c].t)), bits(want[c])), f"RS {kind} {op} N={n} {so}/{do} c={c}"
+        shards[c].check()
+    assert np.array_equal(bits(to_host(red.t)), bits(want_red)), f"reduce {kind} {op} N={n} {so}/{do}"
+    red.check()
+    if kind != "bf16":  # allgather of the shards (each at its own offset) into outputs at `do`
+        full = [Guarded(count, od, misalign=do) for _ in range(n)]
+        cc.cc_allgather([g.t for g in shards], [g.t for g in full])
+        want_ar, _ = C.ring_allreduce(xs, op=op, in_dtype=ind)
+        torch.cuda.synchronize()
+        for r in range(n):
+            assert np.array_equal(bits(to_host(full[r].t)), bits(want_ar[r])), f"AG {kind} {op} N={n} {so}/{do}"
+            full[r].check()
