@@ -306,7 +306,7 @@ def roofline_fields(achieved, peak, peak_kind):
     """The fraction against the measured copy rate (a torch copy_, not a hard ceiling: a
     read-heavy kernel can pass it) and against the nominal 8 TB/s, side by side."""
     return {"achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-            "peak_kind": peak_kind, "frac_of_nominal_8TBps": achieved / NOMINAL_HBM_GBS}
+            "peak_kind": peak_kind, "frac_of_nominal_8TBps": achieved / NOMINAL_HBM_GBS, "bound": "hbm"}
 
 
 def timed_row(torch, call, iters, nbytes, launches_per_call, *, flush=None, warmup=3, local=0, **extra):
@@ -371,6 +371,7 @@ def rows_config1(torch, cc, local, with_cpu=True):
         for name, (nbytes, make) in calls.items():
             rows[name] = timed_row(torch, make(st), 200, nbytes, 1, flush=flush, local=local)
             rows[name]["device_us"] = _us(graph_time_ms(torch, make))
+            rows[name]["roofline"]["bound"] = "latency"  # a few microseconds per call, not bytes
     for r in rows.values():
         r["us"] = r["ms"] * 1e3
     out = {"workload": "config 1: N=4 simulated ranks x 4096 elements, fp32 U[-1,1] and int32 U[-1000,1000] "
@@ -484,6 +485,8 @@ def rows_config4(torch, cc, gen, local, iters, with_cpu=True):
                                       kernel="alltoallv dispatch row copy over a plan"),
             "combine_run": timed_row(torch, comb_run, iters, b_c, 1, local=local,
                                      kernel="alltoallv combine row copy over a plan")}
+    for k in ("route_topk", "plan"):  # microseconds of dependent steps, not bytes
+        rows[k]["roofline"]["bound"] = "latency"
     ms = sum(rows[k]["ms"] for k in ("route_topk", "dispatch", "combine"))
     ms_plan = sum(rows[k]["ms"] for k in ("route_topk", "plan", "dispatch_run", "combine_run"))
     out = {"workload": "config 4 (MoE): N=8 simulated ranks, 8192 tokens x 4096 bf16 per rank, 64 experts (8 per "
@@ -657,6 +660,8 @@ def rows_config5(torch, cc, gen, local, with_cpu=True):
                               own_traffic_bytes=stepped_traffic(n, count, 4, algo))
                 r["own_traffic_GBps"] = r["own_traffic_bytes"] / (r["ms"] * 1e-3) / 1e9
                 r["own_traffic_frac"] = r["own_traffic_GBps"] / measured_peak()[0]
+                if small:  # 2(N-1) or 2 depth dependent steps of a few KiB each
+                    r["roofline"]["bound"] = "latency"
                 t = r["ms"] * 1e-3
                 if small:
                     r["device_us"] = _us(graph_time_ms(torch, make))
