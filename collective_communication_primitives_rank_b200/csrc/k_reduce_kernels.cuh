@@ -481,7 +481,7 @@ struct ReduceParams {
   FoldProgram prog;
   uint64_t count;
   uint64_t lo, hi;       // the elements this launch folds: [lo, hi) of the count
-  uint64_t tile;         // elements per tile (a multiple of 8)
+  uint64_t tile;         // elements per tile (a multiple of 8, or one fold group of fewer than 8)
   uint64_t skew;         // tile k >= 1 starts at lo + k * tile - skew (the first tile is that much shorter)
   uint64_t lshift;       // elements the first source sits past a 128-byte line (16-byte units only)
   uint64_t shift;        // elements every source (and allreduce / root output) sits past a 16-byte boundary
@@ -598,7 +598,10 @@ static cudaError_t run_reduce(ReduceParams& P, cudaStream_t s) {
                            : P.fold == kFoldTree ? 2
                            : P.fold == kFoldHier ? (uint64_t)P.nranks
                            : P.fold == kFoldMultiRing ? (uint64_t)P.nranks * P.per_node : 1;
-  const uint64_t per_group = ((P.count + ngroups - 1) / ngroups + 7) / 8 * 8;
+  // (groups of fewer than 8 elements keep their own size: a tile that spans several of them
+  // folds them one after another, each a dependent round trip)
+  const uint64_t gsz = (P.count + ngroups - 1) / ngroups;
+  const uint64_t per_group = gsz < 8 ? gsz : (gsz + 7) / 8 * 8;
   // units per thread and tile (measured): the linear folds (ring, linear tree, hierarchical)
   // run best with about 24 memory operations per thread and CTA (a unit costs N loads plus
   // N stores for allreduce, one store otherwise), the small-stack tree machines with 16 / N
@@ -612,7 +615,7 @@ static cudaError_t run_reduce(ReduceParams& P, cudaStream_t s) {
                           : (uint64_t)std::max(1, std::min(8, 16 / P.nranks));
   const uint64_t units = (P.hi - P.lo + UE - 1) / UE;
   const uint64_t upt = std::max<uint64_t>(1, std::min<uint64_t>(target, units / (resident * kThreads)));
-  P.tile = std::max<uint64_t>(8, std::min<uint64_t>(upt * kThreads * UE, per_group));
+  P.tile = std::max<uint64_t>(1, std::min<uint64_t>(upt * kThreads * UE, per_group));
   // tiles after the first start on a 128-byte line of the first source (and of the others
   // that share its offset modulo 128 bytes), so that each warp's 512 bytes per buffer fill four
   // whole lines when the buffers sit off a line; aligned buffers keep skew 0
