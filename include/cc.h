@@ -34,8 +34,12 @@
  *     They return after enqueuing; only argument and launch errors are reported
  *     synchronously. A failed launch leaves the outputs undefined.
  *   - count == 0 is a no-op returning CC_OK.
- *   - 16-byte aligned buffers take the 128-bit path; any other alignment of 4-byte
- *     (2-byte for bf16) elements takes an element-wise path with the same results.
+ *   - Any alignment of 4-byte (2-byte for bf16) elements is accepted, with the same results
+ *     on every path. 16-byte aligned buffers take 128-bit loads and stores; buffers that all
+ *     sit the same whole number of elements past a 16-byte boundary take them after a short
+ *     element-wise head; fp32 / int32 sums whose outputs sit at another offset than their
+ *     sources take 128-bit loads and element stores; copies whose destinations share an
+ *     offset that the source does not take 128-bit stores; everything else is element-wise.
  *   - In-place (recv[r] == send[r]) is allowed where stated; any other overlap between
  *     inputs and outputs is undefined.
  *   - Allowed (in, out) dtype pairs for reductions: (F32, F32), (BF16, F32), (I32, I32).
