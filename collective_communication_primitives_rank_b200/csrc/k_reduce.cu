@@ -303,6 +303,18 @@ static cudaError_t dispatch_scalar_out(ReduceParams& P, int kind, cudaStream_t s
   return cudaErrorInvalidValue;
 }
 
+// Linear folds over buffers without 16-byte units: the element-path kernel.
+template <int IN>
+static cudaError_t dispatch_elements(ReduceParams& P, cc_op op, cudaStream_t s) {
+  switch (op) {
+    case CC_SUM: return run_reduce<IN, CC_SUM, kLinear, false, true>(P, s);
+    case CC_MAX: return run_reduce<IN, CC_MAX, kLinear, false, true>(P, s);
+    case CC_MIN: return run_reduce<IN, CC_MIN, kLinear, false, true>(P, s);
+    case CC_PROD: return run_reduce<IN, CC_PROD, kLinear, false, true>(P, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
 template <int IN>
 static cudaError_t dispatch_op(ReduceParams& P, cc_op op, int kind, cudaStream_t s) {
 #define CC_KINDS(OPV)                                                                         \
@@ -397,6 +409,16 @@ cudaError_t launch_reduce(const void* const* send, void* const* dst, int ndst, i
   // N = 2 × 256 MiB: ring 5667 -> 6663 GB/s, reduce-scatter 5399 -> 6832; at N = 3..4 the
   // one-unit fold with 4 resident CTAs is faster)
   if (kind == kLinear && nranks == 2) kind = kLinSmall;
+  // linear folds with no 16-byte units take the element-path kernel (several elements per
+  // thread in flight)
+  if (!vec && (kind == kLinear || kind == kLinSmall)) {
+    switch (in_t) {
+      case CC_F32: return dispatch_elements<CC_F32>(P, op, stream);
+      case CC_BF16: return dispatch_elements<CC_BF16>(P, op, stream);
+      case CC_I32: return dispatch_elements<CC_I32>(P, op, stream);
+    }
+    return cudaErrorInvalidValue;
+  }
   // element stores: the runtime folds and the trees compiled for 8 and 16 ranks (binomial
   // programs run on the fold machine)
   if (scalar_out) {

@@ -331,7 +331,7 @@ constexpr int kTree8 = 20, kTree16 = 21;
 __host__ __device__ constexpr bool is_tree_ct(int kind) { return kind == kTree8 || kind == kTree16; }
 __host__ __device__ constexpr int tree_ct_ranks(int kind) { return kind == kTree8 ? 8 : 16; }
 
-template <int IN, int OP, int KIND, typename RankOf, typename Src, typename EmitU, typename EmitE>
+template <int IN, int OP, int KIND, bool EL = false, typename RankOf, typename Src, typename EmitU, typename EmitE>
 __device__ __forceinline__ void reduce_range(int n, int g, RankOf rank_of, const FoldProgram& prog,
                                              uint64_t a, uint64_t b, uint64_t t, uint64_t T, bool vec,
                                              Src src, EmitU emit_unit, EmitE emit_elem, uint4* stk,
@@ -358,7 +358,44 @@ __device__ __forceinline__ void reduce_range(int n, int g, RankOf rank_of, const
       return machine_fold<IN, OP, A, A, 8>(n, prog, rank_of, ld, same, st);
     }
   };
-  if (vec) {
+  if constexpr (EL) {
+    // element-path kernel (no 16-byte units: sources at unequal offsets, bf16 off a boundary,
+    // or other folds over unequally placed buffers): a linear fold keeps NE elements per thread
+    // (T apart) in flight, each window of W ranks loaded for all of them before it is folded
+    // in, in the same order per element as ring_fold
+    static_assert(RING, "the element-path kernel takes the linear folds");
+    constexpr int NE = 4, W = 4;
+    for (uint64_t e0 = a + t; e0 < b; e0 += NE * T) {
+      A acc[NE];
+      int r = start;
+#pragma unroll
+      for (int q = 0; q < NE; ++q)
+        if (e0 + q * T < b) acc[q] = load_elem<IN>(src(r) + e0 + q * T);
+      for (int j0 = 1; j0 < n; j0 += W) {
+        A x[W][NE];
+#pragma unroll
+        for (int k = 0; k < W; ++k) {
+          const int rk = up ? (r + 1 + k) % n : ((r - 1 - k) % n + n) % n;
+          if (j0 + k < n) {
+#pragma unroll
+            for (int q = 0; q < NE; ++q)
+              if (e0 + q * T < b) x[k][q] = load_elem<IN>(src(rk) + e0 + q * T);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < W; ++k)
+          if (j0 + k < n) {
+#pragma unroll
+            for (int q = 0; q < NE; ++q)
+              if (e0 + q * T < b) acc[q] = op<IN, OP, A>(acc[q], x[k][q]);
+          }
+        r = up ? (r + W) % n : ((r - W) % n + n) % n;
+      }
+#pragma unroll
+      for (int q = 0; q < NE; ++q)
+        if (e0 + q * T < b) emit_elem(e0 + q * T, acc[q]);
+    }
+  } else if (vec) {
     // 16-byte units start where (e + shift) is a multiple of UE: every buffer sits `shift`
     // elements past a 16-byte boundary (0 when aligned)
     uint64_t va = a + (UE - (a + shift) % UE) % UE;
@@ -501,7 +538,7 @@ struct ReduceParams {
 // SS: the units follow the sources and the allreduce / root outputs, which sit at another
 // offset from a 16-byte boundary, take four element stores per unit (fp32 / int32), as
 // reduce-scatter shards that the units meet off a boundary always do.
-template <int IN, int OP, int KIND, bool SS = false>
+template <int IN, int OP, int KIND, bool SS = false, bool EL = false>
 __global__ void __launch_bounds__(kThreads, KIND == kLinear ? CC_RING_MIN_BLOCKS
                                            : KIND == kLinSmall ? CC_LINSMALL_MIN_BLOCKS
                                            : is_binom_ct(KIND) ? (binom_ct_units(KIND) > 1 ? 2 : KIND == kBinom64 ? 3 : 4)
@@ -572,7 +609,7 @@ __global__ void __launch_bounds__(kThreads, KIND == kLinear ? CC_RING_MIN_BLOCKS
                          : P.fold == kFoldMultiRing ? g % n
                          : P.fold == kFoldTree ? (g == 0 ? 0 : n - 1) : P.prog.rmap[0];
       const bool lup = P.fold == kFoldMultiRing ? ((g / n) % 2 == 0) : (P.fold != kFoldTree || g == 0);
-      reduce_range<IN, OP, KIND>(n, g, rank_of, P.prog, s, se, threadIdx.x, blockDim.x, P.vec != 0, src,
+      reduce_range<IN, OP, KIND, EL>(n, g, rank_of, P.prog, s, se, threadIdx.x, blockDim.x, P.vec != 0, src,
                                     emit_unit, emit_elem, s_stk + threadIdx.x, lstart, lup, G, hc, hj, P.shift);
       s = se;
     }
@@ -586,9 +623,9 @@ static int blocks_per_sm(K kernel) {
   return b;
 }
 
-template <int IN, int OP, int KIND, bool SS = false>
+template <int IN, int OP, int KIND, bool SS = false, bool EL = false>
 static cudaError_t run_reduce(ReduceParams& P, cudaStream_t s) {
-  auto k = reduce_kernel<IN, OP, KIND, SS>;
+  auto k = reduce_kernel<IN, OP, KIND, SS, EL>;
   static const int bps = blocks_per_sm(k);
   constexpr uint64_t UE = Tr<IN>::UE;
   const uint64_t resident = (uint64_t)sm_count() * bps;
