@@ -222,6 +222,33 @@ def test_sums_with_sources_and_outputs_at_different_offsets(n, kind, offs, sd):
         mx[r].check()
 
 
+@pytest.mark.parametrize("n", [2, 5, 8])
+@pytest.mark.parametrize("op", ["sum", "max"])
+@pytest.mark.parametrize("kind", ["spread", "i32", "bf16"])
+def test_in_place_with_per_rank_offsets(n, op, kind):
+    """In-place allreduce (ring, tree, multi-ring) over buffers that sit at different offsets per
+    rank (rank r: r mod 4 elements past a 16-byte boundary): the element paths, each element's
+    column read and written by one thread. bf16 inputs are not in place (fp32 outputs)."""
+    count = n * 5_003 + 1
+    xs = _inputs(kind, n, count, seed=34)
+    scale = 1.0 if kind == "i32" or op != "sum" else 0.25
+    for algo, fn in (("ring", C.ring_allreduce), ("tree", C.tree_allreduce),
+                     ("multiring", lambda v, **kw: C.multiring_allreduce(v, 3, **kw))):
+        want, _ = fn(xs, op=op, in_dtype=_IN[kind], scale=scale)
+        if kind == "bf16":
+            bufs = [_shifted(x, r % 4) for r, x in enumerate(xs)]
+            outs = [_shifted(np.zeros(count, np.float32), (r + 1) % 4) for r in range(n)]
+        else:
+            bufs = outs = [_shifted(x, r % 4) for r, x in enumerate(xs)]
+        if algo == "multiring":
+            cc.cc_allreduce_multiring(bufs, outs, 3, op=op, scale=scale)
+        else:
+            cc.cc_allreduce(bufs, outs, op=op, algo=algo, scale=scale)
+        torch.cuda.synchronize()
+        for r in range(n):
+            _assert_same(to_host(outs[r]), want[r], f"in place {algo} {kind} {op} N={n} rank {r}")
+
+
 def test_allreduce_empty_is_a_no_op():
     t = [torch.empty(0, device="cuda") for _ in range(4)]
     cc.cc_allreduce(t, t)
