@@ -162,3 +162,42 @@ def test_config5_sweep_large_points_sampled(n, mib, algo):
         assert np.array_equal(bits(_gather(out[r], pos)), bits(want[r]))
     for r in range(1, n):
         assert torch.equal(out[r], out[0])
+
+
+@pytest.mark.parametrize("so,do", [(1, 1), (1, 0), (0, 3)])
+@pytest.mark.parametrize("algo", ["ring", "tree"])
+def test_large_allreduce_and_reduce_scatter_off_a_boundary_sampled(so, do, algo):
+    """N = 8 x 128 MiB with every source `so` and every output `do` elements past a 16-byte
+    boundary (tens of thousands of line-skewed tiles; element stores where the offsets differ),
+    sampled at every chunk edge and at random positions against the oracle."""
+    n, count = 8, 32 * 1024 * 1024
+    bounds = L.chunk_bounds(count, n) if algo == "ring" else [(0, (count + 1) // 2), ((count + 1) // 2, count)]
+    pos = _positions(count, bounds, np.random.default_rng(so * 4 + do))
+    # every element within 40 of a tile edge (tiles of 1024 elements, skewed onto lines) at
+    # a few hundred places
+    near = (np.arange(1024, count, 1024 * 97)[:, None] + np.arange(-40, 41)[None, :]).ravel()
+    pos = np.unique(np.concatenate([pos, near[(near >= 0) & (near < count)]]))
+    dev, samp = [], []
+    for r in range(n):
+        h = synth.uniform_f32(SEED + 9, r, count)
+        samp.append(h[pos].copy())
+        full = torch.empty(count + 4, device="cuda")
+        full[so:so + count].copy_(torch.from_numpy(h))
+        dev.append(full[so:so + count])
+        del h
+    out = [torch.empty(count + 4, device="cuda")[do:do + count] for _ in range(n)]
+    cc.cc_allreduce(dev, out, algo=algo, scale=0.125)
+    torch.cuda.synchronize()
+    fn = C.ring_allreduce if algo == "ring" else C.tree_allreduce
+    want, _ = fn(samp, count=count, positions=pos, scale=0.125)
+    for r in (0, n - 1):
+        assert np.array_equal(bits(_gather(out[r], pos)), bits(want[r])), f"{algo} {so}/{do} rank {r}"
+    if algo == "ring":
+        shards = [torch.empty(b - a + 4, device="cuda")[do:do + b - a] for a, b in L.chunk_bounds(count, n)]
+        cc.cc_reduce_scatter(dev, shards, scale=0.125)
+        torch.cuda.synchronize()
+        want_rs, _ = C.ring_reduce_scatter(samp, count=count, positions=pos, scale=0.125)
+        for c, (a, b) in enumerate(L.chunk_bounds(count, n)):
+            inside = (pos >= a) & (pos < b)
+            assert np.array_equal(bits(_gather(shards[c], pos[inside] - a)), bits(want_rs[c])), \
+                f"reduce-scatter {so}/{do} shard {c}"
